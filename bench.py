@@ -1,0 +1,405 @@
+"""Throughput of the DeepSeekMoE layer forward on B200, one JSON line.
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl reference]
+
+Default workload: the DeepSeek-V3-shaped prefill layer (T=8192, d=7168, 256 routed
++ 1 shared SwiGLU experts of d_ff=2048, sigmoid scores with a selection-only bias,
+top-8 renormalised), synthetic seeded inputs and random weights of that shape.
+
+A step is one whole layer forward (router, scores, top-k, gates, balance
+statistics, permutation, gate/up and down grouped GEMMs, combine) over one batch of
+T tokens already resident in HBM; with N GPUs every rank runs its own batch of T
+tokens (weak scaling) and the balance statistics are all-reduced across ranks each
+step. Timing: W untimed steps, then K steps between barrier + synchronize, CUDA
+events on the launching stream, max over ranks. The 22.6 GB of expert weights a
+step streams are far larger than L2, so no flush is needed between steps.
+
+Reported alongside: the dominant kernel's roofline (mean in-region duration from
+per-stage CUDA events), the same metric end to end through dsmoe_forward_host with
+pinned host buffers (copies inside the timed region), the oracle timed on the
+host's cores over a bounded sample, SM clocks sampled during the timed region, and
+the number of kernel launches.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "DeepSeekMoE layer fwd tokens/s; achieved TFLOP/s (% bf16 peak) / GB/s on 1 B200"
+SCORE_NAMES = {0: "softmax", 1: "sigmoid", 2: "sqrt_softplus", 3: "hash"}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="v3_prefill")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=None, help="steps of the end-to-end leg (default: --steps)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample", type=int, default=None, help="tokens in the oracle's timed sample")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def config_block(cfg, n_gpus):
+    return {"workload": cfg.name, "T_per_gpu": cfg.T, "global_batch": cfg.T * n_gpus, "d_model": cfg.d_model,
+            "n_routed": cfg.n_routed, "top_k": cfg.top_k, "d_ff": cfg.d_ff, "n_shared": cfg.n_shared,
+            "d_ff_shared": cfg.d_ff_shared, "score": SCORE_NAMES[cfg.score], "renormalize": cfg.renormalize,
+            "parallelism": f"dp{n_gpus} (token shards, full weight replica per GPU)",
+            "l2": f"no flush: inputs larger than L2 ({(cfg.routed_weight_bytes() + cfg.shared_weight_bytes()) / 1e9:.1f}"
+                  " GB of expert weights streamed per step vs 126 MB L2)"}
+
+
+# ----------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ----------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                p = [c.strip() for c in line.split(",")]
+                if len(p) >= 9:
+                    rows.append(p)
+        os.unlink(self.path)
+        if not rows:
+            return None
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return float("nan")
+
+        sm = [num(r[1]) for r in rows]
+        smax = max(num(r[2]) for r in rows)
+        loaded = [v for v, r in zip(sm, rows) if num(r[3]) > 200.0] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        loaded.sort()
+        return {"sm_mhz": loaded[len(loaded) // 2], "sm_max_mhz": smax, "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------------------
+# CPU oracle leg (bounded sample)
+# ----------------------------------------------------------------------------------------
+def default_cpu_sample(cfg):
+    return 512 if cfg.d_model <= 1024 and cfg.T <= 4096 else (64 if cfg.d_model <= 2048 else 8)
+
+
+def cpu_oracle_throughput(cfg, x_cpu, b_cpu, W_router_cpu, token_ids_cpu, expert_source, n_tokens, seed=0):
+    """Time the oracle, as it stands, on a sample of n_tokens tokens of the workload (their
+    own batch: router, scores, top-k, statistics, experts, combine). Expert weights are
+    fetched to host memory before the clock starts. Returns (tokens/s, seconds, threads)."""
+    import numpy as np
+    from oracle import dsmoe_oracle as O
+    T = x_cpu.shape[0]
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(T, size=min(n_tokens, T), replace=False))
+    inp = {"x": x_cpu[rows], "W_router": W_router_cpu, "b": b_cpu,
+           "token_ids": None if token_ids_cpu is None else token_ids_cpu[rows]}
+    r = O.route(cfg, inp)
+    need = sorted(set(np.asarray(r["idx"]).ravel().tolist()))
+    cache = {}
+    for e in need:
+        cache[e] = expert_source(e)
+    shared = [expert_source(("s", s)) for s in range(cfg.n_shared)]
+
+    class _Routed(dict):
+        pass
+
+    inp_w = dict(inp)
+    inp_w["W_gate"] = {e: cache[e][0] for e in need}
+    inp_w["W_up"] = {e: cache[e][1] for e in need}
+    inp_w["W_down"] = {e: cache[e][2] for e in need}
+    inp_w["Ws_gate"] = [s[0] for s in shared]
+    inp_w["Ws_up"] = [s[1] for s in shared]
+    inp_w["Ws_down"] = [s[2] for s in shared]
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    O.forward(cfg, inp_w)
+    dt = time.perf_counter() - t0
+    return len(rows) / dt, dt, threads, len(rows)
+
+
+# ----------------------------------------------------------------------------------------
+# reference arm: the oracle on the host's cores
+# ----------------------------------------------------------------------------------------
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+    import torch
+    import workloads as W
+    inp = W.make_inputs(cfg, seed=0, device="cpu", with_weights=False)
+    n = args.cpu_sample or max(1, default_cpu_sample(cfg) // 4)
+
+    def src(key):
+        if isinstance(key, tuple):
+            return tuple(W.expert_matrix(cfg, w, key[1], 0, "cpu") for w in ("Ws_gate", "Ws_up", "Ws_down"))
+        return tuple(W.expert_matrix(cfg, w, key, 0, "cpu") for w in ("W_gate", "W_up", "W_down"))
+
+    times, toks = [], 0
+    threads = 1
+    for step in range(args.warmup + args.steps):
+        tps, dt, threads, m = cpu_oracle_throughput(cfg, inp["x"], inp["b"], inp["W_router"], inp["token_ids"],
+                                                    src, n, seed=step)
+        if step >= args.warmup:
+            times.append(dt)
+            toks += m
+    value = toks / sum(times)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_block(cfg, 1),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{n} tokens of the workload per step, full layer (float64 oracle)"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------------------
+# native arm
+# ----------------------------------------------------------------------------------------
+def run_native(args, cfg):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import workloads as W
+    import mixture_experts_layer_score_b200 as M
+    from mixture_experts_layer_score_b200.sharded import global_balance_stats
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch N>1 with torch.distributed.run")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", rank=rank, world_size=world, timeout=timedelta(seconds=300),
+                                device_id=dev)
+
+    # inputs: every rank holds the same weights and its own batch of T tokens
+    inp = W.make_inputs(cfg, seed=0, device=dev, with_weights=True)
+    if rank > 0:
+        inp["x"] = W.normal_bf16((cfg.T, cfg.d_model), 1.0, 0, "x", rank, dev)
+        if inp["token_ids"] is not None:
+            g = torch.Generator(device=dev)
+            g.manual_seed(W.derive_seed(0, "token_ids", rank))
+            inp["token_ids"] = torch.randint(0, W.TOKEN_VOCAB, (cfg.T,), generator=g, device=dev,
+                                             dtype=torch.int64).to(torch.int32)
+    layer = M.DSMoE(M.cfg_from(cfg, cfg.T), inp, device=local)
+    out = layer.alloc_outputs(cfg.T)
+    T_total = cfg.T * world
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        layer.forward(inp["x"], token_ids=inp["token_ids"], out=out, stream=stream)
+        if world > 1:
+            global_balance_stats(layer.handle, T_total, out["counts"], out["P_sum"], out["f"], out["P"],
+                                 stream=stream)
+
+    for _ in range(max(args.warmup, 3 if args.warmup >= 3 else args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    st = M.dsmoe_get_status(layer.handle)
+    if st != M.DSMOE_OK:
+        raise SystemExit(f"device status after warm-up: {M.dsmoe_last_error()}")
+
+    # ---- timed region (device)
+    M.dsmoe_set_timing(layer.handle, True)
+    launches0 = M.dsmoe_launch_count(layer.handle)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    clock_info = clocks.stop()
+    launches = M.dsmoe_launch_count(layer.handle) - launches0
+    stage_ms = M.dsmoe_stage_times(layer.handle)
+    M.dsmoe_set_timing(layer.handle, False)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    st = M.dsmoe_get_status(layer.handle)
+    if st != M.DSMOE_OK:
+        raise SystemExit(f"device status after the timed region: {M.dsmoe_last_error()}")
+    ms_per_step = ms / args.steps
+    value = T_total / (ms_per_step / 1e3)
+
+    # ---- roofline of the dominant kernel
+    peaks, peak_src = load_peaks()
+    S = cfg.T * cfg.top_k
+    flops = {
+        "gemm_gate_up": 2.0 * 2 * cfg.d_model * (S * cfg.d_ff + cfg.T * cfg.n_shared * cfg.d_ff_shared),
+        "gemm_down": 2.0 * cfg.d_model * (S * cfg.d_ff + cfg.T * cfg.n_shared * cfg.d_ff_shared),
+    }
+    dom = max(flops, key=lambda k: stage_ms.get(k, 0.0))
+    counts = out["counts"].cpu().numpy()
+    touched = int((counts > 0).sum())
+    weight_bytes = {"gemm_gate_up": 2 * cfg.d_model * (touched * 2 * cfg.d_ff + cfg.n_shared * 2 * cfg.d_ff_shared),
+                    "gemm_down": 2 * cfg.d_model * (touched * cfg.d_ff + cfg.n_shared * cfg.d_ff_shared)}
+    dom_ms = stage_ms[dom]
+    intensity = flops[dom] / max(weight_bytes[dom], 1)
+    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if intensity >= ridge:
+        achieved = flops[dom] / (dom_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak}
+    else:
+        achieved = weight_bytes[dom] / (dom_ms / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak}
+    roof.update({"kernel": dom, "kernel_ms": dom_ms, "traffic": None,
+                 "peak_source": f"{peak_src} ({'bf16_tflops_sustained' if roof['bound'] == 'tensor' else 'hbm_gbs'})",
+                 "algorithmic": {"flops": flops[dom], "weight_bytes": weight_bytes[dom]}})
+    layer_flops = cfg.flops_per_token() * cfg.T
+    layer_tflops = layer_flops / (ms_per_step / 1e3) / 1e12
+
+    # ---- end to end through the C ABI with host buffers
+    e2e_steps = args.e2e_steps or args.steps
+    T, K, N, d = cfg.T, cfg.top_k, cfg.n_routed, cfg.d_model
+    xh = inp["x"].cpu().pin_memory()
+    idh = None if inp["token_ids"] is None else inp["token_ids"].cpu().pin_memory()
+    hh = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
+    th = torch.empty((T, K), dtype=torch.int32).pin_memory()
+    gh = torch.empty((T, K), dtype=torch.float32).pin_memory()
+    ch = torch.empty((N,), dtype=torch.int32).pin_memory()
+    fh = torch.empty((N,), dtype=torch.float32).pin_memory()
+    ph = torch.empty((N,), dtype=torch.float32).pin_memory()
+    w = inp
+
+    def e2e_step():
+        M.dsmoe_forward_host(layer.handle, T, xh, idh, w.get("W_router"), w.get("b"), w["W_gate"], w["W_up"],
+                             w["W_down"], w.get("Ws_gate"), w.get("Ws_up"), w.get("Ws_down"), hh, th, gh, ch, fh,
+                             ph, stream)
+
+    for _ in range(2):
+        e2e_step()
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = xh.numel() * 2 + (0 if idh is None else idh.numel() * 4)
+    d2h = hh.numel() * 2 + th.numel() * 4 + gh.numel() * 4 + 3 * N * 4
+    e2e = {"value": T_total / (e2e_ms / e2e_steps / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h}
+
+    # ---- CPU oracle baseline (rank 0, N=1 only)
+    cpu_base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n = args.cpu_sample or default_cpu_sample(cfg)
+
+        def src(key):
+            if isinstance(key, tuple):
+                s = key[1]
+                return (inp["Ws_gate"][s].cpu(), inp["Ws_up"][s].cpu(), inp["Ws_down"][s].cpu())
+            return (inp["W_gate"][key].cpu(), inp["W_up"][key].cpu(), inp["W_down"][key].cpu())
+
+        tps, dt, threads, m = cpu_oracle_throughput(
+            cfg, inp["x"].cpu(), None if inp["b"] is None else inp["b"].cpu(),
+            None if inp["W_router"] is None else inp["W_router"].cpu(),
+            None if inp["token_ids"] is None else inp["token_ids"].cpu(), src, n)
+        cpu_base = {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                    "sample": f"{m} tokens of the workload as one batch, full layer, float64 oracle, {dt:.1f} s"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; random weights of the layer's shape)",
+                "config": config_block(cfg, world), "roofline": roof, "cpu_baseline": cpu_base, "e2e": e2e,
+                "gpu_launches": int(launches), "clocks": clock_info,
+                "layer_tflops": layer_tflops, "stage_ms": stage_ms, "experts_touched": touched}
+        print(json.dumps(line), flush=True)
+    layer.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    import workloads as W
+    cfg = W.get_config(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_native(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

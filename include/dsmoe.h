@@ -1,0 +1,225 @@
+/*
+ * dsmoe.h -- C ABI of libdsmoe.so, the forward pass of a DeepSeekMoE layer on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (DeepSeekMoE summary, heloowird.com, shared-expert layer equation):
+ *
+ *     h_t = u_t + sum_{i <= K_s} FFN_i(u_t) + sum_{routed i} g_{i,t} FFN_i(u_t)
+ *
+ * with router affinities l = u . e_i ("MoE architecture: how DeepSeek achieves
+ * more", section 2, G(x) = Softmax(W_g x)), scores s = softmax(l) | sigmoid(l) |
+ * sqrt(softplus(l)) (DeepSeek-V4 book ch. 2, section 2), top-K' selection on
+ * s + b with a selection-only bias (same chapter, section 3), gates g = s or
+ * s / sum_selected s, and SwiGLU experts FFN(u) = W_down (SiLU(W_gate u) * W_up u).
+ * The expert-level balance statistics f_i and P_i (DeepSeekMoE summary,
+ * "Expert-level balance loss") are produced alongside.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensors are row-major and caller-owned. bf16 tensors are passed as
+ *     void* to raw IEEE bfloat16 words. Weights use the nn.Linear layout
+ *     [out_features, in_features] (the reduction dimension is contiguous).
+ *   - Device pointers must be 16-byte aligned; NULL is allowed only where
+ *     stated.
+ *   - No entry point allocates device memory except dsmoe_create, and no
+ *     entry point synchronises the device except where it says so. Work is
+ *     enqueued on the caller's stream (a cudaStream_t passed as void*; NULL is
+ *     the legacy default stream).
+ *   - Errors are returned, never raised: no exit, abort or trap. A kernel that
+ *     gives up a bounded wait records DSMOE_ERR_DEVICE_TIMEOUT in a device
+ *     status word that dsmoe_get_status() reports.
+ *   - A handle may be used by one host thread at a time.
+ */
+#ifndef DSMOE_H
+#define DSMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DSMOE_ABI_VERSION 1
+
+typedef enum dsmoe_status {
+  DSMOE_OK = 0,
+  DSMOE_ERR_INVALID_ARG = 1,    /* bad pointer, size or enum value                     */
+  DSMOE_ERR_UNSUPPORTED = 2,    /* valid request outside what the kernels implement    */
+  DSMOE_ERR_WORKSPACE = 3,      /* T above the handle's max_tokens, or allocation fail */
+  DSMOE_ERR_CUDA = 4,           /* a CUDA runtime call failed (see dsmoe_last_error)   */
+  DSMOE_ERR_DEVICE_TIMEOUT = 5  /* a kernel gave up a bounded wait                     */
+} dsmoe_status;
+
+/* Score function (DeepSeek-V4 book ch. 2, sections 2 and 5). */
+typedef enum dsmoe_score {
+  DSMOE_SCORE_SOFTMAX = 0,        /* s = softmax over the routed experts            */
+  DSMOE_SCORE_SIGMOID = 1,        /* s = 1 / (1 + exp(-l))                          */
+  DSMOE_SCORE_SQRT_SOFTPLUS = 2,  /* s = sqrt(log(1 + exp(l)))                      */
+  DSMOE_ROUTE_HASH = 3            /* expert = token_id * hash_mult mod hash_mod, g=1 */
+} dsmoe_score;
+
+/* Where the per-expert bias b enters. */
+typedef enum dsmoe_bias_mode {
+  DSMOE_BIAS_NONE = 0,
+  DSMOE_BIAS_SELECT_ONLY = 1,  /* key s~ = s + b decides the top-K'; gates and P use s
+                                  (V4 book ch. 2 section 3; "MoE: sparse activation",
+                                  load-balancing section)                                 */
+  DSMOE_BIAS_IN_LOGITS = 2     /* l + b is scored ("MoE architecture", section 6 form)    */
+} dsmoe_bias_mode;
+
+/* Layer configuration. Field names follow the pages' notation:
+ * d = d_model, N' = n_routed, K' = top_k, F = d_ff, K_s = n_shared, F_s = d_ff_shared. */
+typedef struct dsmoe_cfg {
+  int32_t d_model;      /* d, multiple of 64, >= 64                                  */
+  int32_t n_routed;     /* N', 1..512                                                */
+  int32_t top_k;        /* K', 1..16 and <= N' (1 for hash routing)                  */
+  int32_t d_ff;         /* F, multiple of 64                                         */
+  int32_t n_shared;     /* K_s, 0..8                                                 */
+  int32_t d_ff_shared;  /* F_s, multiple of 64 when K_s > 0                          */
+  int32_t score;        /* dsmoe_score                                               */
+  int32_t bias_mode;    /* dsmoe_bias_mode                                           */
+  int32_t renormalize;  /* 0: g = s of the selected experts; 1: g = s / sum_sel s    */
+  int32_t max_tokens;   /* largest T a forward call may pass (sizes the workspace)   */
+  uint32_t hash_mult;   /* hash routing multiplier (2654435761 for the V4 layer)     */
+  uint32_t hash_mod;    /* hash routing modulus, 0 means N'; must be <= N'           */
+} dsmoe_cfg;
+
+typedef struct dsmoe_handle dsmoe_handle;
+
+/* Library ABI version (DSMOE_ABI_VERSION). Host only. */
+int32_t dsmoe_abi_version(void);
+
+/* Human-readable name of a status code. Host only; never NULL. */
+const char* dsmoe_status_string(dsmoe_status s);
+
+/* The message of the last error raised on the calling host thread ("" if none). */
+const char* dsmoe_last_error(void);
+
+/* Validate a configuration without touching a GPU. Host only.
+ * Returns DSMOE_OK, DSMOE_ERR_INVALID_ARG or DSMOE_ERR_UNSUPPORTED. */
+dsmoe_status dsmoe_check_config(const dsmoe_cfg* cfg);
+
+/* Device workspace bytes a handle for cfg allocates. Host only. */
+dsmoe_status dsmoe_workspace_bytes(const dsmoe_cfg* cfg, size_t* bytes);
+
+/* Create a handle on CUDA device `device`: validates cfg, allocates the
+ * workspace (expert-contiguous activations, intermediate activations, routing
+ * tables, statistics partials and the status word) sized for cfg->max_tokens.
+ * The caller's current device is restored before returning. On failure *out is
+ * NULL and nothing stays allocated. */
+dsmoe_status dsmoe_create(const dsmoe_cfg* cfg, int32_t device, dsmoe_handle** out);
+
+/* Release a handle and its workspace (synchronises the handle's device). NULL is a no-op. */
+void dsmoe_destroy(dsmoe_handle* h);
+
+/*
+ * One forward pass of the layer for T tokens (0 <= T <= max_tokens), enqueued
+ * on `stream`. Device pointers, all caller-owned:
+ *
+ *   x          bf16 [T, d]        token activations u_t
+ *   token_ids  int32 [T]          hash routing only (else NULL); values >= 0
+ *   W_router   bf16 [N', d]       expert centroids e_i (NULL for hash routing)
+ *   b          fp32 [N']          per-expert bias (NULL iff bias_mode == NONE)
+ *   W_gate     bf16 [N', F, d]    routed experts, gate projection
+ *   W_up       bf16 [N', F, d]    routed experts, up projection
+ *   W_down     bf16 [N', d, F]    routed experts, down projection
+ *   Ws_gate    bf16 [K_s, F_s, d] shared experts (all three NULL iff K_s == 0)
+ *   Ws_up      bf16 [K_s, F_s, d]
+ *   Ws_down    bf16 [K_s, d, F_s]
+ *
+ * Outputs (device, caller-owned, fully overwritten):
+ *
+ *   h          bf16 [T, d]        layer output, accumulated in fp32, rounded once
+ *   topk_idx   int32 [T, K']      selected experts, by descending selection key,
+ *                                 ties to the lower index
+ *   gates      fp32 [T, K']       g_{i,t} of the selected experts, same order
+ *   counts     int32 [N']         sum_t 1(token t selects expert i)
+ *   f          fp32 [N']          f_i = N' / (K' T) * counts_i
+ *   P          fp32 [N']          P_i = (1/T) sum_t s_{i,t} (0 for hash routing)
+ *   P_sum      fp32 [N'] or NULL  sum_t s_{i,t}, for reductions across token shards
+ *   scores_dbg fp32 [T, N'] or NULL  the raw scores s (not for hash routing)
+ *
+ * T == 0 writes counts = f = P = P_sum = 0 and nothing else. Returns
+ * DSMOE_ERR_WORKSPACE if T > max_tokens, DSMOE_ERR_INVALID_ARG for a NULL or
+ * misaligned pointer, DSMOE_ERR_CUDA if a launch fails. The output h does not
+ * depend on the order of slots inside an expert's segment.
+ */
+dsmoe_status dsmoe_forward(dsmoe_handle* h, int32_t T,
+                           const void* x, const int32_t* token_ids,
+                           const void* W_router, const float* b,
+                           const void* W_gate, const void* W_up, const void* W_down,
+                           const void* Ws_gate, const void* Ws_up, const void* Ws_down,
+                           void* h_out, int32_t* topk_idx, float* gates,
+                           int32_t* counts, float* f, float* P, float* P_sum,
+                           float* scores_dbg, void* stream);
+
+/*
+ * The same forward with the per-call tensors in HOST memory: x, token_ids and
+ * every output (h, topk_idx, gates, counts, f, P) are host pointers (pinned
+ * memory gives asynchronous copies; pageable memory works but serialises).
+ * The weights stay device-resident. The inputs are copied into the handle's
+ * workspace, the forward runs on `stream`, the outputs are copied back, and
+ * the call synchronises `stream` before returning.
+ */
+dsmoe_status dsmoe_forward_host(dsmoe_handle* h, int32_t T,
+                                const void* x_host, const int32_t* token_ids_host,
+                                const void* W_router, const float* b,
+                                const void* W_gate, const void* W_up, const void* W_down,
+                                const void* Ws_gate, const void* Ws_up, const void* Ws_down,
+                                void* h_host, int32_t* topk_idx_host, float* gates_host,
+                                int32_t* counts_host, float* f_host, float* P_host,
+                                void* stream);
+
+/*
+ * Expert-level balance statistics from token counts and score sums gathered
+ * over T_total tokens (e.g. summed across token shards on several GPUs):
+ * f_i = N' / (K' T_total) * counts_i and P_i = P_sum_i / T_total
+ * (DeepSeekMoE summary, "Expert-level balance loss"). Device pointers, [N'] each.
+ * T_total == 0 writes zeros.
+ */
+dsmoe_status dsmoe_balance_stats(dsmoe_handle* h, int64_t T_total, const int32_t* counts,
+                                 const float* P_sum, float* f, float* P, void* stream);
+
+/* Read and clear the device status word (synchronises the handle's device).
+ * DSMOE_OK, or DSMOE_ERR_DEVICE_TIMEOUT if a kernel gave up a bounded wait. */
+dsmoe_status dsmoe_get_status(dsmoe_handle* h);
+
+/* Bound on every in-kernel wait, in nanoseconds (default 2e9). */
+dsmoe_status dsmoe_set_wait_limit(dsmoe_handle* h, uint64_t ns);
+
+/* Per-stage timing: while enabled, each forward with T > 0 records CUDA events on its
+ * stream at every stage boundary (no synchronisation). dsmoe_stage_times waits for
+ * the recorded events and writes, per stage, the mean duration in ms over the last
+ * min(64, forwards recorded since timing was enabled) forwards. Enabling (or
+ * disabling) timing resets the record. */
+dsmoe_status dsmoe_set_timing(dsmoe_handle* h, int32_t enable);
+dsmoe_status dsmoe_stage_times(dsmoe_handle* h, float* ms, int32_t max_n, int32_t* n);
+/* Name of stage i ("router", "select", "scan", "permute", "gemm_gate_up", "gemm_down",
+ * "combine"), or NULL past the last. */
+const char* dsmoe_stage_name(int32_t i);
+
+/* Number of kernels this handle has launched since creation. */
+dsmoe_status dsmoe_launch_count(dsmoe_handle* h, int64_t* n);
+
+/*
+ * Device address and shape of one intermediate buffer of the handle's workspace, for
+ * tests and debugging; contents are those of the last forward on this handle:
+ *   "logits"  fp32 [T, N']        router affinities (absent for hash routing)
+ *   "offsets" int32 [N'+1]        first slot of each expert's segment
+ *   "slot_of" int32 [T, K']       slot holding token t's k-th expert row
+ *   "Xp"      bf16 [T K', d]      token rows in expert-contiguous slot order
+ *   "A1"      bf16 [T K', F]      SiLU(X W_gate^T) * (X W_up^T) per slot
+ *   "A1s"     bf16 [T, K_s F_s]   the same for the shared experts, side by side
+ *   "Y"       bf16 [T K', d]      routed expert outputs per slot
+ *   "Hs"      fp32 [T, d]         u_t + sum of the shared experts' outputs
+ * Rows/cols are given for max_tokens; the first T (or T K') rows are meaningful.
+ * Returns DSMOE_ERR_INVALID_ARG for an unknown name or a buffer this cfg lacks.
+ */
+dsmoe_status dsmoe_workspace_tensor(dsmoe_handle* h, const char* name, void** ptr, int64_t* rows,
+                                    int64_t* cols);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif /* DSMOE_H */

@@ -1,0 +1,291 @@
+"""ctypes binding of libdsmoe.so with the C ABI's names.
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels. Torch tensors are passed by data pointer (device tensors for
+dsmoe_forward, host tensors for dsmoe_forward_host); streams are torch CUDA
+streams or raw cudaStream_t integers. Importing this module raises if the
+library has not been built; there is no other code path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional, Sequence
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdsmoe.so")
+
+DSMOE_OK, DSMOE_ERR_INVALID_ARG, DSMOE_ERR_UNSUPPORTED, DSMOE_ERR_WORKSPACE, DSMOE_ERR_CUDA, \
+    DSMOE_ERR_DEVICE_TIMEOUT = range(6)
+DSMOE_SCORE_SOFTMAX, DSMOE_SCORE_SIGMOID, DSMOE_SCORE_SQRT_SOFTPLUS, DSMOE_ROUTE_HASH = range(4)
+DSMOE_BIAS_NONE, DSMOE_BIAS_SELECT_ONLY, DSMOE_BIAS_IN_LOGITS = range(3)
+
+ABI_FUNCTIONS = (
+    "dsmoe_abi_version", "dsmoe_status_string", "dsmoe_last_error", "dsmoe_check_config",
+    "dsmoe_workspace_bytes", "dsmoe_create", "dsmoe_destroy", "dsmoe_forward", "dsmoe_forward_host",
+    "dsmoe_balance_stats", "dsmoe_get_status", "dsmoe_set_wait_limit", "dsmoe_set_timing",
+    "dsmoe_stage_times", "dsmoe_stage_name", "dsmoe_launch_count", "dsmoe_workspace_tensor",
+)
+
+
+class DsmoeCfg(ctypes.Structure):
+    _fields_ = [("d_model", ctypes.c_int32), ("n_routed", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("d_ff", ctypes.c_int32), ("n_shared", ctypes.c_int32), ("d_ff_shared", ctypes.c_int32),
+                ("score", ctypes.c_int32), ("bias_mode", ctypes.c_int32), ("renormalize", ctypes.c_int32),
+                ("max_tokens", ctypes.c_int32), ("hash_mult", ctypes.c_uint32), ("hash_mod", ctypes.c_uint32)]
+
+
+class DsmoeError(RuntimeError):
+    def __init__(self, status: int, where: str, message: str):
+        super().__init__(f"{where}: {status_string(status)} ({status}): {message}")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python mixture_experts_layer_score_b200/build.py` (there is no fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, u64, f32p, i32p = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64,
+                                     ctypes.c_void_p, ctypes.c_void_p)
+    cfgp = ctypes.POINTER(DsmoeCfg)
+    sig = {
+        "dsmoe_abi_version": (i32, []),
+        "dsmoe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "dsmoe_last_error": (ctypes.c_char_p, []),
+        "dsmoe_check_config": (ctypes.c_int, [cfgp]),
+        "dsmoe_workspace_bytes": (ctypes.c_int, [cfgp, ctypes.POINTER(ctypes.c_size_t)]),
+        "dsmoe_create": (ctypes.c_int, [cfgp, i32, ctypes.POINTER(vp)]),
+        "dsmoe_destroy": (None, [vp]),
+        "dsmoe_forward": (ctypes.c_int, [vp, i32] + [vp] * 18 + [vp]),
+        "dsmoe_forward_host": (ctypes.c_int, [vp, i32] + [vp] * 16 + [vp]),
+        "dsmoe_balance_stats": (ctypes.c_int, [vp, i64, vp, vp, vp, vp, vp]),
+        "dsmoe_get_status": (ctypes.c_int, [vp]),
+        "dsmoe_set_wait_limit": (ctypes.c_int, [vp, u64]),
+        "dsmoe_set_timing": (ctypes.c_int, [vp, i32]),
+        "dsmoe_stage_times": (ctypes.c_int, [vp, ctypes.POINTER(ctypes.c_float), i32, ctypes.POINTER(i32)]),
+        "dsmoe_stage_name": (ctypes.c_char_p, [i32]),
+        "dsmoe_launch_count": (ctypes.c_int, [vp, ctypes.POINTER(i64)]),
+        "dsmoe_workspace_tensor": (ctypes.c_int, [vp, ctypes.c_char_p, ctypes.POINTER(vp),
+                                                  ctypes.POINTER(i64), ctypes.POINTER(i64)]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def status_string(status: int) -> str:
+    return _lib.dsmoe_status_string(int(status)).decode()
+
+
+def dsmoe_status_string(status: int) -> str:
+    return status_string(status)
+
+
+def dsmoe_last_error() -> str:
+    return _lib.dsmoe_last_error().decode()
+
+
+def _check(status: int, where: str):
+    if status != DSMOE_OK:
+        raise DsmoeError(status, where, dsmoe_last_error())
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def make_cfg(d_model: int, n_routed: int, top_k: int, d_ff: int, n_shared: int = 0, d_ff_shared: int = 0,
+             score: int = DSMOE_SCORE_SOFTMAX, bias_mode: int = DSMOE_BIAS_NONE, renormalize: bool = False,
+             max_tokens: int = 1, hash_mult: int = 2654435761, hash_mod: int = 0) -> DsmoeCfg:
+    return DsmoeCfg(d_model, n_routed, top_k, d_ff, n_shared, d_ff_shared, score, bias_mode, int(renormalize),
+                    max_tokens, hash_mult, hash_mod)
+
+
+def cfg_from(obj, max_tokens: int) -> DsmoeCfg:
+    """dsmoe_cfg from any object with the layer's field names (d_model, n_routed, top_k, ...)."""
+    return make_cfg(obj.d_model, obj.n_routed, obj.top_k, obj.d_ff, obj.n_shared, obj.d_ff_shared, obj.score,
+                    obj.bias_mode, obj.renormalize, max_tokens, getattr(obj, "hash_mult", 2654435761), 0)
+
+
+def dsmoe_abi_version() -> int:
+    return _lib.dsmoe_abi_version()
+
+
+def dsmoe_check_config(cfg: DsmoeCfg) -> int:
+    return _lib.dsmoe_check_config(ctypes.byref(cfg))
+
+
+def dsmoe_workspace_bytes(cfg: DsmoeCfg) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.dsmoe_workspace_bytes(ctypes.byref(cfg), ctypes.byref(n)), "dsmoe_workspace_bytes")
+    return n.value
+
+
+def dsmoe_create(cfg: DsmoeCfg, device: int = 0) -> int:
+    h = ctypes.c_void_p()
+    _check(_lib.dsmoe_create(ctypes.byref(cfg), int(device), ctypes.byref(h)), "dsmoe_create")
+    return h.value
+
+
+def dsmoe_destroy(handle: int) -> None:
+    _lib.dsmoe_destroy(handle)
+
+
+def dsmoe_forward(handle, T, x, token_ids, W_router, b, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down,
+                  h, topk_idx, gates, counts, f, P, P_sum=None, scores_dbg=None, stream=None) -> None:
+    st = _lib.dsmoe_forward(handle, int(T), *[_ptr(t) for t in (
+        x, token_ids, W_router, b, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, h, topk_idx, gates, counts, f,
+        P, P_sum, scores_dbg)], _stream(stream))
+    _check(st, "dsmoe_forward")
+
+
+def dsmoe_forward_host(handle, T, x_host, token_ids_host, W_router, b, W_gate, W_up, W_down, Ws_gate, Ws_up,
+                       Ws_down, h_host, topk_idx_host, gates_host, counts_host, f_host, P_host,
+                       stream=None) -> None:
+    st = _lib.dsmoe_forward_host(handle, int(T), *[_ptr(t) for t in (
+        x_host, token_ids_host, W_router, b, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, h_host,
+        topk_idx_host, gates_host, counts_host, f_host, P_host)], _stream(stream))
+    _check(st, "dsmoe_forward_host")
+
+
+def dsmoe_balance_stats(handle, T_total, counts, P_sum, f, P, stream=None) -> None:
+    _check(_lib.dsmoe_balance_stats(handle, int(T_total), _ptr(counts), _ptr(P_sum), _ptr(f), _ptr(P),
+                                    _stream(stream)), "dsmoe_balance_stats")
+
+
+def dsmoe_get_status(handle) -> int:
+    return _lib.dsmoe_get_status(handle)
+
+
+def dsmoe_set_wait_limit(handle, ns: int) -> None:
+    _check(_lib.dsmoe_set_wait_limit(handle, int(ns)), "dsmoe_set_wait_limit")
+
+
+def dsmoe_set_timing(handle, enable: bool) -> None:
+    _check(_lib.dsmoe_set_timing(handle, int(bool(enable))), "dsmoe_set_timing")
+
+
+def dsmoe_stage_name(i: int) -> Optional[str]:
+    r = _lib.dsmoe_stage_name(int(i))
+    return None if r is None else r.decode()
+
+
+def stage_names() -> Sequence[str]:
+    out, i = [], 0
+    while (n := dsmoe_stage_name(i)) is not None:
+        out.append(n)
+        i += 1
+    return out
+
+
+def dsmoe_stage_times(handle) -> Dict[str, float]:
+    names = stage_names()
+    buf = (ctypes.c_float * len(names))()
+    n = ctypes.c_int32(0)
+    _check(_lib.dsmoe_stage_times(handle, buf, len(names), ctypes.byref(n)), "dsmoe_stage_times")
+    return {names[i]: float(buf[i]) for i in range(n.value)}
+
+
+def dsmoe_launch_count(handle) -> int:
+    n = ctypes.c_int64(0)
+    _check(_lib.dsmoe_launch_count(handle, ctypes.byref(n)), "dsmoe_launch_count")
+    return n.value
+
+
+_WS_DTYPES = {"logits": "float32", "offsets": "int32", "slot_of": "int32", "Xp": "bfloat16",
+              "A1": "bfloat16", "A1s": "bfloat16", "Y": "bfloat16", "Hs": "float32"}
+
+
+def dsmoe_workspace_tensor(handle, name: str):
+    """(device address, rows, cols) of an intermediate workspace buffer."""
+    p, r, c = ctypes.c_void_p(), ctypes.c_int64(), ctypes.c_int64()
+    _check(_lib.dsmoe_workspace_tensor(handle, name.encode(), ctypes.byref(p), ctypes.byref(r), ctypes.byref(c)),
+           "dsmoe_workspace_tensor")
+    return p.value, r.value, c.value
+
+
+def workspace_view(handle, name: str, device: int = 0):
+    """A torch tensor aliasing a workspace buffer (copy it before the next forward)."""
+    import torch
+    ptr, rows, cols = dsmoe_workspace_tensor(handle, name)
+    dt = getattr(torch, _WS_DTYPES[name])
+    n = rows * cols
+    esz = torch.empty((), dtype=dt).element_size()
+
+    class _Buf:  # minimal __cuda_array_interface__ exporter over the raw device pointer
+        pass
+
+    b = _Buf()
+    typestr = {"float32": "<f4", "int32": "<i4", "bfloat16": "<i2"}[_WS_DTYPES[name]]
+    b.__cuda_array_interface__ = dict(shape=(n,), typestr=typestr, data=(ptr, False), version=3)
+    with torch.cuda.device(device):
+        t = torch.as_tensor(b, device=f"cuda:{device}")
+    if _WS_DTYPES[name] == "bfloat16":
+        t = t.view(torch.bfloat16)
+    assert t.element_size() == esz
+    return t.view(rows, cols)
+
+
+class DSMoE:
+    """A handle plus the weight tensors of one layer; forward() allocates the outputs with
+    torch (device memory only) and calls dsmoe_forward."""
+
+    def __init__(self, cfg: DsmoeCfg, weights: Dict, device: int = 0):
+        self.cfg = cfg
+        self.device = device
+        self.w = weights
+        self.handle = dsmoe_create(cfg, device)
+
+    def close(self):
+        if self.handle:
+            dsmoe_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def alloc_outputs(self, T: int, with_scores: bool = False):
+        import torch
+        dev = torch.device("cuda", self.device)
+        c = self.cfg
+        out = dict(h=torch.empty((T, c.d_model), dtype=torch.bfloat16, device=dev),
+                   topk_idx=torch.empty((T, c.top_k), dtype=torch.int32, device=dev),
+                   gates=torch.empty((T, c.top_k), dtype=torch.float32, device=dev),
+                   counts=torch.empty((c.n_routed,), dtype=torch.int32, device=dev),
+                   f=torch.empty((c.n_routed,), dtype=torch.float32, device=dev),
+                   P=torch.empty((c.n_routed,), dtype=torch.float32, device=dev),
+                   P_sum=torch.empty((c.n_routed,), dtype=torch.float32, device=dev))
+        out["scores"] = (torch.empty((T, c.n_routed), dtype=torch.float32, device=dev)
+                         if with_scores and c.score != DSMOE_ROUTE_HASH else None)
+        return out
+
+    def forward(self, x, token_ids=None, out=None, with_scores: bool = False, stream=None):
+        T = x.shape[0]
+        o = self.alloc_outputs(T, with_scores) if out is None else out
+        w = self.w
+        dsmoe_forward(self.handle, T, x, token_ids, w.get("W_router"), w.get("b"), w["W_gate"], w["W_up"],
+                      w["W_down"], w.get("Ws_gate"), w.get("Ws_up"), w.get("Ws_down"), o["h"], o["topk_idx"],
+                      o["gates"], o["counts"], o["f"], o["P"], o["P_sum"], o["scores"], stream)
+        return o

@@ -1,0 +1,722 @@
+// dsmoe_api.cu -- the C ABI of libdsmoe.so: configuration checks, the handle and its
+// workspace, TMA tensor maps, and the launch sequence of one layer forward:
+//
+//   router logits -> scores / top-K' / gates (+ statistics partials) -> counts scan,
+//   f_i, P_i, segment offsets -> slot permutation + row gather -> gate/up grouped GEMM
+//   with SiLU*up -> down grouped GEMM -> gate-weighted combine + residual.
+//
+// Nothing here synchronises the device inside dsmoe_forward, and nothing allocates
+// outside dsmoe_create.
+#include <cudaTypedefs.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+#include <string>
+
+#include "dsmoe.h"
+#include "kernels.h"
+
+#define DSMOE_EXPORT extern "C" __attribute__((visibility("default")))
+
+using dsmoe::bf16;
+
+namespace {
+
+constexpr int kNumStages = 7;
+const char* const kStageNames[kNumStages] = {"router", "select", "scan", "permute", "gemm_gate_up", "gemm_down",
+                                             "combine"};
+constexpr int kSelectMaxBlocks = 1024;  // rows of the statistics partials
+constexpr int kTimingSlots = 64;        // forwards whose stage events are kept
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+
+thread_local std::string g_last_error;
+
+dsmoe_status fail(dsmoe_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+#define CUDA_TRY(expr)                                                                              \
+  do {                                                                                              \
+    cudaError_t e_ = (expr);                                                                        \
+    if (e_ != cudaSuccess) return fail(DSMOE_ERR_CUDA, "%s failed: %s", #expr, cudaGetErrorString(e_)); \
+  } while (0)
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2D bf16 map [outer, inner] (inner contiguous), 128-byte swizzle, box (64, box_outer).
+bool map_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_outer) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3D bf16 map [experts, rows, inner], 128-byte swizzle, box (64, box_rows, 1).
+bool map_3d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, uint64_t experts, uint32_t box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {inner, rows, experts};
+  cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct DeviceGuard {
+  int prev = -1, want;
+  bool ok = false;
+  explicit DeviceGuard(int d) : want(d) {
+    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+    ok = (prev == d) || cudaSetDevice(d) == cudaSuccess;
+  }
+  ~DeviceGuard() {
+    if (prev >= 0 && prev != want) cudaSetDevice(prev);
+  }
+};
+
+struct Layout {
+  size_t logits, counts_ws, cursor, offsets, P_part, slot_of, Xp, A1, A1s, Y, Hs, status;
+  size_t x_stage, ids_stage, h_stage, topk_stage, gates_stage, counts_stage, f_stage, P_stage;
+  size_t total;
+};
+
+size_t up256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+Layout plan(const dsmoe_cfg& c) {
+  Layout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += up256(bytes > 0 ? bytes : 1);
+    return o;
+  };
+  const size_t T = static_cast<size_t>(c.max_tokens), N = c.n_routed, K = c.top_k, d = c.d_model, F = c.d_ff;
+  const size_t S = T * K, KsFs = static_cast<size_t>(c.n_shared) * c.d_ff_shared;
+  const bool hash = c.score == DSMOE_ROUTE_HASH;
+  L.logits = take(hash ? 0 : T * N * 4);
+  L.counts_ws = take(N * 4);
+  L.cursor = take(N * 4);
+  L.offsets = take((N + 1) * 4);
+  L.P_part = take(hash ? 0 : static_cast<size_t>(kSelectMaxBlocks) * N * 4);
+  L.slot_of = take(S * 4);
+  L.Xp = take(S * d * 2);
+  L.A1 = take(S * F * 2);
+  L.A1s = take(T * KsFs * 2);
+  L.Y = take(S * d * 2);
+  L.Hs = take(c.n_shared > 0 ? T * d * 4 : 0);
+  L.status = take(4);
+  L.x_stage = take(T * d * 2);
+  L.ids_stage = take(hash ? T * 4 : 0);
+  L.h_stage = take(T * d * 2);
+  L.topk_stage = take(S * 4);
+  L.gates_stage = take(S * 4);
+  L.counts_stage = take(N * 4);
+  L.f_stage = take(N * 4);
+  L.P_stage = take(N * 4);
+  L.total = off;
+  return L;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+struct dsmoe_handle {
+  dsmoe_cfg cfg;
+  int device = 0;
+  int num_sms = 148;
+  uint64_t wait_ns = kDefaultWaitNs;
+  char* ws = nullptr;
+  Layout L;
+  float* logits;
+  int32_t *counts_ws, *cursor, *offsets, *slot_of;
+  float* P_part;
+  bf16 *Xp, *A1, *A1s, *Y;
+  float* Hs;
+  uint32_t* status;
+  bf16 *x_stage, *h_stage;
+  int32_t *ids_stage, *topk_stage, *counts_stage;
+  float *gates_stage, *f_stage, *P_stage;
+  CUtensorMap tm_xp, tm_a1, tm_a1s;
+  const void* wkey[6] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+  CUtensorMap tm_w[6];  // W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down
+  bool timing = false;
+  int timed_forwards = 0;               // forwards recorded since timing was enabled
+  cudaEvent_t ev[kTimingSlots][kNumStages + 1] = {};
+  int64_t launches = 0;
+};
+
+// ========================================================================================
+// configuration
+// ========================================================================================
+DSMOE_EXPORT int32_t dsmoe_abi_version(void) { return DSMOE_ABI_VERSION; }
+
+DSMOE_EXPORT const char* dsmoe_status_string(dsmoe_status s) {
+  switch (s) {
+    case DSMOE_OK: return "ok";
+    case DSMOE_ERR_INVALID_ARG: return "invalid argument";
+    case DSMOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case DSMOE_ERR_WORKSPACE: return "workspace too small or allocation failed";
+    case DSMOE_ERR_CUDA: return "CUDA error";
+    case DSMOE_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+DSMOE_EXPORT const char* dsmoe_last_error(void) { return g_last_error.c_str(); }
+
+DSMOE_EXPORT dsmoe_status dsmoe_check_config(const dsmoe_cfg* c) {
+  if (!c) return fail(DSMOE_ERR_INVALID_ARG, "cfg is NULL");
+  if (c->score < DSMOE_SCORE_SOFTMAX || c->score > DSMOE_ROUTE_HASH)
+    return fail(DSMOE_ERR_INVALID_ARG, "score %d is not a dsmoe_score", c->score);
+  if (c->bias_mode < DSMOE_BIAS_NONE || c->bias_mode > DSMOE_BIAS_IN_LOGITS)
+    return fail(DSMOE_ERR_INVALID_ARG, "bias_mode %d is not a dsmoe_bias_mode", c->bias_mode);
+  if (c->renormalize != 0 && c->renormalize != 1) return fail(DSMOE_ERR_INVALID_ARG, "renormalize must be 0 or 1");
+  if (c->d_model <= 0 || c->n_routed <= 0 || c->top_k <= 0 || c->d_ff <= 0 || c->max_tokens <= 0)
+    return fail(DSMOE_ERR_INVALID_ARG, "d_model, n_routed, top_k, d_ff and max_tokens must be positive");
+  if (c->n_shared < 0 || (c->n_shared > 0 && c->d_ff_shared <= 0))
+    return fail(DSMOE_ERR_INVALID_ARG, "n_shared must be >= 0 and d_ff_shared > 0 when it is not");
+  if (c->top_k > c->n_routed) return fail(DSMOE_ERR_INVALID_ARG, "top_k %d exceeds n_routed %d", c->top_k, c->n_routed);
+  if (c->score == DSMOE_ROUTE_HASH) {
+    if (c->top_k != 1) return fail(DSMOE_ERR_INVALID_ARG, "hash routing picks one expert per token (top_k=1)");
+    if (c->bias_mode != DSMOE_BIAS_NONE) return fail(DSMOE_ERR_INVALID_ARG, "hash routing takes no bias");
+    if (c->hash_mult == 0) return fail(DSMOE_ERR_INVALID_ARG, "hash_mult must be non-zero");
+    if (c->hash_mod > static_cast<uint32_t>(c->n_routed))
+      return fail(DSMOE_ERR_INVALID_ARG, "hash_mod %u exceeds n_routed %d", c->hash_mod, c->n_routed);
+  }
+  if (c->d_model % 64 || c->d_ff % 64 || (c->n_shared > 0 && c->d_ff_shared % 64))
+    return fail(DSMOE_ERR_UNSUPPORTED, "d_model, d_ff and d_ff_shared must be multiples of 64");
+  if (c->n_routed > 512) return fail(DSMOE_ERR_UNSUPPORTED, "n_routed %d > 512", c->n_routed);
+  if (c->top_k > 16) return fail(DSMOE_ERR_UNSUPPORTED, "top_k %d > 16", c->top_k);
+  if (c->n_shared > 8) return fail(DSMOE_ERR_UNSUPPORTED, "n_shared %d > 8", c->n_shared);
+  if (c->d_model > 32768 || c->d_ff > 32768 || c->d_ff_shared > 32768)
+    return fail(DSMOE_ERR_UNSUPPORTED, "d_model / d_ff above 32768");
+  if (static_cast<int64_t>(c->max_tokens) * c->top_k > (int64_t{1} << 30))
+    return fail(DSMOE_ERR_UNSUPPORTED, "max_tokens * top_k above 2^30");
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_workspace_bytes(const dsmoe_cfg* cfg, size_t* bytes) {
+  if (!bytes) return fail(DSMOE_ERR_INVALID_ARG, "bytes is NULL");
+  const dsmoe_status st = dsmoe_check_config(cfg);
+  if (st != DSMOE_OK) return st;
+  *bytes = plan(*cfg).total;
+  return DSMOE_OK;
+}
+
+// ========================================================================================
+// handle
+// ========================================================================================
+static void release(dsmoe_handle* h) {
+  if (!h) return;
+  DeviceGuard g(h->device);
+  for (auto& set : h->ev)
+    for (auto& e : set)
+      if (e) cudaEventDestroy(e);
+  if (h->ws) cudaFree(h->ws);
+  delete h;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_create(const dsmoe_cfg* cfg, int32_t device, dsmoe_handle** out) {
+  if (!out) return fail(DSMOE_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  dsmoe_status st = dsmoe_check_config(cfg);
+  if (st != DSMOE_OK) return st;
+  int ndev = 0;
+  CUDA_TRY(cudaGetDeviceCount(&ndev));
+  if (device < 0 || device >= ndev) return fail(DSMOE_ERR_INVALID_ARG, "device %d of %d", device, ndev);
+  DeviceGuard g(device);
+  if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", device);
+  cudaDeviceProp prop;
+  CUDA_TRY(cudaGetDeviceProperties(&prop, device));
+  if (prop.major != 10 || prop.minor != 0)
+    return fail(DSMOE_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", device, prop.major,
+                prop.minor);
+  if (!tensor_map_encoder()) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+
+  dsmoe_handle* h = new dsmoe_handle();
+  h->cfg = *cfg;
+  if (h->cfg.score == DSMOE_ROUTE_HASH && h->cfg.hash_mod == 0) h->cfg.hash_mod = h->cfg.n_routed;
+  h->device = device;
+  h->num_sms = prop.multiProcessorCount;
+  h->L = plan(h->cfg);
+  cudaError_t e = cudaMalloc(&h->ws, h->L.total);
+  if (e != cudaSuccess) {
+    h->ws = nullptr;
+    release(h);
+    return fail(DSMOE_ERR_WORKSPACE, "cudaMalloc(%zu) failed: %s", h->L.total, cudaGetErrorString(e));
+  }
+  char* w = h->ws;
+  const Layout& L = h->L;
+  h->logits = reinterpret_cast<float*>(w + L.logits);
+  h->counts_ws = reinterpret_cast<int32_t*>(w + L.counts_ws);
+  h->cursor = reinterpret_cast<int32_t*>(w + L.cursor);
+  h->offsets = reinterpret_cast<int32_t*>(w + L.offsets);
+  h->P_part = reinterpret_cast<float*>(w + L.P_part);
+  h->slot_of = reinterpret_cast<int32_t*>(w + L.slot_of);
+  h->Xp = reinterpret_cast<bf16*>(w + L.Xp);
+  h->A1 = reinterpret_cast<bf16*>(w + L.A1);
+  h->A1s = reinterpret_cast<bf16*>(w + L.A1s);
+  h->Y = reinterpret_cast<bf16*>(w + L.Y);
+  h->Hs = reinterpret_cast<float*>(w + L.Hs);
+  h->status = reinterpret_cast<uint32_t*>(w + L.status);
+  h->x_stage = reinterpret_cast<bf16*>(w + L.x_stage);
+  h->ids_stage = reinterpret_cast<int32_t*>(w + L.ids_stage);
+  h->h_stage = reinterpret_cast<bf16*>(w + L.h_stage);
+  h->topk_stage = reinterpret_cast<int32_t*>(w + L.topk_stage);
+  h->gates_stage = reinterpret_cast<float*>(w + L.gates_stage);
+  h->counts_stage = reinterpret_cast<int32_t*>(w + L.counts_stage);
+  h->f_stage = reinterpret_cast<float*>(w + L.f_stage);
+  h->P_stage = reinterpret_cast<float*>(w + L.P_stage);
+  e = cudaMemset(h->ws, 0, h->L.total);
+  if (e != cudaSuccess) {
+    release(h);
+    return fail(DSMOE_ERR_CUDA, "cudaMemset failed: %s", cudaGetErrorString(e));
+  }
+  const dsmoe_cfg& c = h->cfg;
+  const uint64_t S = static_cast<uint64_t>(c.max_tokens) * c.top_k;
+  bool ok = map_2d(&h->tm_xp, h->Xp, c.d_model, S, 128) && map_2d(&h->tm_a1, h->A1, c.d_ff, S, 128);
+  if (c.n_shared > 0)
+    ok = ok && map_2d(&h->tm_a1s, h->A1s, static_cast<uint64_t>(c.n_shared) * c.d_ff_shared, c.max_tokens, 128);
+  else
+    h->tm_a1s = h->tm_a1;
+  if (!ok) {
+    release(h);
+    return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a workspace tensor map");
+  }
+  for (auto& set : h->ev)
+    for (auto& ev : set) {
+      e = cudaEventCreate(&ev);
+      if (e != cudaSuccess) {
+        release(h);
+        return fail(DSMOE_ERR_CUDA, "cudaEventCreate failed: %s", cudaGetErrorString(e));
+      }
+    }
+  *out = h;
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT void dsmoe_destroy(dsmoe_handle* h) {
+  if (!h) return;
+  {
+    DeviceGuard g(h->device);
+    cudaDeviceSynchronize();
+  }
+  release(h);
+}
+
+// ========================================================================================
+// forward
+// ========================================================================================
+namespace {
+
+struct FwdArgs {
+  int32_t T;
+  const void *x, *W_router, *W_gate, *W_up, *W_down, *Ws_gate, *Ws_up, *Ws_down;
+  const int32_t* token_ids;
+  const float* b;
+  void* h;
+  int32_t* topk_idx;
+  float* gates;
+  int32_t* counts;
+  float *f, *P, *P_sum, *scores_dbg;
+};
+
+dsmoe_status check_forward(dsmoe_handle* h, const FwdArgs& a) {
+  const dsmoe_cfg& c = h->cfg;
+  if (a.T < 0) return fail(DSMOE_ERR_INVALID_ARG, "T = %d is negative", a.T);
+  if (a.T > c.max_tokens) return fail(DSMOE_ERR_WORKSPACE, "T = %d exceeds max_tokens = %d", a.T, c.max_tokens);
+  if (!a.counts || !a.f || !a.P) return fail(DSMOE_ERR_INVALID_ARG, "counts, f and P are required");
+  if (a.T == 0) return DSMOE_OK;
+  const bool hash = c.score == DSMOE_ROUTE_HASH;
+  if (!a.x || !a.h || !a.topk_idx || !a.gates || !a.W_gate || !a.W_up || !a.W_down)
+    return fail(DSMOE_ERR_INVALID_ARG, "x, h, topk_idx, gates and the routed weights are required");
+  if (hash && !a.token_ids) return fail(DSMOE_ERR_INVALID_ARG, "hash routing needs token_ids");
+  if (!hash && !a.W_router) return fail(DSMOE_ERR_INVALID_ARG, "W_router is required");
+  if (c.bias_mode != DSMOE_BIAS_NONE && !a.b) return fail(DSMOE_ERR_INVALID_ARG, "bias b is required by bias_mode");
+  if (c.n_shared > 0 && (!a.Ws_gate || !a.Ws_up || !a.Ws_down))
+    return fail(DSMOE_ERR_INVALID_ARG, "shared expert weights are required (n_shared = %d)", c.n_shared);
+  const void* must_align[] = {a.x, a.W_router, a.W_gate, a.W_up, a.W_down, a.Ws_gate, a.Ws_up, a.Ws_down, a.h};
+  for (const void* p : must_align)
+    if (p && !aligned16(p)) return fail(DSMOE_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", p);
+  return DSMOE_OK;
+}
+
+const CUtensorMap* weight_map(dsmoe_handle* h, int which, const void* ptr, bool* ok) {
+  if (h->wkey[which] != ptr) {
+    const dsmoe_cfg& c = h->cfg;
+    bool r = false;
+    switch (which) {
+      case 0:
+      case 1: r = map_3d(&h->tm_w[which], ptr, c.d_model, c.d_ff, c.n_routed, 128); break;
+      case 2: r = map_3d(&h->tm_w[which], ptr, c.d_ff, c.d_model, c.n_routed, 256); break;
+      case 3:
+      case 4: r = map_3d(&h->tm_w[which], ptr, c.d_model, c.d_ff_shared, c.n_shared, 128); break;
+      case 5: r = map_3d(&h->tm_w[which], ptr, c.d_ff_shared, c.d_model, c.n_shared, 256); break;
+    }
+    if (!r) {
+      h->wkey[which] = nullptr;
+      *ok = false;
+      return &h->tm_w[which];
+    }
+    h->wkey[which] = ptr;
+  }
+  return &h->tm_w[which];
+}
+
+int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+
+dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
+  const dsmoe_cfg& c = h->cfg;
+  const int T = a.T, N = c.n_routed, K = c.top_k, d = c.d_model, F = c.d_ff;
+  const int Ks = c.n_shared, Fs = c.d_ff_shared;
+  const bool hash = c.score == DSMOE_ROUTE_HASH;
+  const bool timing = h->timing && T > 0;
+  cudaEvent_t* evs = h->ev[h->timed_forwards % kTimingSlots];
+  auto mark = [&](int i) -> cudaError_t { return timing ? cudaEventRecord(evs[i], s) : cudaSuccess; };
+
+  if (T == 0) {
+    CUDA_TRY(cudaMemsetAsync(a.counts, 0, N * sizeof(int32_t), s));
+    CUDA_TRY(cudaMemsetAsync(a.f, 0, N * sizeof(float), s));
+    CUDA_TRY(cudaMemsetAsync(a.P, 0, N * sizeof(float), s));
+    if (a.P_sum) CUDA_TRY(cudaMemsetAsync(a.P_sum, 0, N * sizeof(float), s));
+    return DSMOE_OK;
+  }
+
+  // tensor maps that depend on the call's pointers
+  bool ok = true;
+  const CUtensorMap* m_wg = weight_map(h, 0, a.W_gate, &ok);
+  const CUtensorMap* m_wu = weight_map(h, 1, a.W_up, &ok);
+  const CUtensorMap* m_wd = weight_map(h, 2, a.W_down, &ok);
+  const CUtensorMap* m_swg = Ks ? weight_map(h, 3, a.Ws_gate, &ok) : m_wg;
+  const CUtensorMap* m_swu = Ks ? weight_map(h, 4, a.Ws_up, &ok) : m_wu;
+  const CUtensorMap* m_swd = Ks ? weight_map(h, 5, a.Ws_down, &ok) : m_wd;
+  CUtensorMap m_x;
+  ok = ok && map_2d(&m_x, a.x, d, T, 128);
+  if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map of this call");
+
+  CUDA_TRY(mark(0));
+  CUDA_TRY(cudaMemsetAsync(h->counts_ws, 0, N * sizeof(int32_t), s));
+  int sel_grid = 0;
+  if (hash) {
+    CUDA_TRY(dsmoe::launch_hash_route(a.token_ids, T, N, c.hash_mult, c.hash_mod, a.topk_idx, a.gates, h->counts_ws,
+                                      h->status, s));
+    h->launches += 1;
+    CUDA_TRY(mark(1));
+  } else {
+    CUDA_TRY(dsmoe::launch_router_logits(static_cast<const bf16*>(a.x), static_cast<const bf16*>(a.W_router), a.b,
+                                         c.bias_mode == DSMOE_BIAS_IN_LOGITS, T, N, d, h->logits, s));
+    CUDA_TRY(mark(1));
+    dsmoe::SelectArgs sa;
+    sa.logits = h->logits;
+    sa.b = a.b;
+    sa.T = T;
+    sa.N = N;
+    sa.K = K;
+    sa.score = c.score;
+    sa.bias_select = c.bias_mode == DSMOE_BIAS_SELECT_ONLY;
+    sa.renormalize = c.renormalize;
+    sa.topk_idx = a.topk_idx;
+    sa.gates = a.gates;
+    sa.counts = h->counts_ws;
+    sa.P_part = h->P_part;
+    sa.scores_dbg = a.scores_dbg;
+    sa.status = h->status;
+    sel_grid = dsmoe::select_grid(T, kSelectMaxBlocks / 4);
+    CUDA_TRY(dsmoe::launch_select(sa, sel_grid, s));
+    h->launches += 2;
+  }
+  CUDA_TRY(mark(2));
+
+  dsmoe::ScanArgs sc;
+  sc.counts_ws = h->counts_ws;
+  sc.P_part = hash ? nullptr : h->P_part;
+  sc.n_part = sel_grid;
+  sc.N = N;
+  sc.K = K;
+  sc.T = T;
+  sc.counts = a.counts;
+  sc.f = a.f;
+  sc.P = a.P;
+  sc.P_sum = a.P_sum;
+  sc.offsets = h->offsets;
+  sc.cursor = h->cursor;
+  CUDA_TRY(dsmoe::launch_scan_stats(sc, s));
+  h->launches += 1;
+  CUDA_TRY(mark(3));
+
+  CUDA_TRY(dsmoe::launch_permute_gather(static_cast<const bf16*>(a.x), a.topk_idx, h->offsets, h->cursor, T, K, N, d,
+                                        h->slot_of, h->Xp, h->status, h->num_sms, s));
+  h->launches += 1;
+  CUDA_TRY(mark(4));
+
+  const int64_t S = static_cast<int64_t>(T) * K;
+  // ---- gate/up GEMM with SiLU(gate) * up
+  {
+    dsmoe::GemmArgs g;
+    memset(&g, 0, sizeof(g));
+    g.a_routed = h->tm_xp;
+    g.a_shared = m_x;
+    g.b0_routed = *m_wg;
+    g.b1_routed = *m_wu;
+    g.b0_shared = *m_swg;
+    g.b1_shared = *m_swu;
+    g.offsets = h->offsets;
+    g.n_routed = N;
+    g.n_shared_groups = Ks;
+    g.m_shared = T;
+    g.n_tiles_routed = cdiv(F, 128);
+    g.n_tiles_shared = Ks ? cdiv(Fs, 128) : 0;
+    g.kb_routed = d / 64;
+    g.kb_shared = d / 64;
+    g.kb_per_b_expert_shared = d / 64;
+    g.n_valid_routed = F;
+    g.n_valid_shared = Fs;
+    g.out_routed = h->A1;
+    g.ld_routed = F;
+    g.out_shared = h->A1s;
+    g.ld_shared = static_cast<int64_t>(Ks) * Fs;
+    g.shared_col_stride = Fs;
+    g.status = h->status;
+    g.wait_limit_ns = h->wait_ns;
+    const int64_t bound = (cdiv(S, 128) + N) * static_cast<int64_t>(g.n_tiles_routed) +
+                          static_cast<int64_t>(Ks) * cdiv(T, 128) * g.n_tiles_shared;
+    const int grid = static_cast<int>(bound < h->num_sms ? bound : h->num_sms);
+    CUDA_TRY(dsmoe::launch_grouped_gemm(true, g, grid, s));
+    h->launches += 1;
+  }
+  CUDA_TRY(mark(5));
+  // ---- down GEMM; the shared experts accumulate into one output row per token
+  {
+    dsmoe::GemmArgs g;
+    memset(&g, 0, sizeof(g));
+    g.a_routed = h->tm_a1;
+    g.a_shared = h->tm_a1s;
+    g.b0_routed = *m_wd;
+    g.b1_routed = *m_wd;
+    g.b0_shared = *m_swd;
+    g.b1_shared = *m_swd;
+    g.offsets = h->offsets;
+    g.n_routed = N;
+    g.n_shared_groups = Ks ? 1 : 0;
+    g.m_shared = T;
+    g.n_tiles_routed = cdiv(d, 256);
+    g.n_tiles_shared = Ks ? cdiv(d, 256) : 0;
+    g.kb_routed = F / 64;
+    g.kb_shared = Ks ? Ks * Fs / 64 : 0;
+    g.kb_per_b_expert_shared = Ks ? Fs / 64 : 1;
+    g.n_valid_routed = d;
+    g.n_valid_shared = d;
+    g.out_routed = h->Y;
+    g.ld_routed = d;
+    g.out_shared = nullptr;
+    g.out_shared_f32 = h->Hs;
+    g.residual = static_cast<const bf16*>(a.x);
+    g.ld_shared = d;
+    g.shared_col_stride = 0;
+    g.status = h->status;
+    g.wait_limit_ns = h->wait_ns;
+    const int64_t bound = (cdiv(S, 128) + N) * static_cast<int64_t>(g.n_tiles_routed) +
+                          static_cast<int64_t>(g.n_shared_groups) * cdiv(T, 128) * g.n_tiles_shared;
+    const int grid = static_cast<int>(bound < h->num_sms ? bound : h->num_sms);
+    CUDA_TRY(dsmoe::launch_grouped_gemm(false, g, grid, s));
+    h->launches += 1;
+  }
+  CUDA_TRY(mark(6));
+  CUDA_TRY(dsmoe::launch_combine(static_cast<const bf16*>(a.x), Ks ? h->Hs : nullptr, h->Y, h->slot_of, a.gates, T,
+                                 K, d, static_cast<bf16*>(a.h), h->num_sms, s));
+  h->launches += 1;
+  CUDA_TRY(mark(7));
+  if (timing) h->timed_forwards += 1;
+  return DSMOE_OK;
+}
+
+}  // namespace
+
+DSMOE_EXPORT dsmoe_status dsmoe_forward(dsmoe_handle* h, int32_t T, const void* x, const int32_t* token_ids,
+                                        const void* W_router, const float* b, const void* W_gate, const void* W_up,
+                                        const void* W_down, const void* Ws_gate, const void* Ws_up,
+                                        const void* Ws_down, void* h_out, int32_t* topk_idx, float* gates,
+                                        int32_t* counts, float* f, float* P, float* P_sum, float* scores_dbg,
+                                        void* stream) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  FwdArgs a{T, x, W_router, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, token_ids, b, h_out, topk_idx, gates,
+            counts, f, P, P_sum, scores_dbg};
+  dsmoe_status st = check_forward(h, a);
+  if (st != DSMOE_OK) return st;
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
+  return run_forward(h, a, static_cast<cudaStream_t>(stream));
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_forward_host(dsmoe_handle* h, int32_t T, const void* x_host,
+                                             const int32_t* token_ids_host, const void* W_router, const float* b,
+                                             const void* W_gate, const void* W_up, const void* W_down,
+                                             const void* Ws_gate, const void* Ws_up, const void* Ws_down,
+                                             void* h_host, int32_t* topk_idx_host, float* gates_host,
+                                             int32_t* counts_host, float* f_host, float* P_host, void* stream) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  const dsmoe_cfg& c = h->cfg;
+  if (T < 0) return fail(DSMOE_ERR_INVALID_ARG, "T = %d is negative", T);
+  if (T > c.max_tokens) return fail(DSMOE_ERR_WORKSPACE, "T = %d exceeds max_tokens = %d", T, c.max_tokens);
+  if (!counts_host || !f_host || !P_host) return fail(DSMOE_ERR_INVALID_ARG, "counts, f and P are required");
+  if (T > 0 && (!x_host || !h_host || !topk_idx_host || !gates_host))
+    return fail(DSMOE_ERR_INVALID_ARG, "x, h, topk_idx and gates are required");
+  const bool hash = c.score == DSMOE_ROUTE_HASH;
+  if (T > 0 && hash && !token_ids_host) return fail(DSMOE_ERR_INVALID_ARG, "hash routing needs token_ids");
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t xb = static_cast<size_t>(T) * c.d_model * 2, sb = static_cast<size_t>(T) * c.top_k * 4,
+               nb = static_cast<size_t>(c.n_routed) * 4;
+  if (T > 0) {
+    CUDA_TRY(cudaMemcpyAsync(h->x_stage, x_host, xb, cudaMemcpyHostToDevice, s));
+    if (hash) CUDA_TRY(cudaMemcpyAsync(h->ids_stage, token_ids_host, static_cast<size_t>(T) * 4, cudaMemcpyHostToDevice, s));
+  }
+  FwdArgs a{T, h->x_stage, W_router, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, hash ? h->ids_stage : nullptr,
+            b, h->h_stage, h->topk_stage, h->gates_stage, h->counts_stage, h->f_stage, h->P_stage, nullptr, nullptr};
+  dsmoe_status st = check_forward(h, a);
+  if (st != DSMOE_OK) return st;
+  st = run_forward(h, a, s);
+  if (st != DSMOE_OK) return st;
+  if (T > 0) {
+    CUDA_TRY(cudaMemcpyAsync(h_host, h->h_stage, xb, cudaMemcpyDeviceToHost, s));
+    CUDA_TRY(cudaMemcpyAsync(topk_idx_host, h->topk_stage, sb, cudaMemcpyDeviceToHost, s));
+    CUDA_TRY(cudaMemcpyAsync(gates_host, h->gates_stage, sb, cudaMemcpyDeviceToHost, s));
+  }
+  CUDA_TRY(cudaMemcpyAsync(counts_host, h->counts_stage, nb, cudaMemcpyDeviceToHost, s));
+  CUDA_TRY(cudaMemcpyAsync(f_host, h->f_stage, nb, cudaMemcpyDeviceToHost, s));
+  CUDA_TRY(cudaMemcpyAsync(P_host, h->P_stage, nb, cudaMemcpyDeviceToHost, s));
+  CUDA_TRY(cudaStreamSynchronize(s));
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_balance_stats(dsmoe_handle* h, int64_t T_total, const int32_t* counts,
+                                              const float* P_sum, float* f, float* P, void* stream) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  if (T_total < 0) return fail(DSMOE_ERR_INVALID_ARG, "T_total is negative");
+  if (!counts || !P_sum || !f || !P) return fail(DSMOE_ERR_INVALID_ARG, "counts, P_sum, f and P are required");
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
+  CUDA_TRY(dsmoe::launch_balance_stats(counts, P_sum, T_total, h->cfg.n_routed, h->cfg.top_k, f, P,
+                                       static_cast<cudaStream_t>(stream)));
+  h->launches += 1;
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_get_status(dsmoe_handle* h) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  DeviceGuard g(h->device);
+  CUDA_TRY(cudaDeviceSynchronize());
+  uint32_t v = 0;
+  CUDA_TRY(cudaMemcpy(&v, h->status, 4, cudaMemcpyDeviceToHost));
+  CUDA_TRY(cudaMemset(h->status, 0, 4));
+  if (v & (dsmoe::kStatusTimeoutProducer | dsmoe::kStatusTimeoutMma | dsmoe::kStatusTimeoutEpilogue |
+           dsmoe::kStatusTimeoutDrain))
+    return fail(DSMOE_ERR_DEVICE_TIMEOUT, "device status word 0x%x", v);
+  if (v) return fail(DSMOE_ERR_INVALID_ARG, "device status word 0x%x (out-of-range index)", v);
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_set_wait_limit(dsmoe_handle* h, uint64_t ns) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  h->wait_ns = ns;
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_set_timing(dsmoe_handle* h, int32_t enable) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  h->timing = enable != 0;
+  h->timed_forwards = 0;
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_stage_times(dsmoe_handle* h, float* ms, int32_t max_n, int32_t* n) {
+  if (!h || !ms || !n) return fail(DSMOE_ERR_INVALID_ARG, "NULL argument");
+  *n = 0;
+  if (h->timed_forwards == 0) return fail(DSMOE_ERR_INVALID_ARG, "no timed forward recorded (enable timing first)");
+  DeviceGuard g(h->device);
+  const int kept = h->timed_forwards < kTimingSlots ? h->timed_forwards : kTimingSlots;
+  const int cnt = max_n < kNumStages ? max_n : kNumStages;
+  for (int i = 0; i < cnt; ++i) ms[i] = 0.f;
+  for (int f = 0; f < kept; ++f) {
+    cudaEvent_t* evs = h->ev[(h->timed_forwards - 1 - f) % kTimingSlots];
+    CUDA_TRY(cudaEventSynchronize(evs[kNumStages]));
+    for (int i = 0; i < cnt; ++i) {
+      float v = 0.f;
+      CUDA_TRY(cudaEventElapsedTime(&v, evs[i], evs[i + 1]));
+      ms[i] += v / kept;
+    }
+  }
+  *n = cnt;
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT const char* dsmoe_stage_name(int32_t i) {
+  return (i >= 0 && i < kNumStages) ? kStageNames[i] : nullptr;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_launch_count(dsmoe_handle* h, int64_t* n) {
+  if (!h || !n) return fail(DSMOE_ERR_INVALID_ARG, "NULL argument");
+  *n = h->launches;
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_workspace_tensor(dsmoe_handle* h, const char* name, void** ptr, int64_t* rows,
+                                                 int64_t* cols) {
+  if (!h || !name || !ptr || !rows || !cols) return fail(DSMOE_ERR_INVALID_ARG, "NULL argument");
+  const dsmoe_cfg& c = h->cfg;
+  const int64_t T = c.max_tokens, S = T * c.top_k;
+  const bool hash = c.score == DSMOE_ROUTE_HASH;
+  struct Entry {
+    const char* n;
+    void* p;
+    int64_t r, k;
+    bool present;
+  } table[] = {
+      {"logits", h->logits, T, c.n_routed, !hash},
+      {"offsets", h->offsets, 1, c.n_routed + 1, true},
+      {"slot_of", h->slot_of, T, c.top_k, true},
+      {"Xp", h->Xp, S, c.d_model, true},
+      {"A1", h->A1, S, c.d_ff, true},
+      {"A1s", h->A1s, T, static_cast<int64_t>(c.n_shared) * c.d_ff_shared, c.n_shared > 0},
+      {"Y", h->Y, S, c.d_model, true},
+      {"Hs", h->Hs, T, c.d_model, c.n_shared > 0},
+  };
+  for (const Entry& e : table) {
+    if (strcmp(e.n, name) == 0) {
+      if (!e.present) return fail(DSMOE_ERR_INVALID_ARG, "this configuration has no %s buffer", name);
+      *ptr = e.p;
+      *rows = e.r;
+      *cols = e.k;
+      return DSMOE_OK;
+    }
+  }
+  return fail(DSMOE_ERR_INVALID_ARG, "unknown workspace buffer '%s'", name);
+}

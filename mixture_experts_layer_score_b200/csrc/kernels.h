@@ -1,0 +1,108 @@
+// kernels.h -- host-side launchers of the dsmoe kernels (internal to libdsmoe.so).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dsmoe {
+
+using bf16 = __nv_bfloat16;
+
+// Bits of the device status word.
+enum : uint32_t {
+  kStatusTimeoutProducer = 1u << 0,
+  kStatusTimeoutMma = 1u << 1,
+  kStatusTimeoutEpilogue = 1u << 2,
+  kStatusTimeoutDrain = 1u << 3,
+  kStatusBadIndex = 1u << 4,
+};
+
+
+// ---------------------------------------------------------------- router (router.cu)
+// logits[t, i] = sum_k x[t,k] W_router[i,k] (+ b[i] when bias_in_logits), fp32.
+cudaError_t launch_router_logits(const bf16* x, const bf16* W_router, const float* b, int bias_in_logits,
+                                 int T, int N, int d, float* logits, cudaStream_t s);
+
+struct SelectArgs {
+  const float* logits;   // [T, N]
+  const float* b;        // [N] or nullptr
+  int T, N, K;
+  int score;             // dsmoe_score
+  int bias_select;       // selection-only bias
+  int renormalize;
+  int32_t* topk_idx;     // [T, K]
+  float* gates;          // [T, K]
+  int32_t* counts;       // [N], accumulated with atomics (zeroed by the caller)
+  float* P_part;         // [gridDim.x, N] per-block partial score sums
+  float* scores_dbg;     // [T, N] or nullptr
+  uint32_t* status;
+};
+// Scores, top-K' selection, gates and per-block statistics partials; returns the grid size used.
+cudaError_t launch_select(const SelectArgs& a, int grid, cudaStream_t s);
+int select_grid(int T, int num_sms);
+
+cudaError_t launch_hash_route(const int32_t* token_ids, int T, int N, uint32_t mult, uint32_t mod,
+                              int32_t* topk_idx, float* gates, int32_t* counts, uint32_t* status,
+                              cudaStream_t s);
+
+// ---------------------------------------------------------------- routing tables (permute.cu)
+struct ScanArgs {
+  const int32_t* counts_ws;  // [N]
+  const float* P_part;       // [n_part, N] or nullptr (hash routing)
+  int n_part, N, K;
+  int64_t T;                 // tokens the statistics are taken over
+  int32_t* counts;           // [N] out
+  float* f;                  // [N] out
+  float* P;                  // [N] out
+  float* P_sum;              // [N] out or nullptr
+  int32_t* offsets;          // [N+1] out, or nullptr
+  int32_t* cursor;           // [N] zeroed, or nullptr
+};
+cudaError_t launch_scan_stats(const ScanArgs& a, cudaStream_t s);
+
+// Balance statistics from already-reduced counts and score sums.
+cudaError_t launch_balance_stats(const int32_t* counts, const float* P_sum, int64_t T, int N, int K,
+                                 float* f, float* P, cudaStream_t s);
+
+// slot positions + gather of token rows into expert-contiguous order.
+cudaError_t launch_permute_gather(const bf16* x, const int32_t* topk_idx, const int32_t* offsets,
+                                  int32_t* cursor, int T, int K, int N, int d, int32_t* slot_of, bf16* Xp,
+                                  uint32_t* status, int num_sms, cudaStream_t s);
+
+// ---------------------------------------------------------------- combine (combine.cu)
+// h = base + sum_k gates[t,k] Y[slot_of[t,k]], where base is Hs (fp32 x + shared experts)
+// when Hs is not null, else x.
+cudaError_t launch_combine(const bf16* x, const float* Hs, const bf16* Y, const int32_t* slot_of,
+                           const float* gates, int T, int K, int d, bf16* h, int num_sms, cudaStream_t s);
+
+// ---------------------------------------------------------------- grouped GEMM (gemm_sm100.cu)
+struct GemmArgs {
+  CUtensorMap a_routed;   // 2D [rows, K] activations of routed slots, box (64, 128)
+  CUtensorMap a_shared;   // 2D [T, K_shared] activations of the shared groups, box (64, 128)
+  CUtensorMap b0_routed;  // 3D (K, rows, experts): gate (SwiGLU) or down (plain) weights
+  CUtensorMap b1_routed;  // 3D up-projection weights (SwiGLU only)
+  CUtensorMap b0_shared;
+  CUtensorMap b1_shared;
+  const int32_t* offsets;         // [n_routed + 1] slot offset of each routed expert
+  int32_t n_routed;               // routed groups
+  int32_t n_shared_groups;        // shared groups (tiles run before the routed ones)
+  int32_t m_shared;               // rows of every shared group (T)
+  int32_t n_tiles_routed, n_tiles_shared;  // output tiles along N
+  int32_t kb_routed, kb_shared;            // 64-wide K blocks per tile
+  int32_t kb_per_b_expert_shared;          // shared B switches expert every this many K blocks
+  int32_t n_valid_routed, n_valid_shared;  // valid output columns
+  bf16* out_routed;
+  int64_t ld_routed;
+  bf16* out_shared;               // bf16 output of the shared groups (gate/up GEMM)
+  float* out_shared_f32;          // fp32 output of the shared group + residual (down GEMM)
+  const bf16* residual;           // [m_shared, ld_shared] added to out_shared_f32
+  int64_t ld_shared;
+  int32_t shared_col_stride;      // shared group g writes at column g * shared_col_stride
+  uint32_t* status;
+  uint64_t wait_limit_ns;
+};
+cudaError_t launch_grouped_gemm(bool swiglu, const GemmArgs& a, int grid, cudaStream_t s);
+
+}  // namespace dsmoe

@@ -1,0 +1,283 @@
+// router.cu -- router affinity, scoring, top-K' selection and gates.
+//
+// Affinity l[t,i] = u_t . e_i ("MoE architecture: how DeepSeek achieves more",
+// section 2: G(x) = Softmax(W_g x)); scores softmax / sigmoid / sqrt(softplus)
+// (DeepSeek-V4 book ch. 2, section 2); selection key s + b with the bias deciding
+// selection only (same chapter, section 3); gates g = s or s / sum_selected s;
+// hash routing expert = token_id * mult mod N (same chapter, section 5).
+#include <float.h>
+#include <math.h>
+
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace dsmoe {
+
+// --------------------------------------------------------------------------------------
+// router logits on CUDA cores: a 64 tokens x 64 experts tile per CTA, 4x4 per thread,
+// fp32 FMA accumulation in ascending k.
+// --------------------------------------------------------------------------------------
+namespace {
+constexpr int kRTM = 64, kRTN = 64, kRTK = 32;
+
+__global__ void __launch_bounds__(256) router_logits_kernel(const bf16* __restrict__ x,
+                                                            const bf16* __restrict__ W,
+                                                            const float* __restrict__ b, int bias_in_logits,
+                                                            int T, int N, int d, float* __restrict__ logits) {
+  __shared__ __align__(16) float xs[kRTK][kRTM + 4];
+  __shared__ __align__(16) float ws[kRTK][kRTN + 4];
+  const int t0 = blockIdx.x * kRTM, n0 = blockIdx.y * kRTN;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int lr = tid >> 2, lc = (tid & 3) * 8;  // loader: row, first column of 8
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+
+  for (int k0 = 0; k0 < d; k0 += kRTK) {
+    uint4 vx = make_uint4(0, 0, 0, 0), vw = make_uint4(0, 0, 0, 0);
+    if (t0 + lr < T) vx = *reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t0 + lr) * d + k0 + lc);
+    if (n0 + lr < N) vw = *reinterpret_cast<const uint4*>(W + static_cast<int64_t>(n0 + lr) * d + k0 + lc);
+    const uint32_t ux[4] = {vx.x, vx.y, vx.z, vx.w}, uw[4] = {vw.x, vw.y, vw.z, vw.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 fx = unpack_bf16x2(ux[j]), fw = unpack_bf16x2(uw[j]);
+      xs[lc + 2 * j][lr] = fx.x;
+      xs[lc + 2 * j + 1][lr] = fx.y;
+      ws[lc + 2 * j][lr] = fw.x;
+      ws[lc + 2 * j + 1][lr] = fw.y;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < kRTK; ++kk) {
+      const float4 a = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
+      const float4 w = *reinterpret_cast<const float4*>(&ws[kk][tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], wv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + ty * 4 + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx * 4 + j;
+      if (n < N) logits[static_cast<int64_t>(t) * N + n] = acc[i][j] + (bias_in_logits ? b[n] : 0.f);
+    }
+  }
+}
+}  // namespace
+
+cudaError_t launch_router_logits(const bf16* x, const bf16* W_router, const float* b, int bias_in_logits,
+                                 int T, int N, int d, float* logits, cudaStream_t s) {
+  dim3 grid((T + kRTM - 1) / kRTM, (N + kRTN - 1) / kRTN);
+  router_logits_kernel<<<grid, 256, 0, s>>>(x, W_router, b, bias_in_logits, T, N, d, logits);
+  return cudaGetLastError();
+}
+
+// --------------------------------------------------------------------------------------
+// scores + top-K' + gates + statistics partials: one warp per token, lane j owns experts
+// j, j+32, ... (kNPL per lane). Selection is K' rounds of a warp arg-max over the keys
+// not yet taken; ties go to the lower expert index.
+// --------------------------------------------------------------------------------------
+namespace {
+constexpr int kSelWarps = 8;
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float score_sigmoid(float l) { return 1.f / (1.f + expf(-l)); }
+// sqrt(log(1 + e^l)) through log(1+e^l) = max(l,0) + log1p(e^{-|l|}).
+__device__ __forceinline__ float score_sqrt_softplus(float l) {
+  return sqrtf(fmaxf(l, 0.f) + log1pf(expf(-fabsf(l))));
+}
+
+template <int kNPL>
+__global__ void __launch_bounds__(kSelWarps * 32) select_kernel(const SelectArgs a) {
+  __shared__ float red[kSelWarps][kNPL * 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = a.N, K = a.K;
+  float pacc[kNPL];
+  float bias[kNPL];
+#pragma unroll
+  for (int j = 0; j < kNPL; ++j) {
+    pacc[j] = 0.f;
+    const int i = lane + 32 * j;
+    bias[j] = (a.bias_select && i < N) ? a.b[i] : 0.f;
+  }
+  const int gw = blockIdx.x * kSelWarps + warp, nw = gridDim.x * kSelWarps;
+  for (int t = gw; t < a.T; t += nw) {
+    const float* lrow = a.logits + static_cast<int64_t>(t) * N;
+    float s[kNPL];
+#pragma unroll
+    for (int j = 0; j < kNPL; ++j) {
+      const int i = lane + 32 * j;
+      s[j] = (i < N) ? lrow[i] : -INFINITY;
+    }
+    if (a.score == 0) {  // softmax over the routed experts
+      float m = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < kNPL; ++j) m = fmaxf(m, s[j]);
+      m = warp_max(m);
+      float z = 0.f;
+#pragma unroll
+      for (int j = 0; j < kNPL; ++j) {
+        s[j] = (lane + 32 * j < N) ? expf(s[j] - m) : 0.f;
+        z += s[j];
+      }
+      z = warp_sum(z);
+      const float inv = 1.f / z;
+#pragma unroll
+      for (int j = 0; j < kNPL; ++j) s[j] *= inv;
+    } else if (a.score == 1) {
+#pragma unroll
+      for (int j = 0; j < kNPL; ++j) s[j] = (lane + 32 * j < N) ? score_sigmoid(s[j]) : 0.f;
+    } else {
+#pragma unroll
+      for (int j = 0; j < kNPL; ++j) s[j] = (lane + 32 * j < N) ? score_sqrt_softplus(s[j]) : 0.f;
+    }
+    // selection keys; NaN keys rank last
+    float key[kNPL];
+#pragma unroll
+    for (int j = 0; j < kNPL; ++j) {
+      const float kv = s[j] + bias[j];
+      key[j] = (lane + 32 * j < N && !isnan(kv)) ? kv : -INFINITY;
+    }
+    uint32_t taken = 0;
+    int my_idx = 0;
+    float my_s = 0.f;
+    for (int r = 0; r < K; ++r) {
+      float bk = -INFINITY;
+      int bi = 0x7fffffff;
+      float bs = 0.f;
+#pragma unroll
+      for (int j = 0; j < kNPL; ++j) {
+        const int i = lane + 32 * j;
+        const bool cand = (i < N) && !((taken >> j) & 1u);
+        if (cand && (key[j] > bk || (key[j] == bk && i < bi))) {
+          bk = key[j];
+          bi = i;
+          bs = s[j];
+        }
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        const float os = __shfl_xor_sync(0xffffffffu, bs, o);
+        if (ok > bk || (ok == bk && oi < bi)) {
+          bk = ok;
+          bi = oi;
+          bs = os;
+        }
+      }
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      if (lane == r) {
+        my_idx = bi;
+        my_s = bs;
+      }
+    }
+    float g = my_s;
+    if (a.renormalize) {
+      const float z = warp_sum(lane < K ? my_s : 0.f);
+      g = my_s / fmaxf(z, FLT_MIN);
+    }
+    if (lane < K) {
+      if (my_idx < 0 || my_idx >= N) {  // cannot happen for K <= N; recorded, never dereferenced
+        atomicOr(a.status, kStatusBadIndex);
+        my_idx = 0;
+      }
+      a.topk_idx[static_cast<int64_t>(t) * K + lane] = my_idx;
+      a.gates[static_cast<int64_t>(t) * K + lane] = g;
+      atomicAdd(&a.counts[my_idx], 1);
+    }
+#pragma unroll
+    for (int j = 0; j < kNPL; ++j) pacc[j] += s[j];
+    if (a.scores_dbg) {
+      float* srow = a.scores_dbg + static_cast<int64_t>(t) * N;
+#pragma unroll
+      for (int j = 0; j < kNPL; ++j)
+        if (lane + 32 * j < N) srow[lane + 32 * j] = s[j];
+    }
+  }
+  // per-block partial sums of the scores, reduced over warps in a fixed order
+#pragma unroll
+  for (int j = 0; j < kNPL; ++j) red[warp][lane + 32 * j] = pacc[j];
+  __syncthreads();
+  for (int i = threadIdx.x; i < N; i += blockDim.x) {
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kSelWarps; ++w) v += red[w][i];
+    a.P_part[static_cast<int64_t>(blockIdx.x) * N + i] = v;
+  }
+}
+}  // namespace
+
+int select_grid(int T, int num_sms) {
+  int g = (T + kSelWarps - 1) / kSelWarps;
+  const int cap = 4 * num_sms;
+  if (g > cap) g = cap;
+  if (g < 1) g = 1;
+  return g;
+}
+
+cudaError_t launch_select(const SelectArgs& a, int grid, cudaStream_t s) {
+  const int npl = (a.N + 31) / 32;
+  const dim3 blk(kSelWarps * 32);
+  if (npl <= 1) select_kernel<1><<<grid, blk, 0, s>>>(a);
+  else if (npl <= 2) select_kernel<2><<<grid, blk, 0, s>>>(a);
+  else if (npl <= 4) select_kernel<4><<<grid, blk, 0, s>>>(a);
+  else if (npl <= 8) select_kernel<8><<<grid, blk, 0, s>>>(a);
+  else if (npl <= 12) select_kernel<12><<<grid, blk, 0, s>>>(a);
+  else select_kernel<16><<<grid, blk, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+// --------------------------------------------------------------------------------------
+// hash routing: one expert per token, gate 1. The product is taken in 64 bits (no wrap).
+// --------------------------------------------------------------------------------------
+namespace {
+__global__ void hash_route_kernel(const int32_t* __restrict__ ids, int T, int N, uint32_t mult, uint32_t mod,
+                                  int32_t* __restrict__ topk_idx, float* __restrict__ gates,
+                                  int32_t* __restrict__ counts, uint32_t* status) {
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < T; t += gridDim.x * blockDim.x) {
+    const int32_t id = ids[t];
+    int e = 0;
+    if (id < 0) {
+      atomicOr(status, kStatusBadIndex);
+    } else {
+      e = static_cast<int>((static_cast<uint64_t>(id) * mult) % mod);
+    }
+    if (e >= N) e = 0;
+    topk_idx[t] = e;
+    gates[t] = 1.f;
+    atomicAdd(&counts[e], 1);
+  }
+}
+}  // namespace
+
+cudaError_t launch_hash_route(const int32_t* token_ids, int T, int N, uint32_t mult, uint32_t mod,
+                              int32_t* topk_idx, float* gates, int32_t* counts, uint32_t* status,
+                              cudaStream_t s) {
+  const int blk = 256;
+  int grid = (T + blk - 1) / blk;
+  if (grid < 1) grid = 1;
+  hash_route_kernel<<<grid, blk, 0, s>>>(token_ids, T, N, mult, mod, topk_idx, gates, counts, status);
+  return cudaGetLastError();
+}
+
+}  // namespace dsmoe

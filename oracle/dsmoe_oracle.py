@@ -222,10 +222,13 @@ def swiglu_ffn(U, W_gate, W_up, W_down) -> np.ndarray:
     three-matrix SwiGLU form ([MoE-learn], parameter-count snippet); no biases.
     Weights use the nn.Linear layout [out, in].
     """
+    return swiglu_hidden(U, W_gate, W_up) @ _as_f64(W_down).T
+
+
+def swiglu_hidden(U, W_gate, W_up) -> np.ndarray:
+    """The expert's hidden activation SiLU(W_gate u) * (W_up u) for rows U [m, d]."""
     U = _as_f64(U)
-    Wg, Wu, Wd = _as_f64(W_gate), _as_f64(W_up), _as_f64(W_down)
-    Z = silu(U @ Wg.T) * (U @ Wu.T)
-    return Z @ Wd.T
+    return silu(U @ _as_f64(W_gate).T) * (U @ _as_f64(W_up).T)
 
 
 def moe_layer(x, idx, gates, routed_expert: Callable[[int], Tuple], shared_experts: Sequence[Tuple],
