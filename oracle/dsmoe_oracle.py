@@ -291,3 +291,80 @@ def forward(cfg, inputs: Dict, rows: Optional[Iterable[int]] = None,
 def combinations(n: int, k: int) -> int:
     """Number of ways a router can pick k of n experts, C(n, k) ([DSMoE] segmentation example)."""
     return math.comb(n, k)
+
+
+# ----------------------------------------------------------------------------------------
+# balance control on top of the statistics
+# ----------------------------------------------------------------------------------------
+def expert_balance_loss(f, P, alpha1: float) -> float:
+    """L_ExpBal = alpha_1 * (1/N') * sum_i f_i P_i  ([DSMoE], "Expert-level balance loss").
+
+    Reading: the page writes the 1/N' factor in front of the sum; it is kept as written.
+    """
+    f = np.asarray(f, dtype=np.float64)
+    P = np.asarray(P, dtype=np.float64)
+    return float(alpha1 * (f * P).sum() / f.shape[0])
+
+
+def device_balance(f, P, group_of, n_groups: int, alpha2: float):
+    """Device-level balance ([DSMoE], "Device-level balance loss").
+
+    The routed experts are split into D groups E_1..E_D (group_of[i] = the group of
+    expert i); f'_d = (1/|E_d|) sum_{j in E_d} f_j, P'_d = sum_{j in E_d} P_j and
+    L_DevBal = alpha_2 * sum_d f'_d P'_d. Returns (f', P', L_DevBal).
+    """
+    f = np.asarray(f, dtype=np.float64)
+    P = np.asarray(P, dtype=np.float64)
+    g = np.asarray(group_of)
+    f_dev = np.zeros(n_groups)
+    P_dev = np.zeros(n_groups)
+    size = np.zeros(n_groups)
+    for i in range(f.shape[0]):
+        f_dev[g[i]] += f[i]
+        P_dev[g[i]] += P[i]
+        size[g[i]] += 1
+    f_dev = np.where(size > 0, f_dev / np.maximum(size, 1), 0.0)
+    return f_dev, P_dev, float(alpha2 * (f_dev * P_dev).sum())
+
+
+def classic_balance_loss(counts, P, top_k: int, alpha: float) -> float:
+    """L = alpha * E * sum_i f_i P_i with f_i the fraction of routed assignments that went to
+    expert i ("MoE architecture", section 6). Reading: with K' experts per token the
+    fraction is counts_i / (K' T), so sum_i f_i = 1 as in the top-1 form."""
+    c = np.asarray(counts, dtype=np.float64)
+    E = c.shape[0]
+    frac = c / c.sum()
+    return float(alpha * E * (frac * np.asarray(P, dtype=np.float64)).sum())
+
+
+def sequence_balance(idx, s, seq_len: int, n_routed: int, beta: float):
+    """Sequence-wise balance ([V4-ch2] section 3): for each sequence (consecutive runs of
+    seq_len tokens), f_i^seq = fraction of the sequence's tokens that selected expert i and
+    p_i^seq = the mean router score of expert i over the sequence; the loss of a sequence is
+    beta * sum_i f_i^seq p_i^seq. Reading: the batch loss is the mean over its sequences.
+    Returns (f_seq [S, N'], p_seq [S, N'], loss)."""
+    idx = np.asarray(idx)
+    s = np.asarray(s, dtype=np.float64)
+    T = idx.shape[0]
+    S = T // seq_len
+    f_seq = np.zeros((S, n_routed))
+    p_seq = np.zeros((S, n_routed))
+    for q in range(S):
+        rows = range(q * seq_len, (q + 1) * seq_len)
+        for t in rows:
+            for e in idx[t]:
+                f_seq[q, e] += 1.0
+        f_seq[q] /= seq_len
+        p_seq[q] = s[q * seq_len:(q + 1) * seq_len].mean(axis=0)
+    loss = float(beta * (f_seq * p_seq).sum(axis=1).mean()) if S else 0.0
+    return f_seq, p_seq, loss
+
+
+def bias_update(b, counts, T: int, top_k: int, alpha: float) -> np.ndarray:
+    """Auxiliary-loss-free bias update b_i <- b_i + alpha * (f* - f_i) ([V4-ch2] section 3),
+    with f_i = counts_i / T the fraction of tokens that selected expert i and f* = K'/N'
+    its uniform value. An over-loaded expert's bias falls, an under-loaded one's rises
+    ("MoE architecture", section 6 sign rule)."""
+    b = np.asarray(b, dtype=np.float64)
+    c = np.asarray(counts, dtype=np.float64)
+    return b + alpha * (top_k / c.shape[0] - c / T)
