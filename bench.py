@@ -43,8 +43,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="v3_prefill")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=None, help="steps of the end-to-end leg (default: --steps)")
@@ -152,9 +152,6 @@ def cpu_oracle_throughput(cfg, x_cpu, b_cpu, W_router_cpu, token_ids_cpu, expert
         cache[e] = expert_source(e)
     shared = [expert_source(("s", s)) for s in range(cfg.n_shared)]
 
-    class _Routed(dict):
-        pass
-
     inp_w = dict(inp)
     inp_w["W_gate"] = {e: cache[e][0] for e in need}
     inp_w["W_up"] = {e: cache[e][1] for e in need}
@@ -254,7 +251,7 @@ def run_native(args, cfg):
             global_balance_stats(layer.handle, T_total, out["counts"], out["P_sum"], out["f"], out["P"],
                                  stream=stream)
 
-    for _ in range(max(args.warmup, 3 if args.warmup >= 3 else args.warmup)):
+    for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
     st = M.dsmoe_get_status(layer.handle)

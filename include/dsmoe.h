@@ -204,7 +204,8 @@ dsmoe_status dsmoe_launch_count(dsmoe_handle* h, int64_t* n);
 /*
  * Device address and shape of one intermediate buffer of the handle's workspace, for
  * tests and debugging; contents are those of the last forward on this handle:
- *   "logits"  fp32 [T, N']        router affinities (absent for hash routing)
+ *   "logits"  fp32 [T, N']        router affinities, written when the CUDA-core router
+ *                                 runs (T < 256); absent for hash routing
  *   "offsets" int32 [N'+1]        first slot of each expert's segment
  *   "slot_of" int32 [T, K']       slot holding token t's k-th expert row
  *   "Xp"      bf16 [T K', d]      token rows in expert-contiguous slot order

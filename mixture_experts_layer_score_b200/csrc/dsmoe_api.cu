@@ -29,6 +29,7 @@ const char* const kStageNames[kNumStages] = {"router", "select", "scan", "permut
                                              "combine"};
 constexpr int kSelectMaxBlocks = 1024;  // rows of the statistics partials
 constexpr int kTimingSlots = 64;        // forwards whose stage events are kept
+constexpr int kTcRouterMinTokens = 256; // below this the CUDA-core router spreads over more SMs
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;
 
 thread_local std::string g_last_error;
@@ -164,8 +165,10 @@ struct dsmoe_handle {
   int32_t *ids_stage, *topk_stage, *counts_stage;
   float *gates_stage, *f_stage, *P_stage;
   CUtensorMap tm_xp, tm_a1, tm_a1s;
-  const void* wkey[6] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
-  CUtensorMap tm_w[6];  // W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down
+  const void* wkey[7] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+  CUtensorMap tm_w[7];  // W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, W_router
+  int rt_chunks = 1, rt_nc = 16;
+  uint32_t rt_cols = 32;
   bool timing = false;
   int timed_forwards = 0;               // forwards recorded since timing was enabled
   cudaEvent_t ev[kTimingSlots][kNumStages + 1] = {};
@@ -265,6 +268,7 @@ DSMOE_EXPORT dsmoe_status dsmoe_create(const dsmoe_cfg* cfg, int32_t device, dsm
   if (h->cfg.score == DSMOE_ROUTE_HASH && h->cfg.hash_mod == 0) h->cfg.hash_mod = h->cfg.n_routed;
   h->device = device;
   h->num_sms = prop.multiProcessorCount;
+  dsmoe::router_tc_shape(cfg->n_routed, &h->rt_chunks, &h->rt_nc, &h->rt_cols);
   h->L = plan(h->cfg);
   cudaError_t e = cudaMalloc(&h->ws, h->L.total);
   if (e != cudaSuccess) {
@@ -379,6 +383,7 @@ const CUtensorMap* weight_map(dsmoe_handle* h, int which, const void* ptr, bool*
       case 3:
       case 4: r = map_3d(&h->tm_w[which], ptr, c.d_model, c.d_ff_shared, c.n_shared, 128); break;
       case 5: r = map_3d(&h->tm_w[which], ptr, c.d_ff_shared, c.d_model, c.n_shared, 256); break;
+      case 6: r = map_2d(&h->tm_w[which], ptr, c.d_model, c.n_routed, static_cast<uint32_t>(h->rt_nc)); break;
     }
     if (!r) {
       h->wkey[which] = nullptr;
@@ -427,6 +432,38 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
   if (hash) {
     CUDA_TRY(dsmoe::launch_hash_route(a.token_ids, T, N, c.hash_mult, c.hash_mod, a.topk_idx, a.gates, h->counts_ws,
                                       h->status, s));
+    h->launches += 1;
+    CUDA_TRY(mark(1));
+  } else if (T >= kTcRouterMinTokens) {
+    // tensor-core affinities with scoring, top-K', gates and partials in the epilogue
+    dsmoe::RouterTcArgs ra;
+    memset(&ra, 0, sizeof(ra));
+    const CUtensorMap* m_wr = weight_map(h, 6, a.W_router, &ok);
+    if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected the router tensor map");
+    ra.tm_x = m_x;
+    ra.tm_w = *m_wr;
+    ra.b = a.b;
+    ra.T = T;
+    ra.N = N;
+    ra.K = K;
+    ra.d = d;
+    ra.score = c.score;
+    ra.bias_select = c.bias_mode == DSMOE_BIAS_SELECT_ONLY;
+    ra.bias_in_logits = c.bias_mode == DSMOE_BIAS_IN_LOGITS;
+    ra.renormalize = c.renormalize;
+    ra.n_chunks = h->rt_chunks;
+    ra.nc = h->rt_nc;
+    ra.tmem_cols = h->rt_cols;
+    ra.topk_idx = a.topk_idx;
+    ra.gates = a.gates;
+    ra.counts = h->counts_ws;
+    ra.P_part = h->P_part;
+    ra.scores_dbg = a.scores_dbg;
+    ra.status = h->status;
+    ra.wait_limit_ns = h->wait_ns;
+    const int tiles = cdiv(T, 128);
+    sel_grid = tiles < h->num_sms ? tiles : h->num_sms;
+    CUDA_TRY(dsmoe::launch_router_tc(ra, sel_grid, s));
     h->launches += 1;
     CUDA_TRY(mark(1));
   } else {

@@ -7,20 +7,29 @@
 //   gate/up:  A1[r, n] = SiLU(sum_k X[r,k] W_gate[e,n,k]) * (sum_k X[r,k] W_up[e,n,k])
 //   down:     Y[r, n]  = sum_k A1[r,k] W_down[e,n,k]
 // The routed experts are groups of a variable number of rows (their segment of the
-// expert-contiguous slot order, read from the device-side offsets), the shared
-// experts are dense groups over all T tokens that run first.
+// expert-contiguous slot order, read from the device-side offsets); the shared experts
+// are dense groups over all T tokens that run first.
+//
+// Orientation: the MMA's M dimension is the weights' output features and its N
+// dimension is the group's tokens, D^T[feature, token] = W[feature, :] . X[token, :]^T.
+// A tile is 128 (gate/up: 128 gate + the same 128 up features; down: 2 x 128 output
+// features) by at most 128 tokens, and N is the tile's token count rounded up to 16,
+// so an expert's ragged last tile wastes at most 15 token columns of tensor work and
+// an expert with a handful of decode tokens costs N=16, not a 128-row tile.
 //
 // One CTA per SM, 192 threads in three roles:
-//   warp 0     TMA producer: streams 128x64 A tiles and 256x64 B tiles through a
-//              4-stage shared-memory ring (mbarrier full/empty pairs).
-//   warp 1     allocates 512 TMEM columns (two 128x256 fp32 accumulators) and issues
-//              tcgen05.mma (M=128, N=256, K=16) from one thread; commits free ring
-//              stages and publish finished accumulators.
-//   warps 2-5  epilogue: tcgen05.ld of the accumulator rows, SiLU(gate)*up (gate/up
-//              GEMM) or a plain conversion (down GEMM), bf16 stores; the second TMEM
+//   warp 0     TMA producer: per 64-wide K block a 256x64 weight tile (two 128-row
+//              halves) and a 128x64 token tile through a 4-stage shared-memory ring
+//              (mbarrier full/empty pairs).
+//   warp 1     allocates 512 TMEM columns (two accumulators of 2 x 128 columns) and
+//              issues tcgen05.mma (M=128, N=16..128, K=16) from one thread, two chains
+//              (one per weight half) sharing the token tile; commits free ring stages
+//              and publish finished accumulators.
+//   warps 2-5  epilogue: thread f of TMEM lane f owns output feature f of both chains;
+//              it reads 16 token columns at a time with tcgen05.ld and stores one
+//              element per token (consecutive features across a warp, so each store
+//              instruction writes 32 consecutive features of one row). The second TMEM
 //              accumulator lets the next tile's MMAs overlap this epilogue.
-// For the gate/up GEMM the 256-row B tile is [128 gate rows | 128 up rows] of the same
-// output features, so one MMA chain yields both halves side by side in TMEM.
 //
 // Every wait is bounded (wait_limit_ns); a role that gives up raises a CTA-wide abort
 // flag and a bit of the device status word, the CTA lets in-flight TMA loads and MMAs
@@ -31,9 +40,9 @@
 namespace dsmoe {
 
 namespace {
-constexpr int kBM = 128;        // output rows per tile (= TMEM lanes)
+constexpr int kBM = 128;        // tokens per tile (the MMA's N is this count rounded to 16)
 constexpr int kBK = 64;         // K per ring stage (one 128-byte swizzled row of bf16)
-constexpr int kMmaN = 256;      // N of each tcgen05.mma
+constexpr int kFeat = 128;      // output features per MMA chain (the MMA's M, TMEM lanes)
 constexpr int kMmaK = 16;       // K of each bf16 tcgen05.mma
 constexpr int kStages = 4;
 constexpr int kThreads = 192;
@@ -41,13 +50,13 @@ constexpr int kEpiThreads = 128;
 constexpr uint32_t kAccCols = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxGroups = 8 + 512;
-constexpr uint32_t kABytes = kBM * kBK * 2;    // 16 KB
-constexpr uint32_t kBBytes = kMmaN * kBK * 2;  // 32 KB
-constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr uint32_t kWBytes = 2 * kFeat * kBK * 2;  // 32 KB: two 128-row weight halves
+constexpr uint32_t kXBytes = kBM * kBK * 2;        // 16 KB: 128 token rows
+constexpr uint32_t kStageBytes = kWBytes + kXBytes;
 
-constexpr uint32_t kOffA = 0;
-constexpr uint32_t kOffB = kOffA + kStages * kABytes;
-constexpr uint32_t kOffBars = kOffB + kStages * kBBytes;
+constexpr uint32_t kOffW = 0;
+constexpr uint32_t kOffX = kOffW + kStages * kWBytes;
+constexpr uint32_t kOffBars = kOffX + kStages * kXBytes;
 constexpr uint32_t kNumBars = 2 * kStages + 2 + 2 + 1;
 constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
 constexpr uint32_t kOffTiles = kOffMisc + 16;
@@ -104,8 +113,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_addr(smem_raw) & 1023u)) & 1023u;
   uint8_t* base = smem_raw + pad;
-  uint8_t* sA = base + kOffA;
-  uint8_t* sB = base + kOffB;
+  uint8_t* sW = base + kOffW;
+  uint8_t* sX = base + kOffX;
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + kOffBars);
   uint64_t* full = bars;
   uint64_t* empty = bars + kStages;
@@ -187,9 +196,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
         const Tile t = decode_tile(a, tile_start, G, tile);
-        const CUtensorMap* ta = t.shared ? &a.a_shared : &a.a_routed;
-        const CUtensorMap* tb0 = t.shared ? &a.b0_shared : &a.b0_routed;
-        const CUtensorMap* tb1 = t.shared ? &a.b1_shared : &a.b1_routed;
+        const CUtensorMap* tx = t.shared ? &a.a_shared : &a.a_routed;
+        const CUtensorMap* tw0 = t.shared ? &a.b0_shared : &a.b0_routed;
+        const CUtensorMap* tw1 = t.shared ? &a.b1_shared : &a.b1_routed;
         const int kb_per = t.shared ? a.kb_per_b_expert_shared : t.kb_n;
         for (int kb = 0; kb < t.kb_n; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, a.wait_limit_ns, abort_flag)) {
@@ -197,15 +206,16 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
             break;
           }
           mbar_arrive_expect_tx(&full[stage], kStageBytes);
-          tma_load_2d(sA + stage * kABytes, ta, &full[stage], kb * kBK, t.row0);
           const int be = t.expert + kb / kb_per;
           const int bk = (kb % kb_per) * kBK;
-          if (kSwiGLU) {
-            tma_load_3d(sB + stage * kBBytes, tb0, &full[stage], bk, t.n_blk * (kMmaN / 2), be);
-            tma_load_3d(sB + stage * kBBytes + kBBytes / 2, tb1, &full[stage], bk, t.n_blk * (kMmaN / 2), be);
-          } else {
-            tma_load_3d(sB + stage * kBBytes, tb0, &full[stage], bk, t.n_blk * kMmaN, be);
+          uint8_t* w = sW + stage * kWBytes;
+          if (kSwiGLU) {  // [128 gate rows | the same 128 up rows]
+            tma_load_3d(w, tw0, &full[stage], bk, t.n_blk * kFeat, be);
+            tma_load_3d(w + kWBytes / 2, tw1, &full[stage], bk, t.n_blk * kFeat, be);
+          } else {        // 256 consecutive output rows
+            tma_load_3d(w, tw0, &full[stage], bk, t.n_blk * 2 * kFeat, be);
           }
+          tma_load_2d(sX + stage * kXBytes, tx, &full[stage], kb * kBK, t.row0);
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) {
@@ -222,13 +232,14 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------------ MMA issuer
-      const uint32_t idesc = idesc_bf16_f32(kBM, kMmaN);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       int it = 0;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++it) {
         const Tile t = decode_tile(a, tile_start, G, tile);
+        const int n_mma = (t.m_valid + 15) & ~15;  // tokens, rounded up to the MMA's N step
+        const uint32_t idesc = idesc_bf16_f32(kFeat, n_mma);
         const int acc = it & 1;
         const uint32_t acc_phase = (it >> 1) & 1;
         if (!mbar_wait_bounded(&acc_empty[acc], acc_phase ^ 1u, a.wait_limit_ns, abort_flag)) {
@@ -236,19 +247,23 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * kAccCols;
+        const uint32_t d0 = tmem_base + acc * kAccCols;
         for (int kb = 0; kb < t.kb_n; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, a.wait_limit_ns, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t ad = smem_desc_kmajor_sw128(smem_addr(sA + stage * kABytes));
-          const uint64_t bd = smem_desc_kmajor_sw128(smem_addr(sB + stage * kBBytes));
+          const uint64_t w0 = smem_desc_kmajor_sw128(smem_addr(sW + stage * kWBytes));
+          const uint64_t w1 = smem_desc_kmajor_sw128(smem_addr(sW + stage * kWBytes + kWBytes / 2));
+          const uint64_t xd = smem_desc_kmajor_sw128(smem_addr(sX + stage * kXBytes));
 #pragma unroll
-          for (int k = 0; k < kBK / kMmaK; ++k)
-            mma_bf16_ss(d_tmem, ad + static_cast<uint64_t>(2 * k), bd + static_cast<uint64_t>(2 * k), idesc,
-                        (kb | k) ? 1u : 0u);
+          for (int k = 0; k < kBK / kMmaK; ++k) {
+            const uint64_t dk = static_cast<uint64_t>(2 * k);
+            const uint32_t accum = (kb | k) ? 1u : 0u;
+            mma_bf16_ss(d0, w0 + dk, xd + dk, idesc, accum);
+            mma_bf16_ss(d0 + kFeat, w1 + dk, xd + dk, idesc, accum);
+          }
           mma_commit(&empty[stage]);
           if (++stage == kStages) {
             stage = 0;
@@ -266,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
   } else {
     // -------------------------------------------------------------------- epilogue
     const int q = warp & 3;  // this warp may read TMEM lanes [32q, 32q+32)
-    const int r = q * 32 + lane;
+    const int f = q * 32 + lane;  // output feature of chain 0 (and of chain 1) owned by this thread
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
       const Tile t = decode_tile(a, tile_start, G, tile);
@@ -282,75 +297,64 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       }
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
-      const bool row_ok = r < t.m_valid;
-      bf16* out;
-      int n_valid;
-      if (t.shared) {
-        out = a.out_shared + static_cast<int64_t>(t.row0 + r) * a.ld_shared +
-              static_cast<int64_t>(t.group) * a.shared_col_stride;
-        n_valid = a.n_valid_shared;
-      } else {
-        out = a.out_routed + static_cast<int64_t>(t.row0 + r) * a.ld_routed;
-        n_valid = a.n_valid_routed;
-      }
+      const int n_valid = t.shared ? a.n_valid_shared : a.n_valid_routed;
+      const int64_t ld = t.shared ? a.ld_shared : a.ld_routed;
       if (kSwiGLU) {
+        const int feat = t.n_blk * kFeat + f;
+        const bool ok_f = feat < n_valid;
+        bf16* out = (t.shared ? a.out_shared + static_cast<int64_t>(t.group) * a.shared_col_stride : a.out_routed) +
+                    static_cast<int64_t>(t.row0) * ld + feat;
 #pragma unroll 1
-        for (int c = 0; c < kMmaN / 2; c += 16) {
+        for (int c = 0; c < t.m_valid; c += 16) {
           uint32_t gv[16], uv[16];
           tmem_ld16(tb + c, gv);
-          tmem_ld16(tb + kMmaN / 2 + c, uv);
+          tmem_ld16(tb + kFeat + c, uv);
           tmem_wait_ld();
-          const int col = t.n_blk * (kMmaN / 2) + c;
-          if (row_ok && col < n_valid) {
-            uint32_t pk[8];
+          if (ok_f) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float g0 = __uint_as_float(gv[2 * j]), g1 = __uint_as_float(gv[2 * j + 1]);
-              const float u0 = __uint_as_float(uv[2 * j]), u1 = __uint_as_float(uv[2 * j + 1]);
-              pk[j] = pack_bf16x2(silu(g0) * u0, silu(g1) * u1);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(out + col);
-            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            for (int j = 0; j < 16; ++j)
+              if (c + j < t.m_valid)
+                out[static_cast<int64_t>(c + j) * ld] =
+                    __float2bfloat16_rn(silu(__uint_as_float(gv[j])) * __uint_as_float(uv[j]));
           }
         }
       } else if (t.shared && a.out_shared_f32) {
         // shared experts of the down GEMM: fp32 row of (residual + sum of shared outputs)
-        float* o32 = a.out_shared_f32 + static_cast<int64_t>(t.row0 + r) * a.ld_shared;
-        const bf16* res = a.residual + static_cast<int64_t>(t.row0 + r) * a.ld_shared;
+        const int feat0 = t.n_blk * 2 * kFeat + f, feat1 = feat0 + kFeat;
+        const int64_t r0 = static_cast<int64_t>(t.row0) * ld;
 #pragma unroll 1
-        for (int c = 0; c < kMmaN; c += 16) {
-          uint32_t v[16];
-          tmem_ld16(tb + c, v);
+        for (int c = 0; c < t.m_valid; c += 16) {
+          uint32_t v0[16], v1[16];
+          tmem_ld16(tb + c, v0);
+          tmem_ld16(tb + kFeat + c, v1);
           tmem_wait_ld();
-          const int col = t.n_blk * kMmaN + c;
-          if (row_ok && col < n_valid) {
-            const uint4* r4 = reinterpret_cast<const uint4*>(res + col);
-            const uint4 q0 = r4[0], q1 = r4[1];
-            const uint32_t rw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-            float4* dst = reinterpret_cast<float4*>(o32 + col);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float2 a0 = unpack_bf16x2(rw[2 * j]), a1 = unpack_bf16x2(rw[2 * j + 1]);
-              dst[j] = make_float4(__uint_as_float(v[4 * j]) + a0.x, __uint_as_float(v[4 * j + 1]) + a0.y,
-                                   __uint_as_float(v[4 * j + 2]) + a1.x, __uint_as_float(v[4 * j + 3]) + a1.y);
+          for (int j = 0; j < 16; ++j) {
+            if (c + j < t.m_valid) {
+              const int64_t o = r0 + static_cast<int64_t>(c + j) * ld;
+              if (feat0 < n_valid)
+                a.out_shared_f32[o + feat0] = __uint_as_float(v0[j]) + __bfloat162float(a.residual[o + feat0]);
+              if (feat1 < n_valid)
+                a.out_shared_f32[o + feat1] = __uint_as_float(v1[j]) + __bfloat162float(a.residual[o + feat1]);
             }
           }
         }
       } else {
+        const int feat0 = t.n_blk * 2 * kFeat + f, feat1 = feat0 + kFeat;
+        bf16* out = (t.shared ? a.out_shared : a.out_routed) + static_cast<int64_t>(t.row0) * ld;
 #pragma unroll 1
-        for (int c = 0; c < kMmaN; c += 16) {
-          uint32_t v[16];
-          tmem_ld16(tb + c, v);
+        for (int c = 0; c < t.m_valid; c += 16) {
+          uint32_t v0[16], v1[16];
+          tmem_ld16(tb + c, v0);
+          tmem_ld16(tb + kFeat + c, v1);
           tmem_wait_ld();
-          const int col = t.n_blk * kMmaN + c;
-          if (row_ok && col < n_valid) {
-            uint32_t pk[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-            uint4* dst = reinterpret_cast<uint4*>(out + col);
-            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          for (int j = 0; j < 16; ++j) {
+            if (c + j < t.m_valid) {
+              bf16* o = out + static_cast<int64_t>(c + j) * ld;
+              if (feat0 < n_valid) o[feat0] = __float2bfloat16_rn(__uint_as_float(v0[j]));
+              if (feat1 < n_valid) o[feat1] = __float2bfloat16_rn(__uint_as_float(v1[j]));
+            }
           }
         }
       }

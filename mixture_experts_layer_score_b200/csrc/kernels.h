@@ -43,6 +43,27 @@ struct SelectArgs {
 cudaError_t launch_select(const SelectArgs& a, int grid, cudaStream_t s);
 int select_grid(int T, int num_sms);
 
+// Router on the tensor cores with scoring, top-K', gates and statistics partials fused
+// (router_sm100.cu). The B tile is n_chunks chunks of nc router rows (nc a multiple of
+// 16, at most 256); the accumulator takes tmem_cols TMEM columns.
+struct RouterTcArgs {
+  CUtensorMap tm_x;  // 2D [T, d] bf16, box (64, 128)
+  CUtensorMap tm_w;  // 2D [N', d] bf16, box (64, nc)
+  const float* b;    // [N'] or nullptr
+  int T, N, K, d, score, bias_select, bias_in_logits, renormalize;
+  int n_chunks, nc;
+  uint32_t tmem_cols;
+  int32_t* topk_idx;
+  float* gates;
+  int32_t* counts;     // [N'] accumulated with atomics (zeroed by the caller)
+  float* P_part;       // [gridDim.x, N'] per-CTA partial score sums
+  float* scores_dbg;   // [T, N'] or nullptr
+  uint32_t* status;
+  uint64_t wait_limit_ns;
+};
+void router_tc_shape(int N, int* n_chunks, int* nc, uint32_t* tmem_cols);
+cudaError_t launch_router_tc(const RouterTcArgs& a, int grid, cudaStream_t s);
+
 cudaError_t launch_hash_route(const int32_t* token_ids, int T, int N, uint32_t mult, uint32_t mod,
                               int32_t* topk_idx, float* gates, int32_t* counts, uint32_t* status,
                               cudaStream_t s);

@@ -20,10 +20,12 @@ pytestmark = pytest.mark.gpu
 if not torch.cuda.is_available():
     pytest.skip("no GPU", allow_module_level=True)
 
-CASES = [("tiny", 300), ("gshard_c", 700), ("ds2b", 900)]
+# T < 256 runs the CUDA-core router (logits kept in the workspace); larger T the
+# tensor-core router, whose scores are checked through scores_dbg.
+CASES = [("tiny", 300), ("tiny", 200), ("gshard_c", 700), ("ds2b", 900), ("v4_decode_t64", 64)]
 
 
-@pytest.mark.parametrize("name,T", CASES, ids=[c[0] for c in CASES])
+@pytest.mark.parametrize("name,T", CASES, ids=[f"{c[0]}-T{c[1]}" for c in CASES])
 def test_stages(name, T):
     cfg = W.get_config(name)
     gpu, cpu = make_case(cfg, T)
@@ -36,9 +38,12 @@ def test_stages(name, T):
     layer.close()
     K, N, S = cfg.top_k, cfg.n_routed, T * cfg.top_k
     x64 = O.bf16_bits_to_f64(cpu["x"])
-    # router logits (fp32 accumulation) against float64
+    # router: logits (CUDA-core path) or scores (both paths) against float64
     l_ref = O.router_logits(cpu["x"], cpu["W_router"], cpu.get("b"), cfg.bias_mode)
-    assert np.abs(ws["logits"][:T].numpy() - l_ref).max() < 1e-4
+    if T < 256:
+        assert np.abs(ws["logits"][:T].numpy() - l_ref).max() < 1e-4
+    s_ref = O.scores(l_ref, cfg.score)
+    assert np.abs(out["scores"].cpu().numpy() - s_ref).max() < 2e-5
     # offsets: exclusive scan of the counts
     counts = out["counts"].cpu().numpy()
     offs = ws["offsets"][0].numpy()
