@@ -219,6 +219,38 @@ dsmoe_status dsmoe_launch_count(dsmoe_handle* h, int64_t* n);
 dsmoe_status dsmoe_workspace_tensor(dsmoe_handle* h, const char* name, void** ptr, int64_t* rows,
                                     int64_t* cols);
 
+/*
+ * The routing stage with no allocation: router affinities, scores, top-K' experts,
+ * gates, expert counts, f_i and P_i for T tokens -- the outputs dsmoe_forward gives,
+ * up to fp32 rounding (experts whose keys tie within rounding may be picked or
+ * ordered differently) -- without a handle and without any device allocation.
+ *
+ * The pages have no counterpart to this entry point. It is for callers that cannot
+ * call cudaMalloc when they route a batch: code whose framework has already claimed
+ * all device memory through its own pool, plugins that must not touch the allocator
+ * while their host serves requests, or anything that cannot create a handle
+ * (dsmoe_create allocates a workspace). The caller passes inputs and outputs only:
+ *
+ *   cfg        layer configuration (host); T must not exceed cfg->max_tokens
+ *   x          bf16 [T, d], W_router bf16 [N', d], b fp32 [N'] (NULL iff no bias)
+ *   topk_idx   int32 [T, K'], gates fp32 [T, K'], counts int32 [N'], f fp32 [N'],
+ *              P fp32 [N'] -- device, caller-owned, fully overwritten
+ *
+ * Scratch: a fixed array of about 514 KiB inside the library's device image (each
+ * GPU that loads the library holds it until the process exits); it bounds N' to at
+ * most 512. Learned routing only: hash routing returns DSMOE_ERR_UNSUPPORTED, as
+ * does N' > 512; T > cfg->max_tokens returns DSMOE_ERR_WORKSPACE (dsmoe_last_error
+ * says which). The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call before
+ * any stream capture. Work runs on `stream` of the current device. Every call
+ * shares the array: each call clears the counters it needs on its stream first,
+ * and calls that overlap on the GPU (other streams or threads) race and must be
+ * serialised by the caller.
+ */
+dsmoe_status dsmoe_route_noalloc(const dsmoe_cfg* cfg, int32_t T, const void* x, const void* W_router,
+                                 const float* b, int32_t* topk_idx, float* gates, int32_t* counts, float* f,
+                                 float* P, void* stream);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

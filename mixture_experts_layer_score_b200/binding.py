@@ -25,6 +25,7 @@ ABI_FUNCTIONS = (
     "dsmoe_workspace_bytes", "dsmoe_create", "dsmoe_destroy", "dsmoe_forward", "dsmoe_forward_host",
     "dsmoe_balance_stats", "dsmoe_get_status", "dsmoe_set_wait_limit", "dsmoe_set_timing",
     "dsmoe_stage_times", "dsmoe_stage_name", "dsmoe_launch_count", "dsmoe_workspace_tensor",
+    "dsmoe_route_noalloc",
 )
 
 
@@ -68,6 +69,7 @@ def _load():
         "dsmoe_launch_count": (ctypes.c_int, [vp, ctypes.POINTER(i64)]),
         "dsmoe_workspace_tensor": (ctypes.c_int, [vp, ctypes.c_char_p, ctypes.POINTER(vp),
                                                   ctypes.POINTER(i64), ctypes.POINTER(i64)]),
+        "dsmoe_route_noalloc": (ctypes.c_int, [cfgp, i32] + [vp] * 8 + [vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -209,6 +211,14 @@ def dsmoe_launch_count(handle) -> int:
     n = ctypes.c_int64(0)
     _check(_lib.dsmoe_launch_count(handle, ctypes.byref(n)), "dsmoe_launch_count")
     return n.value
+
+
+def dsmoe_route_noalloc(cfg: DsmoeCfg, T, x, W_router, b, topk_idx, gates, counts, f, P, stream=None) -> None:
+    """The routing stage without a handle or any allocation (scratch is a fixed array in
+    the library); for callers that cannot allocate device memory when they route."""
+    st = _lib.dsmoe_route_noalloc(ctypes.byref(cfg), int(T), *[_ptr(t) for t in (
+        x, W_router, b, topk_idx, gates, counts, f, P)], _stream(stream))
+    _check(st, "dsmoe_route_noalloc")
 
 
 _WS_DTYPES = {"logits": "float32", "offsets": "int32", "slot_of": "int32", "Xp": "bfloat16",

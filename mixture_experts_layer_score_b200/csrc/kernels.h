@@ -126,4 +126,8 @@ struct GemmArgs {
 };
 cudaError_t launch_grouped_gemm(bool swiglu, const GemmArgs& a, int grid, cudaStream_t s);
 
+// ---------------------------------------------------------------- errors (dsmoe_api.cu)
+// Record the calling thread's last-error message (read back by dsmoe_last_error).
+void note_error(const char* fmt, ...);
+
 }  // namespace dsmoe
