@@ -62,6 +62,37 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+KERNEL_SOURCES = {"gemm_gate_up": "mixture_experts_layer_score_b200/csrc/gemm_sm100.cu",
+                  "gemm_down": "mixture_experts_layer_score_b200/csrc/gemm_sm100.cu",
+                  "router": "mixture_experts_layer_score_b200/csrc/router_sm100.cu"}
+
+
+def source_digest(stage):
+    import hashlib
+    path = os.path.join(ROOT, KERNEL_SOURCES[stage])
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def captured_traffic(stage, weight_bytes):
+    """DRAM bytes per launch of `stage` from the committed ncu summary
+    (profiles/ncu_dram_traffic.txt): the captured launch's DRAM read+write bytes divided by
+    the algorithmic weight bytes it streamed, scaled to this launch's weight bytes (the
+    capture runs a smaller case of the same kernel; its DRAM traffic is dominated by the
+    expert weights and grows with them). None when the kernel source changed since the
+    capture or no capture is recorded."""
+    path = os.path.join(ROOT, "profiles", "ncu_dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    digest = source_digest(stage)
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and not line.startswith("#") and parts[0] == stage and parts[1] == digest:
+                return float(parts[2]) / float(parts[3]) * weight_bytes
+    return None
+
+
 def config_block(cfg, n_gpus):
     return {"workload": cfg.name, "T_per_gpu": cfg.T, "global_batch": cfg.T * n_gpus, "d_model": cfg.d_model,
             "n_routed": cfg.n_routed, "top_k": cfg.top_k, "d_ff": cfg.d_ff, "n_shared": cfg.n_shared,
@@ -313,7 +344,8 @@ def run_native(args, cfg):
         achieved = weight_bytes[dom] / (dom_ms / 1e3) / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak}
-    roof.update({"kernel": dom, "kernel_ms": dom_ms, "traffic": None,
+    traffic = captured_traffic(dom, weight_bytes[dom])
+    roof.update({"kernel": dom, "kernel_ms": dom_ms, "traffic": traffic,
                  "peak_source": f"{peak_src} ({'bf16_tflops_sustained' if roof['bound'] == 'tensor' else 'hbm_gbs'})",
                  "algorithmic": {"flops": flops[dom], "weight_bytes": weight_bytes[dom]}})
     layer_flops = cfg.flops_per_token() * cfg.T

@@ -180,6 +180,37 @@ dsmoe_status dsmoe_forward_host(dsmoe_handle* h, int32_t T,
 dsmoe_status dsmoe_balance_stats(dsmoe_handle* h, int64_t T_total, const int32_t* counts,
                                  const float* P_sum, float* f, float* P, void* stream);
 
+/*
+ * Load-balance control from a forward's statistics (all device pointers, [N'] unless
+ * stated; nothing is allocated, work is enqueued on `stream`):
+ *
+ * dsmoe_balance_losses -- expert-level loss L_ExpBal = alpha1 (1/N') sum_i f_i P_i and
+ *   device-level loss over n_groups groups of experts (group_of[i] in [0, n_groups)):
+ *   f_dev[d] = mean of f over group d, P_dev[d] = sum of P over group d,
+ *   L_DevBal = alpha2 sum_d f_dev[d] P_dev[d]  (DeepSeekMoE summary, "Expert-level
+ *   balance loss" and "Device-level balance loss"). losses[0] = L_ExpBal,
+ *   losses[1] = L_DevBal. 1 <= n_groups <= min(N', 512).
+ *
+ * dsmoe_sequence_balance -- sequence-wise statistics for T tokens made of T / seq_len
+ *   whole sequences (DeepSeek-V4 book ch. 2, section 3): f_seq[q,i] = share of sequence
+ *   q's tokens that selected expert i, p_seq[q,i] = mean score of expert i over the
+ *   sequence ([S, N'] each), loss[0] = beta * mean_q sum_i f_seq[q,i] p_seq[q,i].
+ *   topk_idx [T, K'] and scores [T, N'] come from dsmoe_forward (scores_dbg).
+ *   T must be a multiple of seq_len and T <= max_tokens.
+ *
+ * dsmoe_bias_update -- the auxiliary-loss-free bias step b_i += alpha (K'/N' - counts_i/T)
+ *   for counts gathered over T tokens (same chapter, section 3): an over-loaded expert's
+ *   bias falls, an under-loaded one's rises. b is updated in place.
+ */
+dsmoe_status dsmoe_balance_losses(dsmoe_handle* h, const float* f, const float* P, int32_t n_groups,
+                                  const int32_t* group_of, float alpha1, float alpha2, float* f_dev,
+                                  float* P_dev, float* losses, void* stream);
+dsmoe_status dsmoe_sequence_balance(dsmoe_handle* h, int32_t T, int32_t seq_len, const int32_t* topk_idx,
+                                    const float* scores, float beta, float* f_seq, float* p_seq, float* loss,
+                                    void* stream);
+dsmoe_status dsmoe_bias_update(dsmoe_handle* h, int64_t T, const int32_t* counts, float alpha, float* b,
+                               void* stream);
+
 /* Read and clear the device status word (synchronises the handle's device).
  * DSMOE_OK, or DSMOE_ERR_DEVICE_TIMEOUT if a kernel gave up a bounded wait. */
 dsmoe_status dsmoe_get_status(dsmoe_handle* h);
@@ -205,7 +236,8 @@ dsmoe_status dsmoe_launch_count(dsmoe_handle* h, int64_t* n);
  * Device address and shape of one intermediate buffer of the handle's workspace, for
  * tests and debugging; contents are those of the last forward on this handle:
  *   "logits"  fp32 [T, N']        router affinities, written when the CUDA-core router
- *                                 runs (T < 256); absent for hash routing
+ *                                 runs (T < 256) as split-K partial sums: the first
+ *                                 slice of [splits, T, N']; absent for hash routing
  *   "offsets" int32 [N'+1]        first slot of each expert's segment
  *   "slot_of" int32 [T, K']       slot holding token t's k-th expert row
  *   "Xp"      bf16 [T K', d]      token rows in expert-contiguous slot order

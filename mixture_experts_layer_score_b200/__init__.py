@@ -10,4 +10,5 @@ from .binding import (DSMoE, DsmoeCfg, DsmoeError, make_cfg, cfg_from, dsmoe_cre
                       dsmoe_set_wait_limit, dsmoe_set_timing, dsmoe_stage_times, dsmoe_stage_name,
                       dsmoe_launch_count, dsmoe_check_config, dsmoe_workspace_bytes, dsmoe_abi_version,
                       dsmoe_status_string, dsmoe_last_error, stage_names, ABI_FUNCTIONS, LIB_PATH,
-                      dsmoe_workspace_tensor, workspace_view, dsmoe_route_noalloc)
+                      dsmoe_workspace_tensor, workspace_view, dsmoe_balance_losses,
+                      dsmoe_sequence_balance, dsmoe_bias_update, dsmoe_route_noalloc)

@@ -25,6 +25,7 @@ ABI_FUNCTIONS = (
     "dsmoe_workspace_bytes", "dsmoe_create", "dsmoe_destroy", "dsmoe_forward", "dsmoe_forward_host",
     "dsmoe_balance_stats", "dsmoe_get_status", "dsmoe_set_wait_limit", "dsmoe_set_timing",
     "dsmoe_stage_times", "dsmoe_stage_name", "dsmoe_launch_count", "dsmoe_workspace_tensor",
+    "dsmoe_balance_losses", "dsmoe_sequence_balance", "dsmoe_bias_update",
     "dsmoe_route_noalloc",
 )
 
@@ -67,6 +68,10 @@ def _load():
         "dsmoe_stage_times": (ctypes.c_int, [vp, ctypes.POINTER(ctypes.c_float), i32, ctypes.POINTER(i32)]),
         "dsmoe_stage_name": (ctypes.c_char_p, [i32]),
         "dsmoe_launch_count": (ctypes.c_int, [vp, ctypes.POINTER(i64)]),
+        "dsmoe_balance_losses": (ctypes.c_int, [vp, vp, vp, i32, vp, ctypes.c_float, ctypes.c_float, vp, vp, vp,
+                                                vp]),
+        "dsmoe_sequence_balance": (ctypes.c_int, [vp, i32, i32, vp, vp, ctypes.c_float, vp, vp, vp, vp]),
+        "dsmoe_bias_update": (ctypes.c_int, [vp, i64, vp, ctypes.c_float, vp, vp]),
         "dsmoe_workspace_tensor": (ctypes.c_int, [vp, ctypes.c_char_p, ctypes.POINTER(vp),
                                                   ctypes.POINTER(i64), ctypes.POINTER(i64)]),
         "dsmoe_route_noalloc": (ctypes.c_int, [cfgp, i32] + [vp] * 8 + [vp]),
@@ -219,6 +224,23 @@ def dsmoe_route_noalloc(cfg: DsmoeCfg, T, x, W_router, b, topk_idx, gates, count
     st = _lib.dsmoe_route_noalloc(ctypes.byref(cfg), int(T), *[_ptr(t) for t in (
         x, W_router, b, topk_idx, gates, counts, f, P)], _stream(stream))
     _check(st, "dsmoe_route_noalloc")
+
+
+def dsmoe_balance_losses(handle, f, P, n_groups, group_of, alpha1, alpha2, f_dev, P_dev, losses, stream=None):
+    _check(_lib.dsmoe_balance_losses(handle, _ptr(f), _ptr(P), int(n_groups), _ptr(group_of), float(alpha1),
+                                     float(alpha2), _ptr(f_dev), _ptr(P_dev), _ptr(losses), _stream(stream)),
+           "dsmoe_balance_losses")
+
+
+def dsmoe_sequence_balance(handle, T, seq_len, topk_idx, scores, beta, f_seq, p_seq, loss, stream=None):
+    _check(_lib.dsmoe_sequence_balance(handle, int(T), int(seq_len), _ptr(topk_idx), _ptr(scores), float(beta),
+                                       _ptr(f_seq), _ptr(p_seq), _ptr(loss), _stream(stream)),
+           "dsmoe_sequence_balance")
+
+
+def dsmoe_bias_update(handle, T, counts, alpha, b, stream=None):
+    _check(_lib.dsmoe_bias_update(handle, int(T), _ptr(counts), float(alpha), _ptr(b), _stream(stream)),
+           "dsmoe_bias_update")
 
 
 _WS_DTYPES = {"logits": "float32", "offsets": "int32", "slot_of": "int32", "Xp": "bfloat16",

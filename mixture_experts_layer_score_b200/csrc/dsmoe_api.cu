@@ -12,6 +12,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 #include <string>
 
@@ -102,7 +103,7 @@ struct DeviceGuard {
 };
 
 struct Layout {
-  size_t logits, counts_ws, cursor, offsets, P_part, slot_of, Xp, A1, A1s, Y, Hs, status;
+  size_t logits, counts_ws, cursor, offsets, P_part, slot_of, Xp, A1, A1s, Y, Hs, status, seq_terms;
   size_t x_stage, ids_stage, h_stage, topk_stage, gates_stage, counts_stage, f_stage, P_stage;
   size_t total;
 };
@@ -120,7 +121,13 @@ Layout plan(const dsmoe_cfg& c) {
   const size_t T = static_cast<size_t>(c.max_tokens), N = c.n_routed, K = c.top_k, d = c.d_model, F = c.d_ff;
   const size_t S = T * K, KsFs = static_cast<size_t>(c.n_shared) * c.d_ff_shared;
   const bool hash = c.score == DSMOE_ROUTE_HASH;
-  L.logits = take(hash ? 0 : T * N * 4);
+  // router logits as split-K partial sums: up to kRouterMaxSplits slices for small
+  // batches (CUDA-core router), T + kRouterTcExtraRows rows for the tensor-core router
+  const size_t small_T = T < static_cast<size_t>(kTcRouterMinTokens) ? T : kTcRouterMinTokens - 1;
+  size_t logit_floats = dsmoe::kRouterMaxSplits * small_T * N;
+  if (T >= static_cast<size_t>(kTcRouterMinTokens))
+    logit_floats = std::max(logit_floats, (T + static_cast<size_t>(dsmoe::kRouterTcExtraRows)) * N);
+  L.logits = take(hash ? 0 : logit_floats * 4);
   L.counts_ws = take(N * 4);
   L.cursor = take(N * 4);
   L.offsets = take((N + 1) * 4);
@@ -132,6 +139,7 @@ Layout plan(const dsmoe_cfg& c) {
   L.Y = take(S * d * 2);
   L.Hs = take(c.n_shared > 0 ? T * d * 4 : 0);
   L.status = take(4);
+  L.seq_terms = take(T * 4);
   L.x_stage = take(T * d * 2);
   L.ids_stage = take(hash ? T * 4 : 0);
   L.h_stage = take(T * d * 2);
@@ -170,6 +178,7 @@ struct dsmoe_handle {
   bf16 *Xp, *A1, *A1s, *Y;
   float* Hs;
   uint32_t* status;
+  float* seq_terms;
   bf16 *x_stage, *h_stage;
   int32_t *ids_stage, *topk_stage, *counts_stage;
   float *gates_stage, *f_stage, *P_stage;
@@ -299,6 +308,7 @@ DSMOE_EXPORT dsmoe_status dsmoe_create(const dsmoe_cfg* cfg, int32_t device, dsm
   h->Y = reinterpret_cast<bf16*>(w + L.Y);
   h->Hs = reinterpret_cast<float*>(w + L.Hs);
   h->status = reinterpret_cast<uint32_t*>(w + L.status);
+  h->seq_terms = reinterpret_cast<float*>(w + L.seq_terms);
   h->x_stage = reinterpret_cast<bf16*>(w + L.x_stage);
   h->ids_stage = reinterpret_cast<int32_t*>(w + L.ids_stage);
   h->h_stage = reinterpret_cast<bf16*>(w + L.h_stage);
@@ -314,9 +324,10 @@ DSMOE_EXPORT dsmoe_status dsmoe_create(const dsmoe_cfg* cfg, int32_t device, dsm
   }
   const dsmoe_cfg& c = h->cfg;
   const uint64_t S = static_cast<uint64_t>(c.max_tokens) * c.top_k;
-  bool ok = map_2d(&h->tm_xp, h->Xp, c.d_model, S, 128) && map_2d(&h->tm_a1, h->A1, c.d_ff, S, 128);
+  const uint32_t t1 = dsmoe::kGemmGateUpTokenTile, t2 = dsmoe::kGemmDownTokenTile;
+  bool ok = map_2d(&h->tm_xp, h->Xp, c.d_model, S, t1) && map_2d(&h->tm_a1, h->A1, c.d_ff, S, t2);
   if (c.n_shared > 0)
-    ok = ok && map_2d(&h->tm_a1s, h->A1s, static_cast<uint64_t>(c.n_shared) * c.d_ff_shared, c.max_tokens, 128);
+    ok = ok && map_2d(&h->tm_a1s, h->A1s, static_cast<uint64_t>(c.n_shared) * c.d_ff_shared, c.max_tokens, t2);
   else
     h->tm_a1s = h->tm_a1;
   if (!ok) {
@@ -431,8 +442,8 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
   const CUtensorMap* m_swg = Ks ? weight_map(h, 3, a.Ws_gate, &ok) : m_wg;
   const CUtensorMap* m_swu = Ks ? weight_map(h, 4, a.Ws_up, &ok) : m_wu;
   const CUtensorMap* m_swd = Ks ? weight_map(h, 5, a.Ws_down, &ok) : m_wd;
-  CUtensorMap m_x;
-  ok = ok && map_2d(&m_x, a.x, d, T, 128);
+  CUtensorMap m_x, m_x_router;  // token rows of x: GEMM tiles, and the router's 128-token tiles
+  ok = ok && map_2d(&m_x, a.x, d, T, dsmoe::kGemmGateUpTokenTile) && map_2d(&m_x_router, a.x, d, T, 128);
   if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map of this call");
 
   CUDA_TRY(mark(0));
@@ -443,50 +454,46 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
                                       h->status, s));
     h->launches += 1;
     CUDA_TRY(mark(1));
-  } else if (T >= kTcRouterMinTokens) {
-    // tensor-core affinities with scoring, top-K', gates and partials in the epilogue
-    dsmoe::RouterTcArgs ra;
-    memset(&ra, 0, sizeof(ra));
-    const CUtensorMap* m_wr = weight_map(h, 6, a.W_router, &ok);
-    if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected the router tensor map");
-    ra.tm_x = m_x;
-    ra.tm_w = *m_wr;
-    ra.b = a.b;
-    ra.T = T;
-    ra.N = N;
-    ra.K = K;
-    ra.d = d;
-    ra.score = c.score;
-    ra.bias_select = c.bias_mode == DSMOE_BIAS_SELECT_ONLY;
-    ra.bias_in_logits = c.bias_mode == DSMOE_BIAS_IN_LOGITS;
-    ra.renormalize = c.renormalize;
-    ra.n_chunks = h->rt_chunks;
-    ra.nc = h->rt_nc;
-    ra.tmem_cols = h->rt_cols;
-    ra.topk_idx = a.topk_idx;
-    ra.gates = a.gates;
-    ra.counts = h->counts_ws;
-    ra.P_part = h->P_part;
-    ra.scores_dbg = a.scores_dbg;
-    ra.status = h->status;
-    ra.wait_limit_ns = h->wait_ns;
-    const int tiles = cdiv(T, 128);
-    sel_grid = tiles < h->num_sms ? tiles : h->num_sms;
-    CUDA_TRY(dsmoe::launch_router_tc(ra, sel_grid, s));
-    h->launches += 1;
-    CUDA_TRY(mark(1));
   } else {
-    CUDA_TRY(dsmoe::launch_router_logits(static_cast<const bf16*>(a.x), static_cast<const bf16*>(a.W_router), a.b,
-                                         c.bias_mode == DSMOE_BIAS_IN_LOGITS, T, N, d, h->logits, s));
+    // router affinities as split-K partial sums: tensor cores for larger batches,
+    // CUDA cores below kTcRouterMinTokens tokens; then scores, top-K', gates, partials
+    int splits;
+    if (T >= kTcRouterMinTokens) {
+      dsmoe::RouterTcArgs ra;
+      memset(&ra, 0, sizeof(ra));
+      const CUtensorMap* m_wr = weight_map(h, 6, a.W_router, &ok);
+      if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected the router tensor map");
+      splits = dsmoe::router_tc_splits(T, d, h->num_sms);
+      ra.tm_x = m_x_router;
+      ra.tm_w = *m_wr;
+      ra.T = T;
+      ra.N = N;
+      ra.d = d;
+      ra.splits = splits;
+      ra.n_chunks = h->rt_chunks;
+      ra.nc = h->rt_nc;
+      ra.tmem_cols = h->rt_cols;
+      ra.partial = h->logits;
+      ra.status = h->status;
+      ra.wait_limit_ns = h->wait_ns;
+      const int work = cdiv(T, 128) * splits;
+      CUDA_TRY(dsmoe::launch_router_tc(ra, work < h->num_sms ? work : h->num_sms, s));
+    } else {
+      splits = dsmoe::router_logits_splits(T, N, d, h->num_sms);
+      CUDA_TRY(dsmoe::launch_router_logits(static_cast<const bf16*>(a.x), static_cast<const bf16*>(a.W_router), T,
+                                           N, d, splits, h->logits, s));
+    }
     CUDA_TRY(mark(1));
     dsmoe::SelectArgs sa;
     sa.logits = h->logits;
+    sa.splits = splits;
     sa.b = a.b;
     sa.T = T;
     sa.N = N;
     sa.K = K;
     sa.score = c.score;
     sa.bias_select = c.bias_mode == DSMOE_BIAS_SELECT_ONLY;
+    sa.bias_in_logits = c.bias_mode == DSMOE_BIAS_IN_LOGITS;
     sa.renormalize = c.renormalize;
     sa.topk_idx = a.topk_idx;
     sa.gates = a.gates;
@@ -551,8 +558,9 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
     g.shared_col_stride = Fs;
     g.status = h->status;
     g.wait_limit_ns = h->wait_ns;
-    const int64_t bound = (cdiv(S, 128) + N) * static_cast<int64_t>(g.n_tiles_routed) +
-                          static_cast<int64_t>(Ks) * cdiv(T, 128) * g.n_tiles_shared;
+    const int64_t tt = dsmoe::kGemmGateUpTokenTile;
+    const int64_t bound = (cdiv(S, tt) + N) * static_cast<int64_t>(g.n_tiles_routed) +
+                          static_cast<int64_t>(Ks) * cdiv(T, tt) * g.n_tiles_shared;
     const int grid = static_cast<int>(bound < h->num_sms ? bound : h->num_sms);
     CUDA_TRY(dsmoe::launch_grouped_gemm(true, g, grid, s));
     h->launches += 1;
@@ -588,8 +596,9 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
     g.shared_col_stride = 0;
     g.status = h->status;
     g.wait_limit_ns = h->wait_ns;
-    const int64_t bound = (cdiv(S, 128) + N) * static_cast<int64_t>(g.n_tiles_routed) +
-                          static_cast<int64_t>(g.n_shared_groups) * cdiv(T, 128) * g.n_tiles_shared;
+    const int64_t tt = dsmoe::kGemmDownTokenTile;
+    const int64_t bound = (cdiv(S, tt) + N) * static_cast<int64_t>(g.n_tiles_routed) +
+                          static_cast<int64_t>(g.n_shared_groups) * cdiv(T, tt) * g.n_tiles_shared;
     const int grid = static_cast<int>(bound < h->num_sms ? bound : h->num_sms);
     CUDA_TRY(dsmoe::launch_grouped_gemm(false, g, grid, s));
     h->launches += 1;
@@ -765,4 +774,49 @@ DSMOE_EXPORT dsmoe_status dsmoe_workspace_tensor(dsmoe_handle* h, const char* na
     }
   }
   return fail(DSMOE_ERR_INVALID_ARG, "unknown workspace buffer '%s'", name);
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_balance_losses(dsmoe_handle* h, const float* f, const float* P, int32_t n_groups,
+                                               const int32_t* group_of, float alpha1, float alpha2, float* f_dev,
+                                               float* P_dev, float* losses, void* stream) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  if (!f || !P || !group_of || !f_dev || !P_dev || !losses) return fail(DSMOE_ERR_INVALID_ARG, "NULL argument");
+  if (n_groups < 1 || n_groups > h->cfg.n_routed || n_groups > 512)
+    return fail(DSMOE_ERR_INVALID_ARG, "n_groups = %d outside [1, min(N', 512)]", n_groups);
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
+  CUDA_TRY(dsmoe::launch_balance_losses(f, P, h->cfg.n_routed, n_groups, group_of, alpha1, alpha2, f_dev, P_dev,
+                                        losses, static_cast<cudaStream_t>(stream)));
+  h->launches += 1;
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_sequence_balance(dsmoe_handle* h, int32_t T, int32_t seq_len, const int32_t* topk_idx,
+                                                 const float* scores, float beta, float* f_seq, float* p_seq,
+                                                 float* loss, void* stream) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  if (h->cfg.score == DSMOE_ROUTE_HASH) return fail(DSMOE_ERR_UNSUPPORTED, "hash routing has no scores");
+  if (seq_len <= 0 || T < 0 || T % seq_len) return fail(DSMOE_ERR_INVALID_ARG, "T = %d is not whole sequences of %d", T, seq_len);
+  if (T > h->cfg.max_tokens) return fail(DSMOE_ERR_WORKSPACE, "T = %d exceeds max_tokens", T);
+  if (!loss || (T > 0 && (!topk_idx || !scores || !f_seq || !p_seq))) return fail(DSMOE_ERR_INVALID_ARG, "NULL argument");
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
+  const int S = T / seq_len;
+  CUDA_TRY(dsmoe::launch_sequence_balance(topk_idx, scores, S, seq_len, h->cfg.n_routed, h->cfg.top_k, beta, f_seq,
+                                          p_seq, h->seq_terms, loss, static_cast<cudaStream_t>(stream)));
+  h->launches += S > 0 ? 2 : 1;
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_bias_update(dsmoe_handle* h, int64_t T, const int32_t* counts, float alpha, float* b,
+                                            void* stream) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  if (!counts || !b) return fail(DSMOE_ERR_INVALID_ARG, "NULL argument");
+  if (T < 0) return fail(DSMOE_ERR_INVALID_ARG, "T is negative");
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
+  CUDA_TRY(dsmoe::launch_bias_update(counts, T, h->cfg.n_routed, h->cfg.top_k, alpha, b,
+                                     static_cast<cudaStream_t>(stream)));
+  h->launches += 1;
+  return DSMOE_OK;
 }

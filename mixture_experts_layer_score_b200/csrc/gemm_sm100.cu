@@ -19,17 +19,18 @@
 //
 // One CTA per SM, 192 threads in three roles:
 //   warp 0     TMA producer: per 64-wide K block a 256x64 weight tile (two 128-row
-//              halves) and a 128x64 token tile through a 4-stage shared-memory ring
-//              (mbarrier full/empty pairs).
-//   warp 1     allocates 512 TMEM columns (two accumulators of 2 x 128 columns) and
-//              issues tcgen05.mma (M=128, N=16..128, K=16) from one thread, two chains
-//              (one per weight half) sharing the token tile; commits free ring stages
-//              and publish finished accumulators.
+//              halves) and a 128x64 token tile through a 4-stage shared-memory ring of
+//              48 KB stages (mbarrier full/empty pairs).
+//   warp 1     allocates 512 TMEM columns (two accumulators, each two chains of 128
+//              columns) and issues tcgen05.mma (M=128, N=16..128, K=16) from one
+//              thread, two chains (one per weight half) sharing the token tile; commits
+//              free ring stages and publish finished accumulators.
 //   warps 2-5  epilogue: thread f of TMEM lane f owns output feature f of both chains;
-//              it reads 16 token columns at a time with tcgen05.ld and stores one
-//              element per token (consecutive features across a warp, so each store
-//              instruction writes 32 consecutive features of one row). The second TMEM
-//              accumulator lets the next tile's MMAs overlap this epilogue.
+//              per 32 tokens it reads its accumulator columns with tcgen05.ld, applies
+//              SiLU(gate)*up (or the residual), and the warp transposes the 32 x 32
+//              block through shared memory so that each lane stores 16-byte vectors
+//              along output rows. The second TMEM accumulator lets the next tile's MMAs
+//              overlap this epilogue.
 //
 // Every wait is bounded (wait_limit_ns); a role that gives up raises a CTA-wide abort
 // flag and a bit of the device status word, the CTA lets in-flight TMA loads and MMAs
@@ -40,29 +41,41 @@
 namespace dsmoe {
 
 namespace {
-constexpr int kBM = 128;        // tokens per tile (the MMA's N is this count rounded to 16)
 constexpr int kBK = 64;         // K per ring stage (one 128-byte swizzled row of bf16)
 constexpr int kFeat = 128;      // output features per MMA chain (the MMA's M, TMEM lanes)
 constexpr int kMmaK = 16;       // K of each bf16 tcgen05.mma
-constexpr int kStages = 4;
 constexpr int kThreads = 192;
 constexpr int kEpiThreads = 128;
-constexpr uint32_t kAccCols = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxGroups = 8 + 512;
 constexpr uint32_t kWBytes = 2 * kFeat * kBK * 2;  // 32 KB: two 128-row weight halves
-constexpr uint32_t kXBytes = kBM * kBK * 2;        // 16 KB: 128 token rows
-constexpr uint32_t kStageBytes = kWBytes + kXBytes;
+constexpr uint32_t kStageRow = 33;  // epilogue staging rows padded to 33 words
 
-constexpr uint32_t kOffW = 0;
-constexpr uint32_t kOffX = kOffW + kStages * kWBytes;
-constexpr uint32_t kOffBars = kOffX + kStages * kXBytes;
-constexpr uint32_t kNumBars = 2 * kStages + 2 + 2 + 1;
-constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
-constexpr uint32_t kOffTiles = kOffMisc + 16;
-constexpr uint32_t kSmemUsed = kOffTiles + (kMaxGroups + 1) * 4;
-constexpr size_t kSmemBytes = kSmemUsed + 1024;  // slack to align the ring to 1024 bytes
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+// Tile geometry of each projection. Gate/up (long K): 256-token tiles, one accumulator
+// of two 256-column chains, 3 stages of 64 KB: 15.6 KB staged per million MACs. Down
+// (short K): 128-token tiles, two accumulators so the epilogue overlaps the next tile's
+// MMAs, 4 stages of 48 KB.
+template <bool kSwiGLU>
+struct Geo {
+  static constexpr int kTok = kSwiGLU ? kGemmGateUpTokenTile : kGemmDownTokenTile;
+  static constexpr uint32_t kChainCols = kTok;
+  static constexpr uint32_t kAccCols = 2 * kChainCols;
+  static constexpr int kBufs = static_cast<int>(kTmemCols / kAccCols);
+  static constexpr int kStages = kSwiGLU ? 3 : 4;
+  static constexpr uint32_t kXBytes = kTok * kBK * 2;
+  static constexpr uint32_t kStageBytes = kWBytes + kXBytes;
+  static constexpr uint32_t kOffW = 0;
+  static constexpr uint32_t kOffX = kOffW + kStages * kWBytes;
+  static constexpr uint32_t kOffBars = kOffX + kStages * kXBytes;
+  static constexpr uint32_t kNumBars = 2 * kStages + 2 + 2 + 1;
+  static constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
+  static constexpr uint32_t kOffTiles = kOffMisc + 16;
+  static constexpr uint32_t kOffEpi = (kOffTiles + (kMaxGroups + 1) * 4 + 15) & ~15u;
+  static constexpr uint32_t kSmemUsed = kOffEpi + 4 * 32 * kStageRow * 4;
+  static constexpr size_t kSmemBytes = kSmemUsed + 1024;  // slack to align the ring to 1024 bytes
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kBufs >= 1 && kTok % 32 == 0 && kTok <= 256, "tile geometry");
+};
 
 struct Tile {
   int shared;   // 1: shared-expert group
@@ -74,6 +87,7 @@ struct Tile {
   int kb_n;     // K blocks
 };
 
+template <int kBM>
 __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int32_t* tile_start, int G, int tile) {
   int lo = 0, hi = G - 1;
   while (lo < hi) {  // last group whose first tile is <= tile
@@ -106,25 +120,24 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int32_t* ti
   return t;
 }
 
-__device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
-
 template <bool kSwiGLU>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs a) {
+  using G_ = Geo<kSwiGLU>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_addr(smem_raw) & 1023u)) & 1023u;
   uint8_t* base = smem_raw + pad;
-  uint8_t* sW = base + kOffW;
-  uint8_t* sX = base + kOffX;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + kOffBars);
+  uint8_t* sW = base + G_::kOffW;
+  uint8_t* sX = base + G_::kOffX;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + G_::kOffBars);
   uint64_t* full = bars;
-  uint64_t* empty = bars + kStages;
-  uint64_t* acc_full = bars + 2 * kStages;
+  uint64_t* empty = bars + G_::kStages;
+  uint64_t* acc_full = bars + 2 * G_::kStages;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + kOffMisc + 4);
-  volatile int* never_flag = reinterpret_cast<volatile int*>(base + kOffMisc + 8);
-  int32_t* tile_start = reinterpret_cast<int32_t*>(base + kOffTiles);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + G_::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + G_::kOffMisc + 4);
+  volatile int* never_flag = reinterpret_cast<volatile int*>(base + G_::kOffMisc + 8);
+  int32_t* tile_start = reinterpret_cast<int32_t*>(base + G_::kOffTiles);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = a.n_shared_groups + a.n_routed;
@@ -141,13 +154,13 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       nt = a.n_tiles_routed;
     }
     M = max(M, 0);
-    tile_start[g + 1] = ((M + kBM - 1) / kBM) * nt;
+    tile_start[g + 1] = ((M + G_::kTok - 1) / G_::kTok) * nt;
   }
   if (threadIdx.x == 0) {
     tile_start[0] = 0;
     *abort_flag = 0;
     *never_flag = 0;
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < G_::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -195,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       uint32_t phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-        const Tile t = decode_tile(a, tile_start, G, tile);
+        const Tile t = decode_tile<G_::kTok>(a, tile_start, G, tile);
         const CUtensorMap* tx = t.shared ? &a.a_shared : &a.a_routed;
         const CUtensorMap* tw0 = t.shared ? &a.b0_shared : &a.b0_routed;
         const CUtensorMap* tw1 = t.shared ? &a.b1_shared : &a.b1_routed;
@@ -205,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], kStageBytes);
+          mbar_arrive_expect_tx(&full[stage], G_::kStageBytes);
           const int be = t.expert + kb / kb_per;
           const int bk = (kb % kb_per) * kBK;
           uint8_t* w = sW + stage * kWBytes;
@@ -215,10 +228,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
           } else {        // 256 consecutive output rows
             tma_load_3d(w, tw0, &full[stage], bk, t.n_blk * 2 * kFeat, be);
           }
-          tma_load_2d(sX + stage * kXBytes, tx, &full[stage], kb * kBK, t.row0);
+          tma_load_2d(sX + stage * G_::kXBytes, tx, &full[stage], kb * kBK, t.row0);
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == kStages) {
+          if (++stage == G_::kStages) {
             stage = 0;
             phase ^= 1u;
           }
@@ -237,17 +250,16 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       bool ok = true;
       int it = 0;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++it) {
-        const Tile t = decode_tile(a, tile_start, G, tile);
+        const Tile t = decode_tile<G_::kTok>(a, tile_start, G, tile);
         const int n_mma = (t.m_valid + 15) & ~15;  // tokens, rounded up to the MMA's N step
         const uint32_t idesc = idesc_bf16_f32(kFeat, n_mma);
-        const int acc = it & 1;
-        const uint32_t acc_phase = (it >> 1) & 1;
-        if (!mbar_wait_bounded(&acc_empty[acc], acc_phase ^ 1u, a.wait_limit_ns, abort_flag)) {
+        const int acc = it % G_::kBufs;
+        if (!mbar_wait_bounded(&acc_empty[acc], ((it / G_::kBufs) & 1) ^ 1u, a.wait_limit_ns, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d0 = tmem_base + acc * kAccCols;
+        const uint32_t d0 = tmem_base + acc * G_::kAccCols;
         for (int kb = 0; kb < t.kb_n; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, a.wait_limit_ns, abort_flag)) {
             ok = false;
@@ -256,16 +268,16 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
           tc_fence_after();
           const uint64_t w0 = smem_desc_kmajor_sw128(smem_addr(sW + stage * kWBytes));
           const uint64_t w1 = smem_desc_kmajor_sw128(smem_addr(sW + stage * kWBytes + kWBytes / 2));
-          const uint64_t xd = smem_desc_kmajor_sw128(smem_addr(sX + stage * kXBytes));
+          const uint64_t xd = smem_desc_kmajor_sw128(smem_addr(sX + stage * G_::kXBytes));
 #pragma unroll
           for (int k = 0; k < kBK / kMmaK; ++k) {
             const uint64_t dk = static_cast<uint64_t>(2 * k);
             const uint32_t accum = (kb | k) ? 1u : 0u;
             mma_bf16_ss(d0, w0 + dk, xd + dk, idesc, accum);
-            mma_bf16_ss(d0 + kFeat, w1 + dk, xd + dk, idesc, accum);
+            mma_bf16_ss(d0 + G_::kChainCols, w1 + dk, xd + dk, idesc, accum);
           }
           mma_commit(&empty[stage]);
-          if (++stage == kStages) {
+          if (++stage == G_::kStages) {
             stage = 0;
             phase ^= 1u;
           }
@@ -280,15 +292,18 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
     }
   } else {
     // -------------------------------------------------------------------- epilogue
+    // Thread f of TMEM lane f holds output feature f of both chains. Per 32 tokens, the
+    // warp transposes its 32 features x 32 tokens through a padded shared-memory tile,
+    // then lane L stores 8 consecutive features (16 B of bf16, 32 B of fp32) of token
+    // row L/4 + 8i: four lanes cover the warp's 32-feature segment of a row.
     const int q = warp & 3;  // this warp may read TMEM lanes [32q, 32q+32)
-    const int f = q * 32 + lane;  // output feature of chain 0 (and of chain 1) owned by this thread
+    float* stg = reinterpret_cast<float*>(base + G_::kOffEpi) + q * 32 * kStageRow;
+    const int rr = lane >> 2, cc = (lane & 3) * 8;  // read-out: row (plus 8i), first feature
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
-      const Tile t = decode_tile(a, tile_start, G, tile);
-      const int acc = it & 1;
-      const uint32_t acc_phase = (it >> 1) & 1;
-      const bool w = mbar_wait_bounded(&acc_full[acc], acc_phase, a.wait_limit_ns, abort_flag);
-      if (!__all_sync(0xffffffffu, w)) {
+      const Tile t = decode_tile<G_::kTok>(a, tile_start, G, tile);
+      const int acc = it % G_::kBufs;
+      if (!mbar_wait_warp_sleepy(&acc_full[acc], (it / G_::kBufs) & 1, a.wait_limit_ns, abort_flag)) {
         if (lane == 0) {
           *abort_flag = 1;
           atomicOr(a.status, kStatusTimeoutEpilogue);
@@ -296,66 +311,66 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         break;
       }
       tc_fence_after();
-      const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * G_::kAccCols;
       const int n_valid = t.shared ? a.n_valid_shared : a.n_valid_routed;
       const int64_t ld = t.shared ? a.ld_shared : a.ld_routed;
-      if (kSwiGLU) {
-        const int feat = t.n_blk * kFeat + f;
-        const bool ok_f = feat < n_valid;
-        bf16* out = (t.shared ? a.out_shared + static_cast<int64_t>(t.group) * a.shared_col_stride : a.out_routed) +
-                    static_cast<int64_t>(t.row0) * ld + feat;
+      const bool f32_out = !kSwiGLU && t.shared && a.out_shared_f32 != nullptr;
+      // chains whose values leave this tile: gate/up gives one output chain, down two
+      const int n_out = kSwiGLU ? 1 : 2;
 #pragma unroll 1
-        for (int c = 0; c < t.m_valid; c += 16) {
-          uint32_t gv[16], uv[16];
-          tmem_ld16(tb + c, gv);
-          tmem_ld16(tb + kFeat + c, uv);
-          tmem_wait_ld();
-          if (ok_f) {
+      for (int c0 = 0; c0 < t.m_valid; c0 += 32) {
+        uint32_t v0[32], v1[32];
+        tmem_ld16(tb + c0, *reinterpret_cast<uint32_t(*)[16]>(&v0[0]));
+        tmem_ld16(tb + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v0[16]));
+        tmem_ld16(tb + G_::kChainCols + c0, *reinterpret_cast<uint32_t(*)[16]>(&v1[0]));
+        tmem_ld16(tb + G_::kChainCols + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v1[16]));
+        tmem_wait_ld();
+#pragma unroll 1
+        for (int ch = 0; ch < n_out; ++ch) {
+          // stage: row = token (c0 + j), column = this lane's feature
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              if (c + j < t.m_valid)
-                out[static_cast<int64_t>(c + j) * ld] =
-                    __float2bfloat16_rn(silu(__uint_as_float(gv[j])) * __uint_as_float(uv[j]));
+          for (int j = 0; j < 32; ++j) {
+            float val;
+            if (kSwiGLU) {
+              const float g = __uint_as_float(v0[j]);
+              val = __fdividef(g, 1.0f + __expf(-g)) * __uint_as_float(v1[j]);  // SiLU(g) * u
+            } else {
+              val = __uint_as_float(ch == 0 ? v0[j] : v1[j]);
+            }
+            stg[j * kStageRow + lane] = val;
           }
-        }
-      } else if (t.shared && a.out_shared_f32) {
-        // shared experts of the down GEMM: fp32 row of (residual + sum of shared outputs)
-        const int feat0 = t.n_blk * 2 * kFeat + f, feat1 = feat0 + kFeat;
-        const int64_t r0 = static_cast<int64_t>(t.row0) * ld;
-#pragma unroll 1
-        for (int c = 0; c < t.m_valid; c += 16) {
-          uint32_t v0[16], v1[16];
-          tmem_ld16(tb + c, v0);
-          tmem_ld16(tb + kFeat + c, v1);
-          tmem_wait_ld();
+          __syncwarp();
+          const int feat = (kSwiGLU ? t.n_blk * kFeat : t.n_blk * 2 * kFeat + ch * kFeat) + q * 32 + cc;
+          const bool ok_f = feat < n_valid;  // n_valid is a multiple of 64, feat of 8
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (c + j < t.m_valid) {
-              const int64_t o = r0 + static_cast<int64_t>(c + j) * ld;
-              if (feat0 < n_valid)
-                a.out_shared_f32[o + feat0] = __uint_as_float(v0[j]) + __bfloat162float(a.residual[o + feat0]);
-              if (feat1 < n_valid)
-                a.out_shared_f32[o + feat1] = __uint_as_float(v1[j]) + __bfloat162float(a.residual[o + feat1]);
+          for (int i = 0; i < 4; ++i) {
+            const int row = rr + 8 * i;
+            if (ok_f && c0 + row < t.m_valid) {
+              const float* src = stg + row * kStageRow + cc;
+              const int64_t o = static_cast<int64_t>(t.row0 + c0 + row) * ld + feat;
+              if (f32_out) {
+                const uint4 rv = *reinterpret_cast<const uint4*>(a.residual + o);
+                const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
+                float out8[8];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const float2 xr = unpack_bf16x2(rw[k]);
+                  out8[2 * k] = src[2 * k] + xr.x;
+                  out8[2 * k + 1] = src[2 * k + 1] + xr.y;
+                }
+                float4* dst = reinterpret_cast<float4*>(a.out_shared_f32 + o);
+                dst[0] = make_float4(out8[0], out8[1], out8[2], out8[3]);
+                dst[1] = make_float4(out8[4], out8[5], out8[6], out8[7]);
+              } else {
+                bf16* obase = t.shared ? a.out_shared + static_cast<int64_t>(t.group) * a.shared_col_stride
+                                       : a.out_routed;
+                *reinterpret_cast<uint4*>(obase + o) =
+                    make_uint4(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
+                               pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
+              }
             }
           }
-        }
-      } else {
-        const int feat0 = t.n_blk * 2 * kFeat + f, feat1 = feat0 + kFeat;
-        bf16* out = (t.shared ? a.out_shared : a.out_routed) + static_cast<int64_t>(t.row0) * ld;
-#pragma unroll 1
-        for (int c = 0; c < t.m_valid; c += 16) {
-          uint32_t v0[16], v1[16];
-          tmem_ld16(tb + c, v0);
-          tmem_ld16(tb + kFeat + c, v1);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (c + j < t.m_valid) {
-              bf16* o = out + static_cast<int64_t>(c + j) * ld;
-              if (feat0 < n_valid) o[feat0] = __float2bfloat16_rn(__uint_as_float(v0[j]));
-              if (feat1 < n_valid) o[feat1] = __float2bfloat16_rn(__uint_as_float(v1[j]));
-            }
-          }
+          __syncwarp();
         }
       }
       tc_fence_before();
@@ -367,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
   if (*abort_flag) {
     // let every copy and MMA this CTA started finish before its memory is released
     if (warp == 0 && lane == 0) {
-      for (int s = 0; s < kStages; ++s)
+      for (int s = 0; s < G_::kStages; ++s)
         if ((issued_mask >> s) & 1u)
           if (!mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, a.wait_limit_ns, never_flag))
             atomicOr(a.status, kStatusTimeoutDrain);
@@ -392,14 +407,14 @@ cudaError_t launch_grouped_gemm(bool swiglu, const GemmArgs& a, int grid, cudaSt
   cudaError_t e;
   if (swiglu) {
     e = cudaFuncSetAttribute(grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes));
+                             static_cast<int>(Geo<true>::kSmemBytes));
     if (e != cudaSuccess) return e;
-    grouped_gemm_kernel<true><<<grid, kThreads, kSmemBytes, s>>>(a);
+    grouped_gemm_kernel<true><<<grid, kThreads, Geo<true>::kSmemBytes, s>>>(a);
   } else {
     e = cudaFuncSetAttribute(grouped_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes));
+                             static_cast<int>(Geo<false>::kSmemBytes));
     if (e != cudaSuccess) return e;
-    grouped_gemm_kernel<false><<<grid, kThreads, kSmemBytes, s>>>(a);
+    grouped_gemm_kernel<false><<<grid, kThreads, Geo<false>::kSmemBytes, s>>>(a);
   }
   return cudaGetLastError();
 }

@@ -21,16 +21,21 @@ enum : uint32_t {
 
 
 // ---------------------------------------------------------------- router (router.cu)
-// logits[t, i] = sum_k x[t,k] W_router[i,k] (+ b[i] when bias_in_logits), fp32.
-cudaError_t launch_router_logits(const bf16* x, const bf16* W_router, const float* b, int bias_in_logits,
-                                 int T, int N, int d, float* logits, cudaStream_t s);
+// logits[t, i] = sum_k x[t,k] W_router[i,k], fp32, as `splits` partial sums over
+// slices of k (logits holds splits x T x N floats).
+constexpr int kRouterMaxSplits = 64;
+int router_logits_splits(int T, int N, int d, int num_sms);
+cudaError_t launch_router_logits(const bf16* x, const bf16* W_router, int T, int N, int d, int splits,
+                                 float* logits, cudaStream_t s);
 
 struct SelectArgs {
-  const float* logits;   // [T, N]
+  const float* logits;   // [splits, T, N] partial sums
+  int splits;
   const float* b;        // [N] or nullptr
   int T, N, K;
   int score;             // dsmoe_score
   int bias_select;       // selection-only bias
+  int bias_in_logits;    // b is added to the summed logits before scoring
   int renormalize;
   int32_t* topk_idx;     // [T, K]
   float* gates;          // [T, K]
@@ -43,25 +48,25 @@ struct SelectArgs {
 cudaError_t launch_select(const SelectArgs& a, int grid, cudaStream_t s);
 int select_grid(int T, int num_sms);
 
-// Router on the tensor cores with scoring, top-K', gates and statistics partials fused
-// (router_sm100.cu). The B tile is n_chunks chunks of nc router rows (nc a multiple of
-// 16, at most 256); the accumulator takes tmem_cols TMEM columns.
+// Router affinities on the tensor cores (router_sm100.cu): split-K partial sums,
+// partial[slice][t][i] for `splits` slices of the reduction dimension. The B tile is
+// n_chunks chunks of nc router rows (nc a multiple of 16, at most 256); the
+// accumulator takes tmem_cols TMEM columns.
 struct RouterTcArgs {
   CUtensorMap tm_x;  // 2D [T, d] bf16, box (64, 128)
   CUtensorMap tm_w;  // 2D [N', d] bf16, box (64, nc)
-  const float* b;    // [N'] or nullptr
-  int T, N, K, d, score, bias_select, bias_in_logits, renormalize;
+  int T, N, d, splits;
   int n_chunks, nc;
   uint32_t tmem_cols;
-  int32_t* topk_idx;
-  float* gates;
-  int32_t* counts;     // [N'] accumulated with atomics (zeroed by the caller)
-  float* P_part;       // [gridDim.x, N'] per-CTA partial score sums
-  float* scores_dbg;   // [T, N'] or nullptr
+  float* partial;    // [splits, T, N']
   uint32_t* status;
   uint64_t wait_limit_ns;
 };
 void router_tc_shape(int N, int* n_chunks, int* nc, uint32_t* tmem_cols);
+int router_tc_splits(int T, int d, int num_sms);
+// Rows of partial sums the tensor-core router may write beyond T (for any GPU with at
+// most 192 SMs): splits * T <= T + 2 * 192 * 128.
+constexpr int64_t kRouterTcExtraRows = 2 * 192 * 128;
 cudaError_t launch_router_tc(const RouterTcArgs& a, int grid, cudaStream_t s);
 
 cudaError_t launch_hash_route(const int32_t* token_ids, int T, int N, uint32_t mult, uint32_t mod,
@@ -92,6 +97,16 @@ cudaError_t launch_permute_gather(const bf16* x, const int32_t* topk_idx, const 
                                   int32_t* cursor, int T, int K, int N, int d, int32_t* slot_of, bf16* Xp,
                                   uint32_t* status, int num_sms, cudaStream_t s);
 
+// ---------------------------------------------------------------- balance control (balance.cu)
+cudaError_t launch_balance_losses(const float* f, const float* P, int N, int G, const int32_t* group_of,
+                                  float alpha1, float alpha2, float* f_dev, float* P_dev, float* losses,
+                                  cudaStream_t s);
+cudaError_t launch_sequence_balance(const int32_t* topk_idx, const float* scores, int S, int seq_len, int N,
+                                    int K, float beta, float* f_seq, float* p_seq, float* seq_terms, float* loss,
+                                    cudaStream_t s);
+cudaError_t launch_bias_update(const int32_t* counts, int64_t T, int N, int K, float alpha, float* b,
+                               cudaStream_t s);
+
 // ---------------------------------------------------------------- combine (combine.cu)
 // h = base + sum_k gates[t,k] Y[slot_of[t,k]], where base is Hs (fp32 x + shared experts)
 // when Hs is not null, else x.
@@ -99,9 +114,13 @@ cudaError_t launch_combine(const bf16* x, const float* Hs, const bf16* Y, const 
                            const float* gates, int T, int K, int d, bf16* h, int num_sms, cudaStream_t s);
 
 // ---------------------------------------------------------------- grouped GEMM (gemm_sm100.cu)
+// Tokens per grouped-GEMM tile of each projection (the row box of its token-side
+// tensor maps).
+constexpr int kGemmGateUpTokenTile = 256;
+constexpr int kGemmDownTokenTile = 128;
 struct GemmArgs {
-  CUtensorMap a_routed;   // 2D [rows, K] activations of routed slots, box (64, 128)
-  CUtensorMap a_shared;   // 2D [T, K_shared] activations of the shared groups, box (64, 128)
+  CUtensorMap a_routed;   // 2D [rows, K] activations of routed slots, box (64, token tile)
+  CUtensorMap a_shared;   // 2D [T, K_shared] activations of the shared groups, box (64, token tile)
   CUtensorMap b0_routed;  // 3D (K, rows, experts): gate (SwiGLU) or down (plain) weights
   CUtensorMap b1_routed;  // 3D up-projection weights (SwiGLU only)
   CUtensorMap b0_shared;

@@ -20,10 +20,11 @@ namespace dsmoe {
 namespace {
 constexpr int kRTM = 64, kRTN = 64, kRTK = 32;
 
+// blockIdx.z selects a slice [z*kc, (z+1)*kc) of the reduction dimension; slice z
+// writes its partial sums to logits + z*T*N. The select kernel adds the slices in order.
 __global__ void __launch_bounds__(256) router_logits_kernel(const bf16* __restrict__ x,
-                                                            const bf16* __restrict__ W,
-                                                            const float* __restrict__ b, int bias_in_logits,
-                                                            int T, int N, int d, float* __restrict__ logits) {
+                                                            const bf16* __restrict__ W, int T, int N, int d,
+                                                            int kc, float* __restrict__ logits) {
   __shared__ __align__(16) float xs[kRTK][kRTM + 4];
   __shared__ __align__(16) float ws[kRTK][kRTN + 4];
   const int t0 = blockIdx.x * kRTM, n0 = blockIdx.y * kRTN;
@@ -35,7 +36,9 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const bf16* __restri
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 
-  for (int k0 = 0; k0 < d; k0 += kRTK) {
+  const int k_begin = blockIdx.z * kc, k_end = min(d, k_begin + kc);
+  logits += static_cast<int64_t>(blockIdx.z) * T * N;
+  for (int k0 = k_begin; k0 < k_end; k0 += kRTK) {
     uint4 vx = make_uint4(0, 0, 0, 0), vw = make_uint4(0, 0, 0, 0);
     if (t0 + lr < T) vx = *reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t0 + lr) * d + k0 + lc);
     if (n0 + lr < N) vw = *reinterpret_cast<const uint4*>(W + static_cast<int64_t>(n0 + lr) * d + k0 + lc);
@@ -68,16 +71,29 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const bf16* __restri
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int n = n0 + tx * 4 + j;
-      if (n < N) logits[static_cast<int64_t>(t) * N + n] = acc[i][j] + (bias_in_logits ? b[n] : 0.f);
+      if (n < N) logits[static_cast<int64_t>(t) * N + n] = acc[i][j];
     }
   }
 }
 }  // namespace
 
-cudaError_t launch_router_logits(const bf16* x, const bf16* W_router, const float* b, int bias_in_logits,
-                                 int T, int N, int d, float* logits, cudaStream_t s) {
-  dim3 grid((T + kRTM - 1) / kRTM, (N + kRTN - 1) / kRTN);
-  router_logits_kernel<<<grid, 256, 0, s>>>(x, W_router, b, bias_in_logits, T, N, d, logits);
+int router_logits_splits(int T, int N, int d, int num_sms) {
+  const int tiles = ((T + kRTM - 1) / kRTM) * ((N + kRTN - 1) / kRTN);
+  int splits = (2 * num_sms + tiles - 1) / tiles;  // about two CTAs per SM
+  const int max_splits = d / kRTK;
+  if (splits > max_splits) splits = max_splits;
+  if (splits > kRouterMaxSplits) splits = kRouterMaxSplits;
+  if (splits < 1) splits = 1;
+  return splits;
+}
+
+cudaError_t launch_router_logits(const bf16* x, const bf16* W_router, int T, int N, int d, int splits,
+                                 float* logits, cudaStream_t s) {
+  // slice length: a multiple of the 32-wide k step covering d in `splits` slices
+  const int kc = ((d / kRTK + splits - 1) / splits) * kRTK;
+  const int used = (d + kc - 1) / kc;
+  dim3 grid((T + kRTM - 1) / kRTM, (N + kRTN - 1) / kRTN, used);
+  router_logits_kernel<<<grid, 256, 0, s>>>(x, W_router, T, N, d, kc, logits);
   return cudaGetLastError();
 }
 
@@ -122,11 +138,18 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(const SelectArgs
   const int gw = blockIdx.x * kSelWarps + warp, nw = gridDim.x * kSelWarps;
   for (int t = gw; t < a.T; t += nw) {
     const float* lrow = a.logits + static_cast<int64_t>(t) * N;
+    const int64_t slice = static_cast<int64_t>(a.T) * N;
     float s[kNPL];
 #pragma unroll
     for (int j = 0; j < kNPL; ++j) {
       const int i = lane + 32 * j;
-      s[j] = (i < N) ? lrow[i] : -INFINITY;
+      float v = -INFINITY;
+      if (i < N) {
+        v = lrow[i];
+        for (int z = 1; z < a.splits; ++z) v += lrow[z * slice + i];
+        if (a.bias_in_logits) v += a.b[i];
+      }
+      s[j] = v;
     }
     if (a.score == 0) {  // softmax over the routed experts
       float m = -INFINITY;

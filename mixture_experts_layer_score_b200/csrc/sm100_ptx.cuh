@@ -68,6 +68,33 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// The same wait for a whole warp that is not on the critical path (an epilogue waiting
+// for an accumulator): only lane 0 polls, backing off with __nanosleep so that the
+// polling does not compete with the TMA and MMA traffic on the barrier's shared-memory
+// bank; the verdict is broadcast to the warp. Must be called by all 32 lanes.
+__device__ __forceinline__ bool mbar_wait_warp_sleepy(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                                      volatile int* abort_flag) {
+  uint32_t ok = 1;
+  if ((threadIdx.x & 31) == 0) {
+    if (!mbar_try_wait(bar, parity)) {
+      const uint64_t t0 = global_timer_ns();
+      uint32_t sleep_ns = 32;
+      for (;;) {
+        __nanosleep(sleep_ns);
+        if (mbar_try_wait(bar, parity)) break;
+        if (sleep_ns < 512) sleep_ns <<= 1;
+        if (*abort_flag || global_timer_ns() - t0 > limit_ns) {
+          ok = 0;
+          break;
+        }
+      }
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) (void)mbar_try_wait(bar, parity);  // every lane observes the completed phase
+  return ok != 0;
+}
+
 // ------------------------------------------------------------------------------------
 // TMA (tiled tensor loads into shared memory, completion counted on an mbarrier)
 // ------------------------------------------------------------------------------------

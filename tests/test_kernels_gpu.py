@@ -20,8 +20,8 @@ pytestmark = pytest.mark.gpu
 if not torch.cuda.is_available():
     pytest.skip("no GPU", allow_module_level=True)
 
-# T < 256 runs the CUDA-core router (logits kept in the workspace); larger T the
-# tensor-core router, whose scores are checked through scores_dbg.
+# T < 256 runs the CUDA-core router (split-K logits, then the select kernel); larger T
+# the tensor-core router; both are checked through the scores they report.
 CASES = [("tiny", 300), ("tiny", 200), ("gshard_c", 700), ("ds2b", 900), ("v4_decode_t64", 64)]
 
 
@@ -33,15 +33,13 @@ def test_stages(name, T):
     out = layer.forward(gpu["x"], with_scores=True)
     torch.cuda.synchronize()
     ws = {n: M.workspace_view(layer.handle, n).clone().cpu()
-          for n in ("logits", "offsets", "slot_of", "Xp", "A1", "Y") + (("A1s", "Hs") if cfg.n_shared else ())}
+          for n in ("offsets", "slot_of", "Xp", "A1", "Y") + (("A1s", "Hs") if cfg.n_shared else ())}
     assert M.dsmoe_get_status(layer.handle) == M.DSMOE_OK
     layer.close()
     K, N, S = cfg.top_k, cfg.n_routed, T * cfg.top_k
     x64 = O.bf16_bits_to_f64(cpu["x"])
-    # router: logits (CUDA-core path) or scores (both paths) against float64
+    # router scores (either router) against float64
     l_ref = O.router_logits(cpu["x"], cpu["W_router"], cpu.get("b"), cfg.bias_mode)
-    if T < 256:
-        assert np.abs(ws["logits"][:T].numpy() - l_ref).max() < 1e-4
     s_ref = O.scores(l_ref, cfg.score)
     assert np.abs(out["scores"].cpu().numpy() - s_ref).max() < 2e-5
     # offsets: exclusive scan of the counts

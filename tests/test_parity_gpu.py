@@ -186,10 +186,10 @@ def test_stage_timing_and_launch_count():
     layer.forward(gpu["x"])
     t = M.dsmoe_stage_times(layer.handle)
     assert list(t) == M.stage_names() and all(v >= 0 for v in t.values())
-    # tensor-core router (T >= 256): router, scan, permute, two GEMMs, combine
-    assert M.dsmoe_launch_count(layer.handle) - n0 == 6
+    # router logits (tensor cores for T >= 256), select, scan, permute, two GEMMs, combine
+    assert M.dsmoe_launch_count(layer.handle) - n0 == 7
     M.dsmoe_set_timing(layer.handle, False)
     n1 = M.dsmoe_launch_count(layer.handle)
-    layer.forward(gpu["x"][:100].contiguous())  # CUDA-core router + separate select kernel
+    layer.forward(gpu["x"][:100].contiguous())  # CUDA-core router logits below 256 tokens
     assert M.dsmoe_launch_count(layer.handle) - n1 == 7
     layer.close()

@@ -16,7 +16,7 @@ Shapes follow the configurations the DeepSeekMoE pages describe:
   routed experts, top-6, and a Zipf per-expert logit bias for a ~10:1 load skew.
 * ``v3_prefill``: 256 routed + 1 shared, top-8, sigmoid scores with a
   selection-only bias, renormalised gates (V4 book ch. 2, section 2 and 3).
-* ``v3_slice``: the V3 layer's shapes with 16 routed experts and T=512 (the same
+* ``v3_slice``: the V3 layer's shapes with 32 routed experts and T=1024 (the same
   256 rows per expert on average), a small case for profiler captures.
 * ``v4_decode_t{16,64,256}``: 384 routed + 1 shared, top-9, sqrt(softplus)
   scores (V4 book ch. 2, section 2 equation) with a selection-only bias.
@@ -110,9 +110,9 @@ def _cfgs():
                                 d_ff=2048, n_shared=1, d_ff_shared=2048, score=SCORE_SIGMOID,
                                 renormalize=True, bias_mode=BIAS_SELECT_ONLY,
                                 bias_kind="uniform0.1")
-    # the V3 layer's matrix shapes and rows per expert (T K' / N' = 256) with 1/16 of its
+    # the V3 layer's matrix shapes and rows per expert (T K' / N' = 256) with 1/8 of its
     # experts: small enough for profiler captures, weights still far above L2
-    c["v3_slice"] = c["v3_prefill"].replace(name="v3_slice", T=512, n_routed=16)
+    c["v3_slice"] = c["v3_prefill"].replace(name="v3_slice", T=1024, n_routed=32)
     for t in (16, 64, 256):
         c[f"v4_decode_t{t}"] = MoEConfig(f"v4_decode_t{t}", T=t, d_model=7168, n_routed=384,
                                          top_k=9, d_ff=2048, n_shared=1, d_ff_shared=2048,
