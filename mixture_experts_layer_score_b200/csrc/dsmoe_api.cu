@@ -501,7 +501,8 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
     sa.P_part = h->P_part;
     sa.scores_dbg = a.scores_dbg;
     sa.status = h->status;
-    sel_grid = dsmoe::select_grid(T, kSelectMaxBlocks / 4);
+    // two blocks per SM: enough warps for the tokens, few partial rows for the scan
+    sel_grid = dsmoe::select_grid(T, h->num_sms / 2 > 0 ? h->num_sms / 2 : 1);
     CUDA_TRY(dsmoe::launch_select(sa, sel_grid, s));
     h->launches += 2;
   }

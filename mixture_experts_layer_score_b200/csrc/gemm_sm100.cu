@@ -51,17 +51,17 @@ constexpr int kMaxGroups = 8 + 512;
 constexpr uint32_t kWBytes = 2 * kFeat * kBK * 2;  // 32 KB: two 128-row weight halves
 constexpr uint32_t kStageRow = 33;  // epilogue staging rows padded to 33 words
 
-// Tile geometry of each projection. Gate/up (long K): 256-token tiles, one accumulator
-// of two 256-column chains, 3 stages of 64 KB: 15.6 KB staged per million MACs. Down
-// (short K): 128-token tiles, two accumulators so the epilogue overlaps the next tile's
-// MMAs, 4 stages of 48 KB.
+// Tile geometry of each projection: up to 128 tokens per tile, two accumulators (each two
+// 128-column chains) so the epilogue of one tile overlaps the MMAs of the next, and a
+// 4-stage ring of 48 KB. (256-token tiles with one accumulator stage fewer bytes per MAC
+// but measured slower at every shape tried: the epilogue no longer overlaps the MMAs.)
 template <bool kSwiGLU>
 struct Geo {
   static constexpr int kTok = kSwiGLU ? kGemmGateUpTokenTile : kGemmDownTokenTile;
   static constexpr uint32_t kChainCols = kTok;
   static constexpr uint32_t kAccCols = 2 * kChainCols;
   static constexpr int kBufs = static_cast<int>(kTmemCols / kAccCols);
-  static constexpr int kStages = kSwiGLU ? 3 : 4;
+  static constexpr int kStages = 4;
   static constexpr uint32_t kXBytes = kTok * kBK * 2;
   static constexpr uint32_t kStageBytes = kWBytes + kXBytes;
   static constexpr uint32_t kOffW = 0;

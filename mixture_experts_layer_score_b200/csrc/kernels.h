@@ -116,7 +116,7 @@ cudaError_t launch_combine(const bf16* x, const float* Hs, const bf16* Y, const 
 // ---------------------------------------------------------------- grouped GEMM (gemm_sm100.cu)
 // Tokens per grouped-GEMM tile of each projection (the row box of its token-side
 // tensor maps).
-constexpr int kGemmGateUpTokenTile = 256;
+constexpr int kGemmGateUpTokenTile = 128;
 constexpr int kGemmDownTokenTile = 128;
 struct GemmArgs {
   CUtensorMap a_routed;   // 2D [rows, K] activations of routed slots, box (64, token tile)

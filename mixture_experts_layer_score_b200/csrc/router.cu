@@ -80,19 +80,23 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const bf16* __restri
 int router_logits_splits(int T, int N, int d, int num_sms) {
   const int tiles = ((T + kRTM - 1) / kRTM) * ((N + kRTN - 1) / kRTN);
   int splits = (2 * num_sms + tiles - 1) / tiles;  // about two CTAs per SM
-  const int max_splits = d / kRTK;
-  if (splits > max_splits) splits = max_splits;
+  const int steps = d / kRTK;
+  if (splits > steps) splits = steps;
   if (splits > kRouterMaxSplits) splits = kRouterMaxSplits;
   if (splits < 1) splits = 1;
-  return splits;
+  // the launch covers d with slices of ceil(steps/splits) k-steps: only that many slices
+  // are non-empty, and the select kernel adds exactly the slices written
+  const int per = (steps + splits - 1) / splits;
+  return (steps + per - 1) / per;
 }
 
 cudaError_t launch_router_logits(const bf16* x, const bf16* W_router, int T, int N, int d, int splits,
                                  float* logits, cudaStream_t s) {
-  // slice length: a multiple of the 32-wide k step covering d in `splits` slices
+  // slice length: a multiple of the 32-wide k step covering d in `splits` slices (a
+  // count from router_logits_splits, so that every slice is non-empty)
   const int kc = ((d / kRTK + splits - 1) / splits) * kRTK;
-  const int used = (d + kc - 1) / kc;
-  dim3 grid((T + kRTM - 1) / kRTM, (N + kRTN - 1) / kRTN, used);
+  if ((d + kc - 1) / kc != splits) return cudaErrorInvalidValue;
+  dim3 grid((T + kRTM - 1) / kRTM, (N + kRTN - 1) / kRTN, splits);
   router_logits_kernel<<<grid, 256, 0, s>>>(x, W_router, T, N, d, kc, logits);
   return cudaGetLastError();
 }

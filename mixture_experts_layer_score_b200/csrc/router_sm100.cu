@@ -248,7 +248,11 @@ int router_tc_splits(int T, int d, int num_sms) {
   const int kb = d / kBK;
   if (s > kb) s = kb;
   if (s > kRouterMaxSplits) s = kRouterMaxSplits;
-  return s < 1 ? 1 : s;
+  if (s < 1) s = 1;
+  // every slice must hold at least one K block: with ceil(kb/s) blocks per slice, only
+  // ceil(kb / ceil(kb/s)) slices are non-empty
+  const int per = (kb + s - 1) / s;
+  return (kb + per - 1) / per;
 }
 
 cudaError_t launch_router_tc(const RouterTcArgs& a, int grid, cudaStream_t s) {

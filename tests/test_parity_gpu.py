@@ -193,3 +193,23 @@ def test_stage_timing_and_launch_count():
     layer.forward(gpu["x"][:100].contiguous())  # CUDA-core router logits below 256 tokens
     assert M.dsmoe_launch_count(layer.handle) - n1 == 7
     layer.close()
+
+
+def test_varying_batch_sizes_on_one_handle():
+    """One handle serving batches of different sizes (both routers, several split counts)
+    gives the same outputs as a fresh handle per batch: no state of an earlier call leaks
+    into a later one."""
+    cfg = W.get_config("ds2b")
+    gpu, _ = make_case(cfg, 2000)
+    layer = M.DSMoE(M.cfg_from(cfg, 2000), gpu)
+    for T in (2000, 100, 700, 16, 300, 2000):
+        x = gpu["x"][:T].contiguous()
+        a = layer.forward(x, with_scores=True)
+        torch.cuda.synchronize()
+        fresh = M.DSMoE(M.cfg_from(cfg, T), gpu)
+        b = fresh.forward(x, with_scores=True)
+        torch.cuda.synchronize()
+        fresh.close()
+        for k in ("h", "topk_idx", "gates", "counts", "f", "scores"):
+            assert torch.equal(a[k], b[k]), (T, k)
+    layer.close()
