@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=None, help="steps of the end-to-end leg (default: --steps)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample", type=int, default=None, help="tokens in the oracle's timed sample")
+    ap.add_argument("--gemm", default="pair", choices=["pair", "single"],
+                    help="grouped-GEMM kernel: CTA pairs (default) or one CTA per tile")
     return ap.parse_args()
 
 
@@ -62,19 +64,21 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-KERNEL_SOURCES = {"gemm_gate_up": "mixture_experts_layer_score_b200/csrc/gemm_sm100.cu",
-                  "gemm_down": "mixture_experts_layer_score_b200/csrc/gemm_sm100.cu",
+KERNEL_SOURCES = {"gemm_gate_up": "mixture_experts_layer_score_b200/csrc/gemm_pair_sm100.cu",
+                  "gemm_down": "mixture_experts_layer_score_b200/csrc/gemm_pair_sm100.cu",
                   "router": "mixture_experts_layer_score_b200/csrc/router_sm100.cu"}
+SINGLE_CTA_GEMM_SOURCE = "mixture_experts_layer_score_b200/csrc/gemm_sm100.cu"
 
 
-def source_digest(stage):
+def source_digest(stage, gemm="pair"):
     import hashlib
-    path = os.path.join(ROOT, KERNEL_SOURCES[stage])
+    src = SINGLE_CTA_GEMM_SOURCE if (gemm == "single" and stage.startswith("gemm")) else KERNEL_SOURCES[stage]
+    path = os.path.join(ROOT, src)
     with open(path, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def captured_traffic(stage, weight_bytes):
+def captured_traffic(stage, weight_bytes, gemm="pair"):
     """DRAM bytes per launch of `stage` from the committed ncu summary
     (profiles/ncu_dram_traffic.txt): the captured launch's DRAM read+write bytes divided by
     the algorithmic weight bytes it streamed, scaled to this launch's weight bytes (the
@@ -84,7 +88,7 @@ def captured_traffic(stage, weight_bytes):
     path = os.path.join(ROOT, "profiles", "ncu_dram_traffic.txt")
     if not os.path.exists(path):
         return None
-    digest = source_digest(stage)
+    digest = source_digest(stage, gemm)
     with open(path) as f:
         for line in f:
             parts = line.split()
@@ -272,6 +276,7 @@ def run_native(args, cfg):
             inp["token_ids"] = torch.randint(0, W.TOKEN_VOCAB, (cfg.T,), generator=g, device=dev,
                                              dtype=torch.int64).to(torch.int32)
     layer = M.DSMoE(M.cfg_from(cfg, cfg.T), inp, device=local)
+    M.dsmoe_set_gemm_kernel(layer.handle, M.DSMOE_GEMM_SINGLE if args.gemm == "single" else M.DSMOE_GEMM_PAIR)
     out = layer.alloc_outputs(cfg.T)
     T_total = cfg.T * world
     stream = torch.cuda.current_stream(dev)
@@ -344,7 +349,7 @@ def run_native(args, cfg):
         achieved = weight_bytes[dom] / (dom_ms / 1e3) / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak}
-    traffic = captured_traffic(dom, weight_bytes[dom])
+    traffic = captured_traffic(dom, weight_bytes[dom], args.gemm)
     roof.update({"kernel": dom, "kernel_ms": dom_ms, "traffic": traffic,
                  "peak_source": f"{peak_src} ({'bf16_tflops_sustained' if roof['bound'] == 'tensor' else 'hbm_gbs'})",
                  "algorithmic": {"flops": flops[dom], "weight_bytes": weight_bytes[dom]}})
@@ -410,7 +415,7 @@ def run_native(args, cfg):
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; random weights of the layer's shape)",
-                "config": config_block(cfg, world), "roofline": roof, "cpu_baseline": cpu_base, "e2e": e2e,
+                "config": dict(config_block(cfg, world), gemm_kernel=args.gemm), "roofline": roof, "cpu_baseline": cpu_base, "e2e": e2e,
                 "gpu_launches": int(launches), "clocks": clock_info,
                 "layer_tflops": layer_tflops, "stage_ms": stage_ms, "experts_touched": touched}
         print(json.dumps(line), flush=True)

@@ -218,6 +218,21 @@ dsmoe_status dsmoe_get_status(dsmoe_handle* h);
 /* Bound on every in-kernel wait, in nanoseconds (default 2e9). */
 dsmoe_status dsmoe_set_wait_limit(dsmoe_handle* h, uint64_t ns);
 
+/* Which kernel computes the two grouped expert GEMMs of dsmoe_forward (the gate/up
+ * projection with SiLU(gate) * up, and the down projection; DeepSeekMoE summary,
+ * shared-expert layer equation). Both accumulate each output in fp32 over K in
+ * 16-element MMA steps, in the same order, and share the epilogue arithmetic.
+ *   DSMOE_GEMM_PAIR   (default) CTA pairs on neighbouring SMs share one M=256 MMA per
+ *                     K step, tiles of up to 256 tokens.
+ *   DSMOE_GEMM_SINGLE one CTA per tile, M=128 MMAs, tiles of up to 128 tokens.
+ * dsmoe_set_gemm_kernel returns DSMOE_ERR_UNSUPPORTED when the pair kernel cannot be
+ * launched on the device (the handle then keeps DSMOE_GEMM_SINGLE), and
+ * DSMOE_ERR_INVALID_ARG for another kind. dsmoe_get_gemm_kernel returns the kind in use
+ * (-1 for a NULL handle). */
+enum { DSMOE_GEMM_PAIR = 0, DSMOE_GEMM_SINGLE = 1 };
+dsmoe_status dsmoe_set_gemm_kernel(dsmoe_handle* h, int32_t kind);
+int32_t dsmoe_get_gemm_kernel(dsmoe_handle* h);
+
 /* Per-stage timing: while enabled, each forward with T > 0 records CUDA events on its
  * stream at every stage boundary (no synchronisation). dsmoe_stage_times waits for
  * the recorded events and writes, per stage, the mean duration in ms over the last

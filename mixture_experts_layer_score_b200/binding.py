@@ -19,6 +19,7 @@ DSMOE_OK, DSMOE_ERR_INVALID_ARG, DSMOE_ERR_UNSUPPORTED, DSMOE_ERR_WORKSPACE, DSM
     DSMOE_ERR_DEVICE_TIMEOUT = range(6)
 DSMOE_SCORE_SOFTMAX, DSMOE_SCORE_SIGMOID, DSMOE_SCORE_SQRT_SOFTPLUS, DSMOE_ROUTE_HASH = range(4)
 DSMOE_BIAS_NONE, DSMOE_BIAS_SELECT_ONLY, DSMOE_BIAS_IN_LOGITS = range(3)
+DSMOE_GEMM_PAIR, DSMOE_GEMM_SINGLE = range(2)
 
 ABI_FUNCTIONS = (
     "dsmoe_abi_version", "dsmoe_status_string", "dsmoe_last_error", "dsmoe_check_config",
@@ -26,7 +27,7 @@ ABI_FUNCTIONS = (
     "dsmoe_balance_stats", "dsmoe_get_status", "dsmoe_set_wait_limit", "dsmoe_set_timing",
     "dsmoe_stage_times", "dsmoe_stage_name", "dsmoe_launch_count", "dsmoe_workspace_tensor",
     "dsmoe_balance_losses", "dsmoe_sequence_balance", "dsmoe_bias_update",
-    "dsmoe_route_noalloc",
+    "dsmoe_route_noalloc", "dsmoe_set_gemm_kernel", "dsmoe_get_gemm_kernel",
 )
 
 
@@ -65,6 +66,8 @@ def _load():
         "dsmoe_get_status": (ctypes.c_int, [vp]),
         "dsmoe_set_wait_limit": (ctypes.c_int, [vp, u64]),
         "dsmoe_set_timing": (ctypes.c_int, [vp, i32]),
+        "dsmoe_set_gemm_kernel": (ctypes.c_int, [vp, i32]),
+        "dsmoe_get_gemm_kernel": (i32, [vp]),
         "dsmoe_stage_times": (ctypes.c_int, [vp, ctypes.POINTER(ctypes.c_float), i32, ctypes.POINTER(i32)]),
         "dsmoe_stage_name": (ctypes.c_char_p, [i32]),
         "dsmoe_launch_count": (ctypes.c_int, [vp, ctypes.POINTER(i64)]),
@@ -185,6 +188,14 @@ def dsmoe_get_status(handle) -> int:
 
 def dsmoe_set_wait_limit(handle, ns: int) -> None:
     _check(_lib.dsmoe_set_wait_limit(handle, int(ns)), "dsmoe_set_wait_limit")
+
+
+def dsmoe_set_gemm_kernel(handle, kind: int) -> None:
+    _check(_lib.dsmoe_set_gemm_kernel(handle, int(kind)), "dsmoe_set_gemm_kernel")
+
+
+def dsmoe_get_gemm_kernel(handle) -> int:
+    return int(_lib.dsmoe_get_gemm_kernel(handle))
 
 
 def dsmoe_set_timing(handle, enable: bool) -> None:

@@ -169,6 +169,8 @@ struct dsmoe_handle {
   dsmoe_cfg cfg;
   int device = 0;
   int num_sms = 148;
+  int pair_clusters[2] = {0, 0};  // co-resident CTA pairs of the pair GEMM (down, gate/up)
+  int32_t gemm_kernel = DSMOE_GEMM_PAIR;
   uint64_t wait_ns = kDefaultWaitNs;
   char* ws = nullptr;
   Layout L;
@@ -183,8 +185,11 @@ struct dsmoe_handle {
   int32_t *ids_stage, *topk_stage, *counts_stage;
   float *gates_stage, *f_stage, *P_stage;
   CUtensorMap tm_xp, tm_a1, tm_a1s;
-  const void* wkey[7] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
-  CUtensorMap tm_w[7];  // W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, W_router
+  // weight maps, cached per pointer: W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, W_router
+  // for the one-CTA GEMM and the router, then the six expert weights for the pair GEMM
+  static constexpr int kMaps = 13;
+  const void* wkey[kMaps] = {};
+  CUtensorMap tm_w[kMaps];
   int rt_chunks = 1, rt_nc = 16;
   uint32_t rt_cols = 32;
   bool timing = false;
@@ -286,6 +291,9 @@ DSMOE_EXPORT dsmoe_status dsmoe_create(const dsmoe_cfg* cfg, int32_t device, dsm
   if (h->cfg.score == DSMOE_ROUTE_HASH && h->cfg.hash_mod == 0) h->cfg.hash_mod = h->cfg.n_routed;
   h->device = device;
   h->num_sms = prop.multiProcessorCount;
+  h->pair_clusters[0] = dsmoe::grouped_gemm_pair_max_clusters(false);
+  h->pair_clusters[1] = dsmoe::grouped_gemm_pair_max_clusters(true);
+  if (h->pair_clusters[0] < 1 || h->pair_clusters[1] < 1) h->gemm_kernel = DSMOE_GEMM_SINGLE;
   dsmoe::router_tc_shape(cfg->n_routed, &h->rt_chunks, &h->rt_nc, &h->rt_cols);
   h->L = plan(h->cfg);
   cudaError_t e = cudaMalloc(&h->ws, h->L.total);
@@ -404,6 +412,14 @@ const CUtensorMap* weight_map(dsmoe_handle* h, int which, const void* ptr, bool*
       case 4: r = map_3d(&h->tm_w[which], ptr, c.d_model, c.d_ff_shared, c.n_shared, 128); break;
       case 5: r = map_3d(&h->tm_w[which], ptr, c.d_ff_shared, c.d_model, c.n_shared, 256); break;
       case 6: r = map_2d(&h->tm_w[which], ptr, c.d_model, c.n_routed, static_cast<uint32_t>(h->rt_nc)); break;
+      case 7:
+      case 8: r = map_3d(&h->tm_w[which], ptr, c.d_model, c.d_ff, c.n_routed, dsmoe::kGemmPairGateUpRows); break;
+      case 9: r = map_3d(&h->tm_w[which], ptr, c.d_ff, c.d_model, c.n_routed, 128); break;
+      case 10:
+      case 11:
+        r = map_3d(&h->tm_w[which], ptr, c.d_model, c.d_ff_shared, c.n_shared, dsmoe::kGemmPairGateUpRows);
+        break;
+      case 12: r = map_3d(&h->tm_w[which], ptr, c.d_ff_shared, c.d_model, c.n_shared, 128); break;
     }
     if (!r) {
       h->wkey[which] = nullptr;
@@ -436,12 +452,14 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
 
   // tensor maps that depend on the call's pointers
   bool ok = true;
-  const CUtensorMap* m_wg = weight_map(h, 0, a.W_gate, &ok);
-  const CUtensorMap* m_wu = weight_map(h, 1, a.W_up, &ok);
-  const CUtensorMap* m_wd = weight_map(h, 2, a.W_down, &ok);
-  const CUtensorMap* m_swg = Ks ? weight_map(h, 3, a.Ws_gate, &ok) : m_wg;
-  const CUtensorMap* m_swu = Ks ? weight_map(h, 4, a.Ws_up, &ok) : m_wu;
-  const CUtensorMap* m_swd = Ks ? weight_map(h, 5, a.Ws_down, &ok) : m_wd;
+  const bool pair = h->gemm_kernel == DSMOE_GEMM_PAIR;
+  const int wm = pair ? 7 : 0;  // first weight map of the chosen GEMM kernel
+  const CUtensorMap* m_wg = weight_map(h, wm + 0, a.W_gate, &ok);
+  const CUtensorMap* m_wu = weight_map(h, wm + 1, a.W_up, &ok);
+  const CUtensorMap* m_wd = weight_map(h, wm + 2, a.W_down, &ok);
+  const CUtensorMap* m_swg = Ks ? weight_map(h, wm + 3, a.Ws_gate, &ok) : m_wg;
+  const CUtensorMap* m_swu = Ks ? weight_map(h, wm + 4, a.Ws_up, &ok) : m_wu;
+  const CUtensorMap* m_swd = Ks ? weight_map(h, wm + 5, a.Ws_down, &ok) : m_wd;
   CUtensorMap m_x, m_x_router;  // token rows of x: GEMM tiles, and the router's 128-token tiles
   ok = ok && map_2d(&m_x, a.x, d, T, dsmoe::kGemmGateUpTokenTile) && map_2d(&m_x_router, a.x, d, T, 128);
   if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map of this call");
@@ -559,11 +577,16 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
     g.shared_col_stride = Fs;
     g.status = h->status;
     g.wait_limit_ns = h->wait_ns;
-    const int64_t tt = dsmoe::kGemmGateUpTokenTile;
+    const int64_t tt = pair ? dsmoe::kGemmPairTokenTile : dsmoe::kGemmGateUpTokenTile;
     const int64_t bound = (cdiv(S, tt) + N) * static_cast<int64_t>(g.n_tiles_routed) +
                           static_cast<int64_t>(Ks) * cdiv(T, tt) * g.n_tiles_shared;
-    const int grid = static_cast<int>(bound < h->num_sms ? bound : h->num_sms);
-    CUDA_TRY(dsmoe::launch_grouped_gemm(true, g, grid, s));
+    if (pair) {
+      const int clusters = static_cast<int>(bound < h->pair_clusters[1] ? bound : h->pair_clusters[1]);
+      CUDA_TRY(dsmoe::launch_grouped_gemm_pair(true, g, clusters, s));
+    } else {
+      const int grid = static_cast<int>(bound < h->num_sms ? bound : h->num_sms);
+      CUDA_TRY(dsmoe::launch_grouped_gemm(true, g, grid, s));
+    }
     h->launches += 1;
   }
   CUDA_TRY(mark(5));
@@ -597,11 +620,16 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
     g.shared_col_stride = 0;
     g.status = h->status;
     g.wait_limit_ns = h->wait_ns;
-    const int64_t tt = dsmoe::kGemmDownTokenTile;
+    const int64_t tt = pair ? dsmoe::kGemmPairTokenTile : dsmoe::kGemmDownTokenTile;
     const int64_t bound = (cdiv(S, tt) + N) * static_cast<int64_t>(g.n_tiles_routed) +
                           static_cast<int64_t>(g.n_shared_groups) * cdiv(T, tt) * g.n_tiles_shared;
-    const int grid = static_cast<int>(bound < h->num_sms ? bound : h->num_sms);
-    CUDA_TRY(dsmoe::launch_grouped_gemm(false, g, grid, s));
+    if (pair) {
+      const int clusters = static_cast<int>(bound < h->pair_clusters[0] ? bound : h->pair_clusters[0]);
+      CUDA_TRY(dsmoe::launch_grouped_gemm_pair(false, g, clusters, s));
+    } else {
+      const int grid = static_cast<int>(bound < h->num_sms ? bound : h->num_sms);
+      CUDA_TRY(dsmoe::launch_grouped_gemm(false, g, grid, s));
+    }
     h->launches += 1;
   }
   CUDA_TRY(mark(6));
@@ -705,6 +733,18 @@ DSMOE_EXPORT dsmoe_status dsmoe_set_wait_limit(dsmoe_handle* h, uint64_t ns) {
   h->wait_ns = ns;
   return DSMOE_OK;
 }
+
+DSMOE_EXPORT dsmoe_status dsmoe_set_gemm_kernel(dsmoe_handle* h, int32_t kind) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  if (kind != DSMOE_GEMM_PAIR && kind != DSMOE_GEMM_SINGLE)
+    return fail(DSMOE_ERR_INVALID_ARG, "unknown GEMM kernel kind %d", kind);
+  if (kind == DSMOE_GEMM_PAIR && (h->pair_clusters[0] < 1 || h->pair_clusters[1] < 1))
+    return fail(DSMOE_ERR_UNSUPPORTED, "the CTA-pair GEMM cannot be launched on this device");
+  h->gemm_kernel = kind;
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT int32_t dsmoe_get_gemm_kernel(dsmoe_handle* h) { return h ? h->gemm_kernel : -1; }
 
 DSMOE_EXPORT dsmoe_status dsmoe_set_timing(dsmoe_handle* h, int32_t enable) {
   if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");

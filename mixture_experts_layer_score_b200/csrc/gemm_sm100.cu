@@ -35,7 +35,7 @@
 // Every wait is bounded (wait_limit_ns); a role that gives up raises a CTA-wide abort
 // flag and a bit of the device status word, the CTA lets in-flight TMA loads and MMAs
 // finish (again bounded), frees its TMEM and returns.
-#include "kernels.h"
+#include "grouped_tiles.cuh"
 #include "sm100_ptx.cuh"
 
 namespace dsmoe {
@@ -47,7 +47,6 @@ constexpr int kMmaK = 16;       // K of each bf16 tcgen05.mma
 constexpr int kThreads = 192;
 constexpr int kEpiThreads = 128;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kMaxGroups = 8 + 512;
 constexpr uint32_t kWBytes = 2 * kFeat * kBK * 2;  // 32 KB: two 128-row weight halves
 constexpr uint32_t kStageRow = 33;  // epilogue staging rows padded to 33 words
 
@@ -70,55 +69,12 @@ struct Geo {
   static constexpr uint32_t kNumBars = 2 * kStages + 2 + 2 + 1;
   static constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
   static constexpr uint32_t kOffTiles = kOffMisc + 16;
-  static constexpr uint32_t kOffEpi = (kOffTiles + (kMaxGroups + 1) * 4 + 15) & ~15u;
+  static constexpr uint32_t kOffEpi = (kOffTiles + (kGemmMaxGroups + 1) * 4 + 15) & ~15u;
   static constexpr uint32_t kSmemUsed = kOffEpi + 4 * 32 * kStageRow * 4;
   static constexpr size_t kSmemBytes = kSmemUsed + 1024;  // slack to align the ring to 1024 bytes
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(kBufs >= 1 && kTok % 32 == 0 && kTok <= 256, "tile geometry");
 };
-
-struct Tile {
-  int shared;   // 1: shared-expert group
-  int group;    // group index (shared groups first)
-  int expert;   // expert index inside its kind
-  int row0;     // first A / output row of the tile
-  int m_valid;  // valid rows in the tile
-  int n_blk;    // output tile index along N
-  int kb_n;     // K blocks
-};
-
-template <int kBM>
-__device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int32_t* tile_start, int G, int tile) {
-  int lo = 0, hi = G - 1;
-  while (lo < hi) {  // last group whose first tile is <= tile
-    const int mid = (lo + hi + 1) >> 1;
-    if (tile_start[mid] <= tile) lo = mid;
-    else hi = mid - 1;
-  }
-  Tile t;
-  t.group = lo;
-  int M, base;
-  if (lo < a.n_shared_groups) {
-    t.shared = 1;
-    t.expert = lo;
-    M = a.m_shared;
-    base = 0;
-    t.kb_n = a.kb_shared;
-  } else {
-    t.shared = 0;
-    t.expert = lo - a.n_shared_groups;
-    base = a.offsets[t.expert];
-    M = a.offsets[t.expert + 1] - base;
-    t.kb_n = a.kb_routed;
-  }
-  const int mt = (M + kBM - 1) / kBM;
-  const int local = tile - tile_start[lo];
-  const int m_blk = local % mt;
-  t.n_blk = local / mt;
-  t.row0 = base + m_blk * kBM;
-  t.m_valid = min(kBM, M - m_blk * kBM);
-  return t;
-}
 
 template <bool kSwiGLU>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs a) {
@@ -142,22 +98,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = a.n_shared_groups + a.n_routed;
 
-  // tiles of each group, then an inclusive prefix -> first tile of each group
-  for (int g = threadIdx.x; g < G; g += kThreads) {
-    int M, nt;
-    if (g < a.n_shared_groups) {
-      M = a.m_shared;
-      nt = a.n_tiles_shared;
-    } else {
-      const int e = g - a.n_shared_groups;
-      M = a.offsets[e + 1] - a.offsets[e];
-      nt = a.n_tiles_routed;
-    }
-    M = max(M, 0);
-    tile_start[g + 1] = ((M + G_::kTok - 1) / G_::kTok) * nt;
-  }
+  tile_counts<G_::kTok>(a, tile_start, G);
   if (threadIdx.x == 0) {
-    tile_start[0] = 0;
     *abort_flag = 0;
     *never_flag = 0;
     for (int s = 0; s < G_::kStages; ++s) {
@@ -176,20 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
     tmem_relinquish();
   }
   __syncthreads();
-  if (warp == 0) {
-    int carry = 0;
-    for (int b0 = 1; b0 <= G; b0 += 32) {
-      const int i = b0 + lane;
-      int v = (i <= G) ? tile_start[i] : 0;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += n;
-      }
-      if (i <= G) tile_start[i] = v + carry;
-      carry += __shfl_sync(0xffffffffu, v, 31);
-    }
-  }
+  if (warp == 0) tile_scan(tile_start, G, lane);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -402,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
 }  // namespace
 
 cudaError_t launch_grouped_gemm(bool swiglu, const GemmArgs& a, int grid, cudaStream_t s) {
-  if (a.n_shared_groups + a.n_routed > kMaxGroups) return cudaErrorInvalidValue;
+  if (a.n_shared_groups + a.n_routed > kGemmMaxGroups) return cudaErrorInvalidValue;
   if (grid < 1) grid = 1;
   cudaError_t e;
   if (swiglu) {

@@ -116,6 +116,7 @@ cudaError_t launch_combine(const bf16* x, const float* Hs, const bf16* Y, const 
 // ---------------------------------------------------------------- grouped GEMM (gemm_sm100.cu)
 // Tokens per grouped-GEMM tile of each projection (the row box of its token-side
 // tensor maps).
+constexpr int kGemmMaxGroups = 8 + 512;  // shared + routed groups of one grouped GEMM
 constexpr int kGemmGateUpTokenTile = 128;
 constexpr int kGemmDownTokenTile = 128;
 struct GemmArgs {
@@ -144,6 +145,17 @@ struct GemmArgs {
   uint64_t wait_limit_ns;
 };
 cudaError_t launch_grouped_gemm(bool swiglu, const GemmArgs& a, int grid, cudaStream_t s);
+
+// The same grouped GEMM on CTA pairs (clusters of two, tcgen05 cta_group::2): a pair
+// computes 128 features (gate/up) or 256 output rows (down) by up to
+// kGemmPairTokenTile tokens; each CTA stages 128 weight rows and half of the tile's
+// token rows. Weight maps: box (64, kGemmPairGateUpRows) for gate/up, (64, 128) for
+// down; token maps: box (64, 128).
+constexpr int kGemmPairTokenTile = 256;
+constexpr int kGemmPairGateUpRows = 64;
+// Largest number of co-resident pairs (0 when the pair kernel cannot be launched).
+int grouped_gemm_pair_max_clusters(bool swiglu);
+cudaError_t launch_grouped_gemm_pair(bool swiglu, const GemmArgs& a, int clusters, cudaStream_t s);
 
 // ---------------------------------------------------------------- errors (dsmoe_api.cu)
 // Record the calling thread's last-error message (read back by dsmoe_last_error).

@@ -95,6 +95,18 @@ __device__ __forceinline__ bool mbar_wait_warp_sleepy(uint64_t* bar, uint32_t pa
   return ok != 0;
 }
 
+// The same wait without back-off, for a warp on the critical path: lane 0 polls, the
+// verdict is broadcast and every lane then observes the completed phase itself (so each
+// lane acquires what the arrivals released). Must be called by all 32 lanes.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                               volatile int* abort_flag) {
+  uint32_t ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait_bounded(bar, parity, limit_ns, abort_flag) ? 1u : 0u;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) (void)mbar_try_wait(bar, parity);
+  return ok != 0;
+}
+
 // ------------------------------------------------------------------------------------
 // TMA (tiled tensor loads into shared memory, completion counted on an mbarrier)
 // ------------------------------------------------------------------------------------

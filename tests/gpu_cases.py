@@ -44,9 +44,12 @@ def make_case(cfg: W.MoEConfig, T: int, seed: int = 0, gen_device: str = "cpu"):
     return gpu, cpu
 
 
-def run_cuda(cfg: W.MoEConfig, gpu: dict, T: int, max_tokens: int = None, with_scores: bool = True):
+def run_cuda(cfg: W.MoEConfig, gpu: dict, T: int, max_tokens: int = None, with_scores: bool = True,
+             gemm_kernel: int = None):
     layer = M.DSMoE(M.cfg_from(cfg, max_tokens or max(T, 1)), gpu)
     try:
+        if gemm_kernel is not None:
+            M.dsmoe_set_gemm_kernel(layer.handle, gemm_kernel)
         out = layer.forward(gpu["x"], token_ids=gpu.get("token_ids"), with_scores=with_scores)
         torch.cuda.synchronize()
         st = M.dsmoe_get_status(layer.handle)

@@ -94,3 +94,6 @@ def test_null_handle_is_rejected_without_a_gpu():
     lib.dsmoe_destroy(None)  # documented no-op
     with pytest.raises(M.DsmoeError):
         M.dsmoe_set_timing(None, 1)
+    with pytest.raises(M.DsmoeError):
+        M.dsmoe_set_gemm_kernel(None, M.DSMOE_GEMM_SINGLE)
+    assert M.dsmoe_get_gemm_kernel(None) == -1

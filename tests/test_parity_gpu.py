@@ -19,9 +19,9 @@ if not torch.cuda.is_available():
     pytest.skip("no GPU", allow_module_level=True)
 
 
-def _check(cfg, T, rows_n=None, gen_device="cpu", seed=0):
+def _check(cfg, T, rows_n=None, gen_device="cpu", seed=0, gemm_kernel=None):
     gpu, cpu = make_case(cfg, T, seed=seed, gen_device=gen_device)
-    out = run_cuda(cfg, gpu, T)
+    out = run_cuda(cfg, gpu, T, gemm_kernel=gemm_kernel)
     ref = PAR.reference_selection(cfg, cpu, out["topk_idx"], out["scores"])
     rr = PAR.check_routing(cfg, ref, out, T)
     rows = np.arange(T) if rows_n is None else sample_rows(T, rows_n)
@@ -38,6 +38,31 @@ SMALL = [("tiny", 512, None), ("tiny", 131, None), ("gshard_a", 1000, None), ("g
 @pytest.mark.parametrize("name,T,rows", SMALL, ids=[f"{n}-T{t}" for n, t, _ in SMALL])
 def test_small_parity(name, T, rows):
     _check(W.get_config(name), T, rows)
+
+
+SINGLE_CTA = [("tiny", 131), ("gshard_c", 1000), ("v3_prefill", 300), ("v4_decode_t16", 16)]
+
+
+@pytest.mark.parametrize("name,T", SINGLE_CTA, ids=[f"{n}-T{t}" for n, t in SINGLE_CTA])
+def test_small_parity_single_cta_gemm(name, T):
+    """The one-CTA grouped GEMM (the alternative to the default CTA-pair kernel)."""
+    _check(W.get_config(name), T, 48, gemm_kernel=M.DSMOE_GEMM_SINGLE)
+
+
+def test_gemm_kernels_agree():
+    """The CTA-pair and one-CTA GEMM kernels on the same inputs: identical routing, and h
+    equal up to the accumulation order inside the tensor core."""
+    cfg = W.get_config("gshard_b").replace(T=1500)
+    gpu, _ = make_case(cfg, cfg.T)
+    a = run_cuda(cfg, gpu, cfg.T, gemm_kernel=M.DSMOE_GEMM_PAIR)
+    b = run_cuda(cfg, gpu, cfg.T, gemm_kernel=M.DSMOE_GEMM_SINGLE)
+    for k in ("topk_idx", "gates", "counts", "f", "P"):
+        assert torch.equal(a[k], b[k]), k
+    d = (a["h"].float() - b["h"].float()).abs()
+    rms = b["h"].float().pow(2).mean().sqrt()
+    print("pair vs single: bitwise equal rows", int((d.amax(1) == 0).sum()), "of", cfg.T,
+          "max|diff|", float(d.max()), "rms", float(rms))
+    assert float(d.max()) <= PAR.H_TOL * float(rms)
 
 
 FULL = [("gshard_a", 128), ("gshard_b", 128), ("gshard_c", 128), ("ds2b", 128), ("v3_prefill", 32),
@@ -174,6 +199,19 @@ def test_balance_stats_entry_point():
     assert torch.equal(c1 + h2["counts"], o["counts"])
     assert torch.equal(f2, o["f"])
     assert torch.allclose(P2, o["P"], rtol=1e-5, atol=1e-7)
+    layer.close()
+
+
+def test_gemm_kernel_selector():
+    cfg = W.get_config("tiny")
+    gpu, _ = make_case(cfg, 8)
+    layer = M.DSMoE(M.cfg_from(cfg, 8), gpu)
+    assert M.dsmoe_get_gemm_kernel(layer.handle) == M.DSMOE_GEMM_PAIR  # the default on B200
+    M.dsmoe_set_gemm_kernel(layer.handle, M.DSMOE_GEMM_SINGLE)
+    assert M.dsmoe_get_gemm_kernel(layer.handle) == M.DSMOE_GEMM_SINGLE
+    with pytest.raises(M.DsmoeError) as ei:
+        M.dsmoe_set_gemm_kernel(layer.handle, 7)
+    assert ei.value.status == M.DSMOE_ERR_INVALID_ARG
     layer.close()
 
 
