@@ -50,8 +50,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=None, help="steps of the end-to-end leg (default: --steps)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample", type=int, default=None, help="tokens in the oracle's timed sample")
-    ap.add_argument("--gemm", default="pair", choices=["pair", "single"],
-                    help="grouped-GEMM kernel: CTA pairs (default) or one CTA per tile")
+    ap.add_argument("--gemm", default="single", choices=["single", "pair"],
+                    help="grouped-GEMM kernel: one CTA per tile (default) or CTA pairs")
     return ap.parse_args()
 
 
@@ -64,21 +64,21 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-KERNEL_SOURCES = {"gemm_gate_up": "mixture_experts_layer_score_b200/csrc/gemm_pair_sm100.cu",
-                  "gemm_down": "mixture_experts_layer_score_b200/csrc/gemm_pair_sm100.cu",
+KERNEL_SOURCES = {"gemm_gate_up": "mixture_experts_layer_score_b200/csrc/gemm_sm100.cu",
+                  "gemm_down": "mixture_experts_layer_score_b200/csrc/gemm_sm100.cu",
                   "router": "mixture_experts_layer_score_b200/csrc/router_sm100.cu"}
-SINGLE_CTA_GEMM_SOURCE = "mixture_experts_layer_score_b200/csrc/gemm_sm100.cu"
+PAIR_GEMM_SOURCE = "mixture_experts_layer_score_b200/csrc/gemm_pair_sm100.cu"
 
 
-def source_digest(stage, gemm="pair"):
+def source_digest(stage, gemm="single"):
     import hashlib
-    src = SINGLE_CTA_GEMM_SOURCE if (gemm == "single" and stage.startswith("gemm")) else KERNEL_SOURCES[stage]
+    src = PAIR_GEMM_SOURCE if (gemm == "pair" and stage.startswith("gemm")) else KERNEL_SOURCES[stage]
     path = os.path.join(ROOT, src)
     with open(path, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def captured_traffic(stage, weight_bytes, gemm="pair"):
+def captured_traffic(stage, weight_bytes, gemm="single"):
     """DRAM bytes per launch of `stage` from the committed ncu summary
     (profiles/ncu_dram_traffic.txt): the captured launch's DRAM read+write bytes divided by
     the algorithmic weight bytes it streamed, scaled to this launch's weight bytes (the

@@ -222,16 +222,32 @@ dsmoe_status dsmoe_set_wait_limit(dsmoe_handle* h, uint64_t ns);
  * projection with SiLU(gate) * up, and the down projection; DeepSeekMoE summary,
  * shared-expert layer equation). Both accumulate each output in fp32 over K in
  * 16-element MMA steps, in the same order, and share the epilogue arithmetic.
- *   DSMOE_GEMM_PAIR   (default) CTA pairs on neighbouring SMs share one M=256 MMA per
- *                     K step, tiles of up to 256 tokens.
- *   DSMOE_GEMM_SINGLE one CTA per tile, M=128 MMAs, tiles of up to 128 tokens.
+ *   DSMOE_GEMM_SINGLE (default) one CTA per tile, M=128 MMAs, tiles of up to 128 tokens.
+ *   DSMOE_GEMM_PAIR   CTA pairs on neighbouring SMs share one M=256 MMA per K step,
+ *                     tiles of up to 256 tokens.
  * dsmoe_set_gemm_kernel returns DSMOE_ERR_UNSUPPORTED when the pair kernel cannot be
- * launched on the device (the handle then keeps DSMOE_GEMM_SINGLE), and
- * DSMOE_ERR_INVALID_ARG for another kind. dsmoe_get_gemm_kernel returns the kind in use
- * (-1 for a NULL handle). */
+ * launched on the device (the handle keeps its kind), and DSMOE_ERR_INVALID_ARG for
+ * another kind. dsmoe_get_gemm_kernel returns the kind in use (-1 for a NULL handle). */
 enum { DSMOE_GEMM_PAIR = 0, DSMOE_GEMM_SINGLE = 1 };
 dsmoe_status dsmoe_set_gemm_kernel(dsmoe_handle* h, int32_t kind);
 int32_t dsmoe_get_gemm_kernel(dsmoe_handle* h);
+
+/* Inference-time selection variants of the DeepSeekMoE summary's expert-specialisation
+ * analysis, applied by later dsmoe_forward / dsmoe_forward_host calls on this handle:
+ *   mask_top = r >= 0 -- per token, the r experts ranked first by the selection key
+ *     (s + b with a selection-only bias, else s; ties to the lower index) are masked out
+ *     before the top-K' choice ("disable the top routed experts");
+ *   k_active in [1, cfg.top_k] -- the number of routed experts each token activates
+ *     ("fewer activated routed experts"): topk_idx and gates are then [T, k_active]
+ *     row-major, gates are renormalised over the kept experts when cfg.renormalize is
+ *     set, and f_i = N'/(k_active T) counts_i (also in dsmoe_balance_stats,
+ *     dsmoe_sequence_balance and dsmoe_bias_update).
+ * Requires mask_top + k_active <= n_routed; hash routing accepts only (0, top_k)
+ * (DSMOE_ERR_UNSUPPORTED otherwise). Defaults (0, cfg.top_k) give the trained router's
+ * selection. P_i (the mean score) does not depend on the variant.
+ * dsmoe_route_noalloc always uses the configuration's plain selection. */
+dsmoe_status dsmoe_set_selection(dsmoe_handle* h, int32_t mask_top, int32_t k_active);
+dsmoe_status dsmoe_get_selection(dsmoe_handle* h, int32_t* mask_top, int32_t* k_active);
 
 /* Per-stage timing: while enabled, each forward with T > 0 records CUDA events on its
  * stream at every stage boundary (no synchronisation). dsmoe_stage_times waits for

@@ -28,6 +28,7 @@ ABI_FUNCTIONS = (
     "dsmoe_stage_times", "dsmoe_stage_name", "dsmoe_launch_count", "dsmoe_workspace_tensor",
     "dsmoe_balance_losses", "dsmoe_sequence_balance", "dsmoe_bias_update",
     "dsmoe_route_noalloc", "dsmoe_set_gemm_kernel", "dsmoe_get_gemm_kernel",
+    "dsmoe_set_selection", "dsmoe_get_selection",
 )
 
 
@@ -68,6 +69,8 @@ def _load():
         "dsmoe_set_timing": (ctypes.c_int, [vp, i32]),
         "dsmoe_set_gemm_kernel": (ctypes.c_int, [vp, i32]),
         "dsmoe_get_gemm_kernel": (i32, [vp]),
+        "dsmoe_set_selection": (ctypes.c_int, [vp, i32, i32]),
+        "dsmoe_get_selection": (ctypes.c_int, [vp, ctypes.POINTER(i32), ctypes.POINTER(i32)]),
         "dsmoe_stage_times": (ctypes.c_int, [vp, ctypes.POINTER(ctypes.c_float), i32, ctypes.POINTER(i32)]),
         "dsmoe_stage_name": (ctypes.c_char_p, [i32]),
         "dsmoe_launch_count": (ctypes.c_int, [vp, ctypes.POINTER(i64)]),
@@ -198,6 +201,16 @@ def dsmoe_get_gemm_kernel(handle) -> int:
     return int(_lib.dsmoe_get_gemm_kernel(handle))
 
 
+def dsmoe_set_selection(handle, mask_top: int, k_active: int) -> None:
+    _check(_lib.dsmoe_set_selection(handle, int(mask_top), int(k_active)), "dsmoe_set_selection")
+
+
+def dsmoe_get_selection(handle):
+    m, k = ctypes.c_int32(), ctypes.c_int32()
+    _check(_lib.dsmoe_get_selection(handle, ctypes.byref(m), ctypes.byref(k)), "dsmoe_get_selection")
+    return m.value, k.value
+
+
 def dsmoe_set_timing(handle, enable: bool) -> None:
     _check(_lib.dsmoe_set_timing(handle, int(bool(enable))), "dsmoe_set_timing")
 
@@ -297,6 +310,13 @@ class DSMoE:
         self.device = device
         self.w = weights
         self.handle = dsmoe_create(cfg, device)
+        self.mask_top, self.k_active = 0, cfg.top_k
+
+    def set_selection(self, mask_top: int = 0, k_active: Optional[int] = None):
+        """Selection variant for later forwards (see dsmoe_set_selection)."""
+        k = self.cfg.top_k if k_active is None else int(k_active)
+        dsmoe_set_selection(self.handle, mask_top, k)
+        self.mask_top, self.k_active = int(mask_top), k
 
     def close(self):
         if self.handle:
@@ -314,8 +334,8 @@ class DSMoE:
         dev = torch.device("cuda", self.device)
         c = self.cfg
         out = dict(h=torch.empty((T, c.d_model), dtype=torch.bfloat16, device=dev),
-                   topk_idx=torch.empty((T, c.top_k), dtype=torch.int32, device=dev),
-                   gates=torch.empty((T, c.top_k), dtype=torch.float32, device=dev),
+                   topk_idx=torch.empty((T, self.k_active), dtype=torch.int32, device=dev),
+                   gates=torch.empty((T, self.k_active), dtype=torch.float32, device=dev),
                    counts=torch.empty((c.n_routed,), dtype=torch.int32, device=dev),
                    f=torch.empty((c.n_routed,), dtype=torch.float32, device=dev),
                    P=torch.empty((c.n_routed,), dtype=torch.float32, device=dev),

@@ -170,7 +170,9 @@ struct dsmoe_handle {
   int device = 0;
   int num_sms = 148;
   int pair_clusters[2] = {0, 0};  // co-resident CTA pairs of the pair GEMM (down, gate/up)
-  int32_t gemm_kernel = DSMOE_GEMM_PAIR;
+  int32_t gemm_kernel = DSMOE_GEMM_SINGLE;
+  int32_t mask_top = 0;  // selection variant: top-ranked experts masked before the choice
+  int32_t k_active = 0;  // selection variant: experts kept per token (cfg.top_k by default)
   uint64_t wait_ns = kDefaultWaitNs;
   char* ws = nullptr;
   Layout L;
@@ -290,10 +292,10 @@ DSMOE_EXPORT dsmoe_status dsmoe_create(const dsmoe_cfg* cfg, int32_t device, dsm
   h->cfg = *cfg;
   if (h->cfg.score == DSMOE_ROUTE_HASH && h->cfg.hash_mod == 0) h->cfg.hash_mod = h->cfg.n_routed;
   h->device = device;
+  h->k_active = h->cfg.top_k;
   h->num_sms = prop.multiProcessorCount;
   h->pair_clusters[0] = dsmoe::grouped_gemm_pair_max_clusters(false);
   h->pair_clusters[1] = dsmoe::grouped_gemm_pair_max_clusters(true);
-  if (h->pair_clusters[0] < 1 || h->pair_clusters[1] < 1) h->gemm_kernel = DSMOE_GEMM_SINGLE;
   dsmoe::router_tc_shape(cfg->n_routed, &h->rt_chunks, &h->rt_nc, &h->rt_cols);
   h->L = plan(h->cfg);
   cudaError_t e = cudaMalloc(&h->ws, h->L.total);
@@ -435,7 +437,7 @@ int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
 dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
   const dsmoe_cfg& c = h->cfg;
-  const int T = a.T, N = c.n_routed, K = c.top_k, d = c.d_model, F = c.d_ff;
+  const int T = a.T, N = c.n_routed, K = h->k_active, d = c.d_model, F = c.d_ff;
   const int Ks = c.n_shared, Fs = c.d_ff_shared;
   const bool hash = c.score == DSMOE_ROUTE_HASH;
   const bool timing = h->timing && T > 0;
@@ -509,6 +511,7 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
     sa.T = T;
     sa.N = N;
     sa.K = K;
+    sa.mask_top = h->mask_top;
     sa.score = c.score;
     sa.bias_select = c.bias_mode == DSMOE_BIAS_SELECT_ONLY;
     sa.bias_in_logits = c.bias_mode == DSMOE_BIAS_IN_LOGITS;
@@ -677,7 +680,7 @@ DSMOE_EXPORT dsmoe_status dsmoe_forward_host(dsmoe_handle* h, int32_t T, const v
   DeviceGuard g(h->device);
   if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t xb = static_cast<size_t>(T) * c.d_model * 2, sb = static_cast<size_t>(T) * c.top_k * 4,
+  const size_t xb = static_cast<size_t>(T) * c.d_model * 2, sb = static_cast<size_t>(T) * h->k_active * 4,
                nb = static_cast<size_t>(c.n_routed) * 4;
   if (T > 0) {
     CUDA_TRY(cudaMemcpyAsync(h->x_stage, x_host, xb, cudaMemcpyHostToDevice, s));
@@ -708,7 +711,7 @@ DSMOE_EXPORT dsmoe_status dsmoe_balance_stats(dsmoe_handle* h, int64_t T_total, 
   if (!counts || !P_sum || !f || !P) return fail(DSMOE_ERR_INVALID_ARG, "counts, P_sum, f and P are required");
   DeviceGuard g(h->device);
   if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
-  CUDA_TRY(dsmoe::launch_balance_stats(counts, P_sum, T_total, h->cfg.n_routed, h->cfg.top_k, f, P,
+  CUDA_TRY(dsmoe::launch_balance_stats(counts, P_sum, T_total, h->cfg.n_routed, h->k_active, f, P,
                                        static_cast<cudaStream_t>(stream)));
   h->launches += 1;
   return DSMOE_OK;
@@ -745,6 +748,28 @@ DSMOE_EXPORT dsmoe_status dsmoe_set_gemm_kernel(dsmoe_handle* h, int32_t kind) {
 }
 
 DSMOE_EXPORT int32_t dsmoe_get_gemm_kernel(dsmoe_handle* h) { return h ? h->gemm_kernel : -1; }
+
+DSMOE_EXPORT dsmoe_status dsmoe_set_selection(dsmoe_handle* h, int32_t mask_top, int32_t k_active) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  const dsmoe_cfg& c = h->cfg;
+  if (k_active < 1 || k_active > c.top_k)
+    return fail(DSMOE_ERR_INVALID_ARG, "k_active = %d is outside [1, top_k = %d]", k_active, c.top_k);
+  if (mask_top < 0 || mask_top + k_active > c.n_routed)
+    return fail(DSMOE_ERR_INVALID_ARG, "mask_top = %d with k_active = %d exceeds n_routed = %d", mask_top, k_active,
+                c.n_routed);
+  if (c.score == DSMOE_ROUTE_HASH && (mask_top != 0 || k_active != c.top_k))
+    return fail(DSMOE_ERR_UNSUPPORTED, "hash routing has no ranking to mask or shorten");
+  h->mask_top = mask_top;
+  h->k_active = k_active;
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_get_selection(dsmoe_handle* h, int32_t* mask_top, int32_t* k_active) {
+  if (!h || !mask_top || !k_active) return fail(DSMOE_ERR_INVALID_ARG, "NULL argument");
+  *mask_top = h->mask_top;
+  *k_active = h->k_active;
+  return DSMOE_OK;
+}
 
 DSMOE_EXPORT dsmoe_status dsmoe_set_timing(dsmoe_handle* h, int32_t enable) {
   if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
@@ -798,7 +823,7 @@ DSMOE_EXPORT dsmoe_status dsmoe_workspace_tensor(dsmoe_handle* h, const char* na
   } table[] = {
       {"logits", h->logits, T, c.n_routed, !hash},
       {"offsets", h->offsets, 1, c.n_routed + 1, true},
-      {"slot_of", h->slot_of, T, c.top_k, true},
+      {"slot_of", h->slot_of, T, h->k_active, true},
       {"Xp", h->Xp, S, c.d_model, true},
       {"A1", h->A1, S, c.d_ff, true},
       {"A1s", h->A1s, T, static_cast<int64_t>(c.n_shared) * c.d_ff_shared, c.n_shared > 0},
@@ -843,7 +868,7 @@ DSMOE_EXPORT dsmoe_status dsmoe_sequence_balance(dsmoe_handle* h, int32_t T, int
   DeviceGuard g(h->device);
   if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
   const int S = T / seq_len;
-  CUDA_TRY(dsmoe::launch_sequence_balance(topk_idx, scores, S, seq_len, h->cfg.n_routed, h->cfg.top_k, beta, f_seq,
+  CUDA_TRY(dsmoe::launch_sequence_balance(topk_idx, scores, S, seq_len, h->cfg.n_routed, h->k_active, beta, f_seq,
                                           p_seq, h->seq_terms, loss, static_cast<cudaStream_t>(stream)));
   h->launches += S > 0 ? 2 : 1;
   return DSMOE_OK;
@@ -856,7 +881,7 @@ DSMOE_EXPORT dsmoe_status dsmoe_bias_update(dsmoe_handle* h, int64_t T, const in
   if (T < 0) return fail(DSMOE_ERR_INVALID_ARG, "T is negative");
   DeviceGuard g(h->device);
   if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
-  CUDA_TRY(dsmoe::launch_bias_update(counts, T, h->cfg.n_routed, h->cfg.top_k, alpha, b,
+  CUDA_TRY(dsmoe::launch_bias_update(counts, T, h->cfg.n_routed, h->k_active, alpha, b,
                                      static_cast<cudaStream_t>(stream)));
   h->launches += 1;
   return DSMOE_OK;

@@ -7,8 +7,11 @@
 // but each tile is computed by a cluster of two CTAs on neighbouring SMs with one M=256
 // MMA per K step (weights on M, tokens on N, N = the tile's token count rounded up to
 // 16, at most 256). Each SM stages only its own 128 weight rows and half of the token
-// rows, so per MAC it moves half the shared-memory operand bytes of a one-CTA M=128,
-// N=128 MMA (which the tensor core's shared-memory read port caps well below peak).
+// rows, so per MAC it reads half the shared-memory operand bytes of a one-CTA M=128,
+// N=128 MMA. Its outputs are bit-identical to the one-CTA kernel's. On B200 it halves
+// the tensor core's shared-memory read traffic but is not faster than the one-CTA
+// kernel, which therefore stays the default: both are bound by the latency of their
+// operand loads, not by that port.
 //
 // Tile of a pair (even CTA = rank 0, odd = rank 1):
 //   gate/up: 128 output features f0..f0+127; rank r holds the 64 gate rows and then
@@ -86,7 +89,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair_kernel(const __
   uint64_t* acc_full = bars + 2 * kStages;
   uint64_t* acc_empty = acc_full + kBufs;
   uint64_t* drain = acc_empty + kBufs;
-  uint64_t* xbar = drain + 1;  // [slot][pair]: both warps of a pair (64 threads) arrive
+  uint64_t* xbar = drain + 1;  // [slot][pair]: one lane of each warp of the pair arrives
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + kOffMisc + 4);
   volatile int* never_flag = reinterpret_cast<volatile int*>(base + kOffMisc + 8);
@@ -113,7 +116,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair_kernel(const __
       mbar_init(&acc_empty[i], 2 * 4);  // one lane of each epilogue warp of both CTAs
     }
     mbar_init(drain, 1);
-    for (int i = 0; i < 4; ++i) mbar_init(&xbar[i], 64);
+    for (int i = 0; i < 4; ++i) mbar_init(&xbar[i], 2);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -274,7 +277,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair_kernel(const __
 #pragma unroll
           for (int j = 0; j < 16; ++j)  // gate sends tokens 16-31, up sends tokens 0-15
             mine[j * 32 + lane] = __uint_as_float(is_gate ? v[16 + j] : v[j]);
-          mbar_arrive(&xbar[sl * 2 + p]);
+          __syncwarp();  // the warp's writes are ordered before its one arrival
+          if (lane == 0) mbar_arrive(&xbar[sl * 2 + p]);
           if (!mbar_wait_warp(&xbar[sl * 2 + p], (n_xchg >> 1) & 1u, a.wait_limit_ns, abort_flag)) {
             ok = false;
             break;

@@ -32,7 +32,8 @@ struct SelectArgs {
   const float* logits;   // [splits, T, N] partial sums
   int splits;
   const float* b;        // [N] or nullptr
-  int T, N, K;
+  int T, N, K;           // K: experts kept per token
+  int mask_top;          // experts ranked first that are masked before the K are kept
   int score;             // dsmoe_score
   int bias_select;       // selection-only bias
   int bias_in_logits;    // b is added to the summed logits before scoring

@@ -103,8 +103,10 @@ cudaError_t launch_router_logits(const bf16* x, const bf16* W_router, int T, int
 
 // --------------------------------------------------------------------------------------
 // scores + top-K' + gates + statistics partials: one warp per token, lane j owns experts
-// j, j+32, ... (kNPL per lane). Selection is K' rounds of a warp arg-max over the keys
-// not yet taken; ties go to the lower expert index.
+// j, j+32, ... (kNPL per lane). Selection is rounds of a warp arg-max over the keys not
+// yet taken; ties go to the lower expert index. The first mask_top rounds only mask
+// their winner (the DeepSeekMoE summary's "disable the top routed experts" analysis);
+// the next K' rounds select.
 // --------------------------------------------------------------------------------------
 namespace {
 constexpr int kSelWarps = 8;
@@ -187,7 +189,8 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(const SelectArgs
     uint32_t taken = 0;
     int my_idx = 0;
     float my_s = 0.f;
-    for (int r = 0; r < K; ++r) {
+    const int rounds = a.mask_top + K;
+    for (int r = 0; r < rounds; ++r) {
       float bk = -INFINITY;
       int bi = 0x7fffffff;
       float bs = 0.f;
@@ -213,7 +216,7 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(const SelectArgs
         }
       }
       if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      if (lane == r) {
+      if (lane == r - a.mask_top) {
         my_idx = bi;
         my_s = bs;
       }

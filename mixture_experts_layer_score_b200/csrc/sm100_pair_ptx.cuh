@@ -41,18 +41,21 @@ __device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t caddr) {
   return v;
 }
 
-// Arrive on an mbarrier that may live in the other CTA of the pair.
+// Arrive on an mbarrier that may live in the other CTA of the pair. Default (CTA-scope)
+// release: what it orders for the other CTA is tensor-memory reads, which the caller
+// completes (tcgen05.wait::ld) and fences (tcgen05.fence::before_thread_sync) first;
+// a cluster-scope release would also wait for this thread's earlier global stores.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
 }
 
-// try_wait with cluster-scope acquire: for barriers that the other CTA (its threads,
-// its copies or the pair's MMA commits) arrives on.
+// try_wait for barriers that the other CTA (its copies, its arrivals or the pair's MMA
+// commits) completes; default acquire semantics, as for the CTA's own barriers.
 __device__ __forceinline__ bool mbar_try_wait_cl(uint64_t* bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(done)
       : "r"(smem_addr(bar)), "r"(parity)
@@ -60,7 +63,7 @@ __device__ __forceinline__ bool mbar_try_wait_cl(uint64_t* bar, uint32_t parity)
   return done != 0;
 }
 
-// Bounded wait (see mbar_wait_bounded) with cluster-scope acquire.
+// Bounded wait (see mbar_wait_bounded) on such a barrier.
 __device__ __forceinline__ bool mbar_wait_bounded_cl(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
                                                      volatile int* abort_flag) {
   if (mbar_try_wait_cl(bar, parity)) return true;
@@ -74,7 +77,7 @@ __device__ __forceinline__ bool mbar_wait_bounded_cl(uint64_t* bar, uint32_t par
   }
 }
 
-// Whole-warp bounded wait with back-off (see mbar_wait_warp_sleepy), cluster scope.
+// Whole-warp bounded wait with back-off (see mbar_wait_warp_sleepy) on such a barrier.
 __device__ __forceinline__ bool mbar_wait_warp_sleepy_cl(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
                                                          volatile int* abort_flag) {
   uint32_t ok = 1;

@@ -129,13 +129,19 @@ def scores(logits, score: int) -> np.ndarray:
 
 
 def select_topk(s, top_k: int, b=None, bias_mode: int = BIAS_NONE, renormalize: bool = False,
-                decision_dtype=np.float64) -> Tuple[np.ndarray, np.ndarray]:
+                decision_dtype=np.float64, mask_top: int = 0) -> Tuple[np.ndarray, np.ndarray]:
     """Top-K' selection and gates ([DSMoE] gate equation; [V4-ch2] sections 2-3).
 
     Selection key: s~_i = s_i + b_i when the bias is selection-only
     ([V4-ch2] section 3; [MoE-learn]: the bias only decides who is selected),
     else s_i. Experts are ordered by key descending, ties to the lower index
     (reading: the pages do not say how ties break), and the first K' are kept.
+
+    mask_top = r > 0 is the [DSMoE] expert-specialisation analysis ("disable the top
+    routed experts"): per token the r experts ranked first are masked out and the top
+    K' of the remaining ones are kept (reading: "ranked first" uses the same key as
+    the selection). A K' below the trained one is the same analysis's "fewer
+    activated routed experts". Gates are taken over the kept experts.
 
     Gates use the raw score: g = s_i for the selected experts ([DSMoE] gate
     equation), or g = s_i / sum_{selected} s_j when renormalize is set
@@ -159,7 +165,7 @@ def select_topk(s, top_k: int, b=None, bias_mode: int = BIAS_NONE, renormalize: 
     ar = np.arange(N)
     for t in range(T):
         order[t] = np.lexsort((ar, -key[t]))  # primary: key descending; secondary: index ascending
-    idx = order[:, :top_k].astype(np.int32)
+    idx = order[:, mask_top:mask_top + top_k].astype(np.int32)
     g = np.take_along_axis(s, idx.astype(np.int64), axis=1)
     if renormalize:
         g = g / g.sum(axis=1, keepdims=True)
@@ -270,7 +276,8 @@ def route(cfg, inputs: Dict) -> Dict[str, np.ndarray]:
         return dict(idx=idx, gates=g, counts=counts, f=f, P=P, scores=None, logits=None)
     l = router_logits(inputs["x"], inputs["W_router"], inputs.get("b"), cfg.bias_mode)
     s = scores(l, cfg.score)
-    idx, g = select_topk(s, cfg.top_k, inputs.get("b"), cfg.bias_mode, cfg.renormalize)
+    idx, g = select_topk(s, cfg.top_k, inputs.get("b"), cfg.bias_mode, cfg.renormalize,
+                         mask_top=getattr(cfg, "mask_top", 0))
     counts, f, P = balance_stats(idx, s, cfg.n_routed, cfg.top_k)
     return dict(idx=idx, gates=g, counts=counts, f=f, P=P, scores=s, logits=l)
 

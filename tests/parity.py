@@ -3,8 +3,9 @@ smoke check and the benchmark's sampled parity check).
 
 Acceptance rules:
 * expert indices: bit-exact, in order, on every token whose sorted selection keys
-  are separated by more than GAP at every adjacent position up to K'+1; as a set on
-  tokens separated only at the K'-th/(K'+1)-th boundary; every other (near-tie)
+  are separated by more than GAP at every adjacent position that decides the output
+  (up to K'+1, or from the mask boundary r to r+K'+1 when the top r are masked); as a
+  set on tokens separated only at the boundaries; every other (near-tie)
   token is re-decided by the oracle from the kernel's own fp32 scores, in fp32,
   and must then match bit-exactly.
 * counts: bit-exact against the histogram of the reference selection, and equal to
@@ -52,16 +53,22 @@ def reference_selection(cfg, inp_cpu, gpu_topk, gpu_scores):
     s = r["scores"]
     b = None if inp_cpu.get("b") is None else _np(inp_cpu["b"]).astype(np.float64)
     keys = _sorted_keys(s, b, cfg.bias_mode)
-    upto = min(K + 1, cfg.n_routed)
-    gaps = keys[:, :upto - 1] - keys[:, 1:upto] if upto > 1 else np.full((T, 1), np.inf)
-    boundary = gaps[:, K - 1] if K < cfg.n_routed else np.full(T, np.inf)
+    N, m = cfg.n_routed, getattr(cfg, "mask_top", 0)
+    # adjacent key gaps that decide the output: the mask boundary (positions m-1, m), the
+    # order of the kept experts (m .. m+K-1) and the selection boundary (m+K-1, m+K)
+    lo, hi = max(m - 1, 0), min(m + K, N - 1)
+    gaps = keys[:, lo:hi] - keys[:, lo + 1:hi + 1] if hi > lo else np.full((T, 1), np.inf)
+    inf = np.full(T, np.inf)
+    mask_gap = keys[:, m - 1] - keys[:, m] if m > 0 else inf
+    sel_gap = keys[:, m + K - 1] - keys[:, m + K] if m + K < N else inf
     clean = (gaps > GAP).all(axis=1) if gaps.size else np.ones(T, bool)
-    set_only = (~clean) & (boundary > GAP)
+    set_only = (~clean) & (mask_gap > GAP) & (sel_gap > GAP)
     near = ~(clean | set_only)
     idx = r["idx"].copy()
     if near.any():
         gs = _np(gpu_scores)[near].astype(np.float64)
-        idx_n, _ = O.select_topk(gs, K, b, cfg.bias_mode, cfg.renormalize, decision_dtype=np.float32)
+        idx_n, _ = O.select_topk(gs, K, b, cfg.bias_mode, cfg.renormalize, decision_dtype=np.float32,
+                                 mask_top=m)
         idx[near] = idx_n
     if set_only.any():
         # the order inside the selected set is not fixed by a margin: take the kernel's order

@@ -22,19 +22,19 @@ if not torch.cuda.is_available():
 
 # T < 256 runs the CUDA-core router (split-K logits, then the select kernel); larger T
 # the tensor-core router; both are checked through the scores they report.
-# The grouped GEMMs run on the default CTA-pair kernel; the "-single" cases run the
-# one-CTA kernel.
+# The grouped GEMMs run on the default one-CTA kernel; the "-pair" cases run the CTA-pair
+# kernel.
 CASES = [("tiny", 300, 0), ("tiny", 200, 0), ("gshard_c", 700, 0), ("ds2b", 900, 0), ("v4_decode_t64", 64, 0),
          ("tiny", 300, 1), ("ds2b", 900, 1)]
 
 
-@pytest.mark.parametrize("name,T,kind", CASES,
-                         ids=[f"{c[0]}-T{c[1]}" + ("-single" if c[2] else "") for c in CASES])
-def test_stages(name, T, kind):
+@pytest.mark.parametrize("name,T,pair", CASES,
+                         ids=[f"{c[0]}-T{c[1]}" + ("-pair" if c[2] else "") for c in CASES])
+def test_stages(name, T, pair):
     cfg = W.get_config(name)
     gpu, cpu = make_case(cfg, T)
     layer = M.DSMoE(M.cfg_from(cfg, T), gpu)
-    M.dsmoe_set_gemm_kernel(layer.handle, M.DSMOE_GEMM_SINGLE if kind else M.DSMOE_GEMM_PAIR)
+    M.dsmoe_set_gemm_kernel(layer.handle, M.DSMOE_GEMM_PAIR if pair else M.DSMOE_GEMM_SINGLE)
     out = layer.forward(gpu["x"], with_scores=True)
     torch.cuda.synchronize()
     ws = {n: M.workspace_view(layer.handle, n).clone().cpu()

@@ -27,6 +27,22 @@ def _topk_ties_to_higher_index(s, top_k, b=None, bias_mode=0, renormalize=False,
     return (N - 1 - idx).astype(np.int32), g
 
 
+def _mask_ranked_by_raw_score(s, top_k, b=None, bias_mode=0, renormalize=False,
+                              decision_dtype=np.float64, mask_top=0):
+    """Masks the r experts with the highest raw score instead of the highest selection key."""
+    s = np.asarray(s, dtype=np.float64)
+    if mask_top == 0:
+        return _orig["select_topk"](s, top_k, b, bias_mode, renormalize, decision_dtype)
+    masked, _ = _orig["select_topk"](s, mask_top)
+    s2 = s.copy()
+    np.put_along_axis(s2, masked.astype(np.int64), -np.inf, axis=1)
+    idx, _ = _orig["select_topk"](s2, top_k, b, bias_mode, False, decision_dtype)
+    g = np.take_along_axis(s, idx.astype(np.int64), axis=1)
+    if renormalize:
+        g = g / g.sum(axis=1, keepdims=True)
+    return idx, g
+
+
 def _f_without_topk(idx, s, n_routed, top_k):
     c, f, p = _orig["balance_stats"](idx, s, n_routed, top_k)
     return c, f * top_k, p
@@ -59,6 +75,7 @@ def _softmax_over_wrong_axis(l):
 MUTATIONS = [
     ("silu", _silu_without_sigmoid, P.test_swiglu_matches_torch_library, ()),
     ("select_topk", _topk_ties_to_higher_index, P.test_topk_bruteforce, (9, 3)),
+    ("select_topk", _mask_ranked_by_raw_score, P.test_masked_topk_bruteforce, (8, 3, 2)),
     ("balance_stats", _f_without_topk, P.test_balance_worked_example, "golden"),
     ("sqrt_softplus", _softplus_without_sqrt, P.test_score_page_readings, "golden"),
     ("moe_layer", _layer_drops_shared, P.test_identical_experts_reduce_to_one_dense_ffn, ()),
@@ -68,7 +85,7 @@ MUTATIONS = [
 ]
 
 
-@pytest.mark.parametrize("name,mut,pin,args", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+@pytest.mark.parametrize("name,mut,pin,args", MUTATIONS, ids=[m[1].__name__.strip("_") for m in MUTATIONS])
 def test_pin_catches_mutation(monkeypatch, golden_dir, name, mut, pin, args):
     monkeypatch.setattr(O, name, mut)
     call_args = (golden_dir,) if args == "golden" else args

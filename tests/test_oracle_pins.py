@@ -156,6 +156,51 @@ def test_topk_bruteforce_with_selection_bias():
         np.testing.assert_array_equal(g[0], s[idx[0]])
 
 
+def _iterative_masked_pick(key, r, k):
+    """The "disable the top routed experts" analysis of the DeepSeekMoE summary written as
+    repeated arg-max: remove the best expert r times, then take the best k of the rest
+    one at a time (ties to the lower index at every step)."""
+    alive = list(range(len(key)))
+    def pop_best():
+        best = max(alive, key=lambda i: (key[i], -i))
+        alive.remove(best)
+        return best
+    for _ in range(r):
+        pop_best()
+    return [pop_best() for _ in range(k)]
+
+
+@pytest.mark.parametrize("N,K,r", [(8, 2, 1), (8, 3, 2), (12, 4, 3), (6, 1, 5), (9, 3, 0)])
+def test_masked_topk_bruteforce(N, K, r):
+    rng = np.random.default_rng(100 * N + 10 * K + r)
+    for trial in range(20):
+        s = rng.integers(0, 5, size=N) / 4.0
+        b = rng.integers(-2, 3, size=N) / 8.0
+        idx, g = O.select_topk(s[None, :], K, b, O.BIAS_SELECT_ONLY, mask_top=r)
+        assert idx[0].tolist() == _iterative_masked_pick((s + b).tolist(), r, K)
+        np.testing.assert_array_equal(g[0], s[idx[0]])  # gates stay raw scores
+
+
+def test_masked_and_reduced_k_compose_with_the_plain_selection():
+    """Masking the top r and keeping K' leaves exactly the plain top-(r+K') minus the plain
+    top-r; a smaller K' keeps a prefix of the K' order; renormalised gates sum to one
+    over the kept experts."""
+    rng = np.random.default_rng(11)
+    s = O.softmax(rng.normal(size=(50, 16)))
+    full, _ = O.select_topk(s, 7)
+    for r, k in [(1, 6), (2, 4), (3, 3), (0, 3)]:
+        idx, g = O.select_topk(s, k, mask_top=r, renormalize=True)
+        np.testing.assert_array_equal(idx, full[:, r:r + k])
+        np.testing.assert_allclose(g.sum(axis=1), 1.0, rtol=1e-12)
+    # the route of a config with mask_top equals select_topk on the same scores
+    cfg = W.get_config("tiny").replace(T=40, mask_top=2, top_k=3)
+    inp = W.make_inputs(cfg, seed=3, with_weights=False)
+    r = O.route(cfg, inp)
+    idx, _ = O.select_topk(r["scores"], 3, inp.get("b"), cfg.bias_mode, cfg.renormalize, mask_top=2)
+    np.testing.assert_array_equal(r["idx"], idx)
+    assert r["counts"].sum() == 40 * 3
+
+
 def test_gates_raw_and_renormalised():
     rng = np.random.default_rng(6)
     s = O.sigmoid(rng.normal(size=(11, 20)))

@@ -40,18 +40,19 @@ def test_small_parity(name, T, rows):
     _check(W.get_config(name), T, rows)
 
 
-SINGLE_CTA = [("tiny", 131), ("gshard_c", 1000), ("v3_prefill", 300), ("v4_decode_t16", 16)]
+PAIR = [("tiny", 131), ("gshard_c", 1000), ("v3_prefill", 300), ("v4_decode_t16", 16), ("ds2b", 2000)]
 
 
-@pytest.mark.parametrize("name,T", SINGLE_CTA, ids=[f"{n}-T{t}" for n, t in SINGLE_CTA])
-def test_small_parity_single_cta_gemm(name, T):
-    """The one-CTA grouped GEMM (the alternative to the default CTA-pair kernel)."""
-    _check(W.get_config(name), T, 48, gemm_kernel=M.DSMOE_GEMM_SINGLE)
+@pytest.mark.parametrize("name,T", PAIR, ids=[f"{n}-T{t}" for n, t in PAIR])
+def test_small_parity_pair_gemm(name, T):
+    """The CTA-pair grouped GEMM (the alternative to the default one-CTA kernel)."""
+    _check(W.get_config(name), T, 48, gemm_kernel=M.DSMOE_GEMM_PAIR)
 
 
 def test_gemm_kernels_agree():
     """The CTA-pair and one-CTA GEMM kernels on the same inputs: identical routing, and h
-    equal up to the accumulation order inside the tensor core."""
+    identical too (both accumulate each output over K in the same 16-element MMA steps
+    and share the epilogue arithmetic; measured bit-identical on B200)."""
     cfg = W.get_config("gshard_b").replace(T=1500)
     gpu, _ = make_case(cfg, cfg.T)
     a = run_cuda(cfg, gpu, cfg.T, gemm_kernel=M.DSMOE_GEMM_PAIR)
@@ -62,7 +63,7 @@ def test_gemm_kernels_agree():
     rms = b["h"].float().pow(2).mean().sqrt()
     print("pair vs single: bitwise equal rows", int((d.amax(1) == 0).sum()), "of", cfg.T,
           "max|diff|", float(d.max()), "rms", float(rms))
-    assert float(d.max()) <= PAR.H_TOL * float(rms)
+    assert float(d.max()) == 0.0
 
 
 FULL = [("gshard_a", 128), ("gshard_b", 128), ("gshard_c", 128), ("ds2b", 128), ("v3_prefill", 32),
@@ -206,9 +207,9 @@ def test_gemm_kernel_selector():
     cfg = W.get_config("tiny")
     gpu, _ = make_case(cfg, 8)
     layer = M.DSMoE(M.cfg_from(cfg, 8), gpu)
-    assert M.dsmoe_get_gemm_kernel(layer.handle) == M.DSMOE_GEMM_PAIR  # the default on B200
-    M.dsmoe_set_gemm_kernel(layer.handle, M.DSMOE_GEMM_SINGLE)
-    assert M.dsmoe_get_gemm_kernel(layer.handle) == M.DSMOE_GEMM_SINGLE
+    assert M.dsmoe_get_gemm_kernel(layer.handle) == M.DSMOE_GEMM_SINGLE  # the default
+    M.dsmoe_set_gemm_kernel(layer.handle, M.DSMOE_GEMM_PAIR)
+    assert M.dsmoe_get_gemm_kernel(layer.handle) == M.DSMOE_GEMM_PAIR
     with pytest.raises(M.DsmoeError) as ei:
         M.dsmoe_set_gemm_kernel(layer.handle, 7)
     assert ei.value.status == M.DSMOE_ERR_INVALID_ARG

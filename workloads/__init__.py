@@ -67,6 +67,7 @@ class MoEConfig:
     bias_kind: str = "none"          # "none" | "uniform0.1" | "zipf"
     router_std: Optional[float] = None  # None -> 1/sqrt(d)
     hash_mult: int = HASH_MULT
+    mask_top: int = 0      # experts masked before the top-K' choice (inference analysis variant)
 
     @property
     def slots(self) -> int:
