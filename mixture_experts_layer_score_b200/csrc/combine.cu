@@ -13,6 +13,9 @@ namespace dsmoe {
 namespace {
 constexpr int kCombineThreads = 128;
 
+// KMAX >= K bounds the unrolled gather: every 16-byte load of a chunk's K expert rows
+// is issued before the first FMA, so a thread keeps K loads in flight instead of one.
+template <int KMAX>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const bf16* __restrict__ x,
                                                                   const float* __restrict__ Hs,
                                                                   const bf16* __restrict__ Y,
@@ -33,6 +36,12 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const bf16* __
     }
     __syncthreads();
     for (int c = threadIdx.x; c < d8; c += kCombineThreads) {
+      uint4 yv[KMAX];
+#pragma unroll
+      for (int k = 0; k < KMAX; ++k) {
+        const int p = k < K ? s_slot[k] : -1;
+        yv[k] = p >= 0 ? y4[static_cast<int64_t>(p) * d8 + c] : make_uint4(0u, 0u, 0u, 0u);
+      }
       float acc[8];
       if (Hs) {
         const float4* hs4 = reinterpret_cast<const float4*>(Hs + static_cast<int64_t>(t) * d) + 2 * c;
@@ -49,12 +58,11 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const bf16* __
           acc[2 * j + 1] = f.y;
         }
       }
-      for (int k = 0; k < K; ++k) {
-        const int p = s_slot[k];
-        if (p < 0) continue;
+#pragma unroll
+      for (int k = 0; k < KMAX; ++k) {
+        if (k >= K || s_slot[k] < 0) continue;
         const float g = s_gate[k];
-        const uint4 v = y4[static_cast<int64_t>(p) * d8 + c];
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        const uint32_t w[4] = {yv[k].x, yv[k].y, yv[k].z, yv[k].w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const float2 f = unpack_bf16x2(w[j]);
@@ -78,7 +86,16 @@ cudaError_t launch_combine(const bf16* x, const float* Hs, const bf16* Y, const 
   int grid = T;
   if (grid > 16 * num_sms) grid = 16 * num_sms;
   if (grid < 1) grid = 1;
-  combine_kernel<<<grid, kCombineThreads, 0, s>>>(x, Hs, Y, slot_of, gates, T, K, d, h);
+  if (K <= 2)
+    combine_kernel<2><<<grid, kCombineThreads, 0, s>>>(x, Hs, Y, slot_of, gates, T, K, d, h);
+  else if (K <= 4)
+    combine_kernel<4><<<grid, kCombineThreads, 0, s>>>(x, Hs, Y, slot_of, gates, T, K, d, h);
+  else if (K <= 8)
+    combine_kernel<8><<<grid, kCombineThreads, 0, s>>>(x, Hs, Y, slot_of, gates, T, K, d, h);
+  else if (K <= 16)
+    combine_kernel<16><<<grid, kCombineThreads, 0, s>>>(x, Hs, Y, slot_of, gates, T, K, d, h);
+  else
+    return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 

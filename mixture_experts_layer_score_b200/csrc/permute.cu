@@ -86,11 +86,24 @@ __global__ void __launch_bounds__(256) permute_gather_kernel(const bf16* __restr
 #pragma unroll
     for (int k = 0; k < 16; ++k) pk[k] = __shfl_sync(0xffffffffu, pos, k);
     const uint4* src = x4 + static_cast<int64_t>(t) * d8;
-    for (int c = lane; c < d8; c += 32) {
-      const uint4 v = src[c];
+    // four 16-byte chunks per lane per step: their loads are all in flight before the
+    // first store
+    for (int c0 = lane; c0 < d8; c0 += 4 * 32) {
+      uint4 v[4];
 #pragma unroll
-      for (int k = 0; k < 16; ++k)
-        if (k < K && pk[k] >= 0) xp4[static_cast<int64_t>(pk[k]) * d8 + c] = v;
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + 32 * u;
+        if (c < d8) v[u] = src[c];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + 32 * u;
+        if (c < d8) {
+#pragma unroll
+          for (int k = 0; k < 16; ++k)
+            if (k < K && pk[k] >= 0) xp4[static_cast<int64_t>(pk[k]) * d8 + c] = v[u];
+        }
+      }
     }
   }
 }
