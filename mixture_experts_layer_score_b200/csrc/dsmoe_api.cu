@@ -10,7 +10,6 @@
 #include <cudaTypedefs.h>
 #include <stdarg.h>
 #include <stdio.h>
-#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -174,7 +173,6 @@ struct dsmoe_handle {
   int32_t gemm_kernel = DSMOE_GEMM_SINGLE;
   int32_t mask_top = 0;  // selection variant: top-ranked experts masked before the choice
   int32_t k_active = 0;  // selection variant: experts kept per token (cfg.top_k by default)
-  int32_t l2_prefetch_ahead = 0;  // one-CTA GEMM: K blocks of weight L2 prefetch ahead of the loads
   uint64_t wait_ns = kDefaultWaitNs;
   char* ws = nullptr;
   Layout L;
@@ -295,8 +293,6 @@ DSMOE_EXPORT dsmoe_status dsmoe_create(const dsmoe_cfg* cfg, int32_t device, dsm
   if (h->cfg.score == DSMOE_ROUTE_HASH && h->cfg.hash_mod == 0) h->cfg.hash_mod = h->cfg.n_routed;
   h->device = device;
   h->k_active = h->cfg.top_k;
-  // DSMOE_L2_PREFETCH_AHEAD: the one-CTA GEMM's weight-prefetch distance in K blocks
-  if (const char* env = getenv("DSMOE_L2_PREFETCH_AHEAD")) h->l2_prefetch_ahead = atoi(env);
   h->num_sms = prop.multiProcessorCount;
   h->pair_clusters[0] = dsmoe::grouped_gemm_pair_max_clusters(false);
   h->pair_clusters[1] = dsmoe::grouped_gemm_pair_max_clusters(true);
@@ -577,15 +573,6 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
     g.kb_per_b_expert_shared = d / 64;
     g.n_valid_routed = F;
     g.n_valid_shared = Fs;
-    g.w_ptr[0] = static_cast<const bf16*>(a.W_gate);
-    g.w_ptr[1] = static_cast<const bf16*>(a.W_up);
-    g.w_ptr[2] = static_cast<const bf16*>(Ks ? a.Ws_gate : a.W_gate);
-    g.w_ptr[3] = static_cast<const bf16*>(Ks ? a.Ws_up : a.W_up);
-    g.w_rows_routed = F;
-    g.w_rows_shared = Fs;
-    g.w_k_routed = d;
-    g.w_k_shared = d;
-    g.l2_prefetch_ahead = h->l2_prefetch_ahead;
     g.out_routed = h->A1;
     g.ld_routed = F;
     g.out_shared = h->A1s;
@@ -627,13 +614,6 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
     g.kb_per_b_expert_shared = Ks ? Fs / 64 : 1;
     g.n_valid_routed = d;
     g.n_valid_shared = d;
-    g.w_ptr[0] = g.w_ptr[1] = static_cast<const bf16*>(a.W_down);
-    g.w_ptr[2] = g.w_ptr[3] = static_cast<const bf16*>(Ks ? a.Ws_down : a.W_down);
-    g.w_rows_routed = d;
-    g.w_rows_shared = d;
-    g.w_k_routed = F;
-    g.w_k_shared = Fs;
-    g.l2_prefetch_ahead = h->l2_prefetch_ahead;
     g.out_routed = h->Y;
     g.ld_routed = d;
     g.out_shared = nullptr;

@@ -44,7 +44,7 @@ namespace {
 constexpr int kBK = 64;         // K per ring stage (one 128-byte swizzled row of bf16)
 constexpr int kFeat = 128;      // output features per MMA chain (the MMA's M, TMEM lanes)
 constexpr int kMmaK = 16;       // K of each bf16 tcgen05.mma
-constexpr int kThreads = 224;  // 6 warps of roles + the L2-prefetch warp
+constexpr int kThreads = 192;
 constexpr int kEpiThreads = 128;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kWBytes = 2 * kFeat * kBK * 2;  // 32 KB: two 128-row weight halves
@@ -93,7 +93,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + G_::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + G_::kOffMisc + 4);
   volatile int* never_flag = reinterpret_cast<volatile int*>(base + G_::kOffMisc + 8);
-  volatile uint32_t* loads_issued = reinterpret_cast<volatile uint32_t*>(base + G_::kOffMisc + 12);
   int32_t* tile_start = reinterpret_cast<int32_t*>(base + G_::kOffTiles);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -103,7 +102,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     *never_flag = 0;
-    *loads_issued = 0;
     for (int s = 0; s < G_::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -160,7 +158,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
             tma_load_3d(w, tw0, &full[stage], bk, t.n_blk * 2 * kFeat, be);
           }
           tma_load_2d(sX + stage * G_::kXBytes, tx, &full[stage], kb * kBK, t.row0);
-          *loads_issued = *loads_issued + 1;
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == G_::kStages) {
@@ -220,57 +217,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       if (!ok) {
         *abort_flag = 1;
         atomicOr(a.status, kStatusTimeoutMma);
-      }
-    }
-  } else if (warp == 6) {
-    // ------------------------------------------------------------ L2 prefetch of weights
-    // Walks the producer's (tile, K block) sequence and touches every weight line of a K
-    // block (128 B of each weight row the TMA will load) l2_prefetch_ahead blocks before
-    // the producer loads it, so those loads find the weights in L2 instead of DRAM. It
-    // paces itself on the producer's count of issued blocks (bounded wait) and only
-    // prefetches addresses inside the weight tensors.
-    const int ahead = a.l2_prefetch_ahead;
-    if (ahead > 0) {
-      uint32_t n = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-        const Tile t = decode_tile<G_::kTok>(a, tile_start, G, tile);
-        const int kb_per = t.shared ? a.kb_per_b_expert_shared : t.kb_n;
-        const bf16* w0 = a.w_ptr[t.shared ? 2 : 0];
-        const bf16* w1 = a.w_ptr[t.shared ? 3 : 1];
-        const int rows = t.shared ? a.w_rows_shared : a.w_rows_routed;
-        const int64_t klen = t.shared ? a.w_k_shared : a.w_k_routed;
-        const int r0 = kSwiGLU ? t.n_blk * kFeat : t.n_blk * 2 * kFeat;
-        constexpr int kRows = kSwiGLU ? kFeat : 2 * kFeat;
-        for (int kb = 0; kb < t.kb_n; ++kb, ++n) {
-          if (*loads_issued + ahead < n) {  // too far ahead: wait for the producer
-            uint32_t go = 1;
-            if (lane == 0) {
-              const uint64_t t0 = global_timer_ns();
-              while (*loads_issued + ahead < n) {
-                __nanosleep(128);
-                if (*abort_flag || global_timer_ns() - t0 > a.wait_limit_ns) {
-                  go = 0;
-                  break;
-                }
-              }
-            }
-            if (!__shfl_sync(0xffffffffu, go, 0)) {
-              ok = false;  // a hint only: stop prefetching, no status bit
-              break;
-            }
-          }
-          const int be = t.expert + kb / kb_per;
-          const int64_t col = static_cast<int64_t>(kb % kb_per) * kBK;
-          for (int r = lane; r < kRows; r += 32) {
-            const int row = r0 + r;
-            if (row < rows) {
-              const int64_t off = (static_cast<int64_t>(be) * rows + row) * klen + col;
-              prefetch_l2(w0 + off);
-              if (kSwiGLU) prefetch_l2(w1 + off);
-            }
-          }
-        }
       }
     }
   } else {

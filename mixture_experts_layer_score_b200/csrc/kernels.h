@@ -144,12 +144,6 @@ struct GemmArgs {
   int32_t shared_col_stride;      // shared group g writes at column g * shared_col_stride
   uint32_t* status;
   uint64_t wait_limit_ns;
-  // one-CTA kernel only: an extra warp prefetches the weight rows of the K blocks
-  // l2_prefetch_ahead blocks ahead of the TMA loads into L2 (0 turns it off)
-  const bf16* w_ptr[4];                   // raw b0/b1 routed, b0/b1 shared weights
-  int32_t w_rows_routed, w_rows_shared;   // weight rows per expert
-  int32_t w_k_routed, w_k_shared;         // weight row length (the contraction) in elements
-  int32_t l2_prefetch_ahead;
 };
 cudaError_t launch_grouped_gemm(bool swiglu, const GemmArgs& a, int grid, cudaStream_t s);
 

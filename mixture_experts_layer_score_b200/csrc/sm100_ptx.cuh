@@ -132,11 +132,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-// Hint: bring the 128-byte line holding `p` (a valid global address) into L2.
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-
 // ------------------------------------------------------------------------------------
 // tcgen05: tensor memory and the 5th-generation tensor core
 // ------------------------------------------------------------------------------------
