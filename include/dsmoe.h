@@ -127,7 +127,8 @@ void dsmoe_destroy(dsmoe_handle* h);
  *   Ws_up      bf16 [K_s, F_s, d]
  *   Ws_down    bf16 [K_s, d, F_s]
  *
- * Outputs (device, caller-owned, fully overwritten):
+ * Outputs (device, caller-owned, fully overwritten; K' here is the handle's k_active,
+ * cfg.top_k unless dsmoe_set_selection changed it):
  *
  *   h          bf16 [T, d]        layer output, accumulated in fp32, rounded once
  *   topk_idx   int32 [T, K']      selected experts, by descending selection key,
