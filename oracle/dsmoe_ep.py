@@ -1,0 +1,98 @@
+"""Reference oracle for the expert-parallel form of the DeepSeekMoE layer forward.
+
+TEST INFRASTRUCTURE ONLY, like dsmoe_oracle.py (float64, CPU; used only by the
+tests). It restates the layer for R ranks that each hold a shard of the tokens, a
+replica of the router and of the shared experts, and N'/R of the routed experts
+(the "DeepSeek-MoE interview card", section 4: shared experts replicated, routed
+experts sharded across devices; the DeepSeekMoE summary's device-level balance
+section groups experts by device the same way). Experts are assigned to ranks in
+contiguous blocks: expert e lives on rank e // (N'/R).
+
+One rank's forward, written as the steps a distributed implementation takes:
+  1. route its own tokens (dsmoe_oracle.route on the local shard);
+  2. order its (token, k) pairs by expert, ties by token then k: the
+     expert-contiguous slot order, which is also destination-rank order;
+  3. exchange the per-destination row counts, then the token rows and their
+     expert ids (all-to-all);
+  4. apply each received row's expert FFN (the owner holds those weights);
+  5. send the outputs back along the reverse exchange;
+  6. combine: h_t = u_t + sum_shared FFN(u_t) + sum_k g_{t,k} y_{t,k}.
+The result equals the single-device layer on the concatenated batch, which is
+what tests/test_oracle_ep.py checks on gloo ranks.
+
+`comm` supplies the exchange: alltoall(list of R numpy arrays) -> list of R arrays
+(element j of the input goes to rank j; element j of the output came from rank j).
+"""
+from __future__ import annotations
+
+from typing import Callable, Dict, List
+
+import numpy as np
+
+from oracle import dsmoe_oracle as O
+
+
+def expert_owner(e, n_routed: int, world: int):
+    """Rank that holds routed expert e (contiguous blocks of N'/R experts)."""
+    return np.asarray(e) // (n_routed // world)
+
+
+def ep_forward_rank(cfg, local_inputs: Dict, local_experts: Dict[int, tuple], shared: List[tuple],
+                    world: int, alltoall: Callable[[List[np.ndarray]], List[np.ndarray]]) -> Dict:
+    """The layer on this rank's tokens (local_inputs: x, W_router, b, token_ids as for
+    dsmoe_oracle.route). local_experts maps each routed expert this rank owns to its
+    (W_gate, W_up, W_down); shared lists the replicated shared experts.
+
+    Returns h (float64, one row per local token) and the local routing."""
+    assert cfg.n_routed % world == 0, "experts must split evenly across ranks"
+    X = O._as_f64(local_inputs["x"])
+    T, d = X.shape
+    r = O.route(cfg, local_inputs)
+    idx = np.asarray(r["idx"], dtype=np.int64)
+    K = idx.shape[1]
+
+    # 2. slot order: by expert, then token, then k
+    pairs = sorted(((int(idx[t, k]), t, k) for t in range(T) for k in range(K)))
+    dest = [int(expert_owner(e, cfg.n_routed, world)) for e, _, _ in pairs]
+
+    # 3. rows and expert ids per destination, in slot order
+    send_rows = [np.zeros((0, d)) for _ in range(world)]
+    send_eids = [np.zeros((0,), dtype=np.int64) for _ in range(world)]
+    for j in range(world):
+        sel = [i for i, dj in enumerate(dest) if dj == j]
+        send_rows[j] = X[[pairs[i][1] for i in sel]] if sel else np.zeros((0, d))
+        send_eids[j] = np.asarray([pairs[i][0] for i in sel], dtype=np.int64)
+    recv_rows = alltoall(send_rows)
+    recv_eids = alltoall([e.astype(np.float64) for e in send_eids])
+
+    # 4. the owner applies its experts, row by row grouped by expert
+    outs = []
+    for rows, eids in zip(recv_rows, recv_eids):
+        eids = eids.astype(np.int64)
+        y = np.zeros_like(rows)
+        for e in np.unique(eids):
+            m = eids == e
+            Wg, Wu, Wd = local_experts[int(e)]
+            y[m] = O.swiglu_ffn(rows[m], Wg, Wu, Wd)
+        outs.append(y)
+
+    # 5. back to the sources, in the order they were sent
+    back = alltoall(outs)
+
+    # 6. combine
+    h = X.copy()
+    for (Wg, Wu, Wd) in shared:
+        h += O.swiglu_ffn(X, Wg, Wu, Wd)
+    g = np.asarray(r["gates"], dtype=np.float64)
+    cursor = [0] * world
+    for (e, t, k), j in zip(pairs, dest):
+        h[t] += g[t, k] * back[j][cursor[j]]
+        cursor[j] += 1
+    return dict(h=h, idx=idx, gates=g, counts=r["counts"], scores=r["scores"])
+
+
+def device_loads(counts, n_routed: int, world: int) -> np.ndarray:
+    """Rows each rank's experts receive: the per-device sums of the expert counts (the
+    quantity the DeepSeekMoE summary's device-level balance loss evens out)."""
+    c = np.asarray(counts, dtype=np.int64)
+    return c.reshape(world, n_routed // world).sum(axis=1)
