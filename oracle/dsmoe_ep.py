@@ -18,7 +18,9 @@ One rank's forward, written as the steps a distributed implementation takes:
   5. send the outputs back along the reverse exchange;
   6. combine: h_t = u_t + sum_shared FFN(u_t) + sum_k g_{t,k} y_{t,k}.
 The result equals the single-device layer on the concatenated batch, which is
-what tests/test_oracle_ep.py checks on gloo ranks.
+what tests/test_oracle_ep.py checks on gloo ranks. ep_gather_forward_rank is the
+second form (gather every token, apply the local experts, sum the partial outputs),
+suited to decode batches.
 
 `comm` supplies the exchange: alltoall(list of R numpy arrays) -> list of R arrays
 (element j of the input goes to rank j; element j of the output came from rank j).
@@ -96,3 +98,44 @@ def device_loads(counts, n_routed: int, world: int) -> np.ndarray:
     quantity the DeepSeekMoE summary's device-level balance loss evens out)."""
     c = np.asarray(counts, dtype=np.int64)
     return c.reshape(world, n_routed // world).sum(axis=1)
+
+
+def ep_gather_forward_rank(cfg, local_inputs: Dict, local_experts: Dict[int, tuple], shared: List[tuple],
+                           world: int, rank: int, allgather_rows: Callable[[np.ndarray], List[np.ndarray]],
+                           allreduce_sum: Callable[[np.ndarray], np.ndarray]) -> Dict:
+    """The decode-shaped expert-parallel form: every rank gathers all ranks' tokens, routes
+    them (router replicated, so every rank makes the same choice), applies only the
+    routed experts it owns to the rows that chose them, and the partial outputs are summed
+    across ranks; each rank keeps its own tokens' rows and adds the residual and the
+    (replicated) shared experts. Few tokens, many experts: each weight is read on one rank
+    only, instead of once per token shard.
+
+    allgather_rows(a) returns every rank's array (rank order); allreduce_sum(a) sums an
+    array over ranks. local_inputs as for ep_forward_rank (token_ids included for hash
+    routing)."""
+    assert cfg.n_routed % world == 0, "experts must split evenly across ranks"
+    X_local = O._as_f64(local_inputs["x"])
+    parts = allgather_rows(X_local)
+    X = np.concatenate(parts, axis=0)
+    start = sum(p.shape[0] for p in parts[:rank])
+    full = dict(local_inputs)
+    full["x"] = X
+    if local_inputs.get("token_ids") is not None:
+        ids = allgather_rows(np.asarray(local_inputs["token_ids"], dtype=np.float64).reshape(-1, 1))
+        full["token_ids"] = np.concatenate(ids, axis=0).reshape(-1).astype(np.int64)
+    r = O.route(cfg, full)
+    idx = np.asarray(r["idx"], dtype=np.int64)
+    g = np.asarray(r["gates"], dtype=np.float64)
+    partial = np.zeros_like(X)
+    for e in np.unique(idx):
+        if int(expert_owner(e, cfg.n_routed, world)) != rank:
+            continue
+        rows, ks = np.nonzero(idx == e)
+        Wg, Wu, Wd = local_experts[int(e)]
+        partial[rows] += g[rows, ks][:, None] * O.swiglu_ffn(X[rows], Wg, Wu, Wd)
+    total = allreduce_sum(partial)
+    n = X_local.shape[0]
+    h = X_local + total[start:start + n]
+    for (Wg, Wu, Wd) in shared:
+        h += O.swiglu_ffn(X_local, Wg, Wu, Wd)
+    return dict(h=h, idx=idx[start:start + n], gates=g[start:start + n])

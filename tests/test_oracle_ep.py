@@ -1,7 +1,8 @@
 """The expert-parallel oracle (oracle/dsmoe_ep.py) on gloo ranks on the CPU: with the
 routed experts split across 2 or 4 ranks and the tokens split unevenly, every rank's
-layer output equals the single-device oracle's rows for its tokens, and the per-device
-loads add up to the whole batch's slots."""
+layer output equals the single-device oracle's rows for its tokens in both forms (the
+all-to-all dispatch and the gather / all-reduce form), and the per-device loads add up to
+the whole batch's slots."""
 import os
 import socket
 
@@ -39,6 +40,26 @@ def _alltoall(parts):
     return out
 
 
+def _allgather_rows(a):
+    """Every rank's float64 array [n_r, ...] (uneven n_r), in rank order, over gloo."""
+    world = dist.get_world_size()
+    n = torch.tensor([a.shape[0]], dtype=torch.int64)
+    ns = [torch.empty_like(n) for _ in range(world)]
+    dist.all_gather(ns, n)
+    m = int(max(int(v) for v in ns))
+    buf = torch.zeros((m,) + a.shape[1:], dtype=torch.float64)
+    buf[:a.shape[0]] = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64))
+    outs = [torch.empty_like(buf) for _ in range(world)]
+    dist.all_gather(outs, buf)
+    return [o[:int(k)].numpy() for o, k in zip(outs, ns)]
+
+
+def _allreduce_sum(a):
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64))
+    dist.all_reduce(t)
+    return t.numpy()
+
+
 def _cfg(name):
     import workloads as W
     cfg = W.get_config(name).replace(T=157)
@@ -72,7 +93,8 @@ def _worker(rank, world, port, name, result_q):
         out = EP.ep_forward_rank(cfg, local, mine, shared, world, _alltoall)
         loads = torch.as_tensor(EP.device_loads(out["counts"], cfg.n_routed, world))
         dist.all_reduce(loads)
-        result_q.put((rank, a, b, out["h"], loads.numpy()))
+        gath = EP.ep_gather_forward_rank(cfg, local, mine, shared, world, rank, _allgather_rows, _allreduce_sum)
+        result_q.put((rank, a, b, out["h"], loads.numpy(), gath["h"]))
     finally:
         dist.destroy_process_group()
 
@@ -94,6 +116,7 @@ def test_expert_parallel_oracle_equals_single_device(name, world):
         assert p.exitcode == 0
     inp = W.make_inputs(cfg, seed=2)
     ref = O.forward(cfg, inp)
-    for rank, a, b, h, loads in res:
+    for rank, a, b, h, loads, h_gather in res:
         np.testing.assert_allclose(h, ref["h"][a:b], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(h_gather, ref["h"][a:b], rtol=1e-12, atol=1e-12)
         assert loads.sum() == cfg.T * cfg.top_k
