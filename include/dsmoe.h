@@ -27,7 +27,9 @@
  *   - Errors are returned, never raised: no exit, abort or trap. A kernel that
  *     gives up a bounded wait records DSMOE_ERR_DEVICE_TIMEOUT in a device
  *     status word that dsmoe_get_status() reports.
- *   - A handle may be used by one host thread at a time.
+ *   - A handle may be used by one host thread at a time. Its forwards share one
+ *     workspace: enqueue them on one stream (or order the streams); two forwards of
+ *     the same handle that overlap on the GPU race. Separate handles are independent.
  */
 #ifndef DSMOE_H
 #define DSMOE_H
