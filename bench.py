@@ -15,10 +15,15 @@ events on the launching stream, max over ranks. The 22.6 GB of expert weights a
 step streams are far larger than L2, so no flush is needed between steps.
 
 Reported alongside: the dominant kernel's roofline (mean in-region duration from
-per-stage CUDA events), the same metric end to end through dsmoe_forward_host with
-pinned host buffers (copies inside the timed region), the oracle timed on the
-host's cores over a bounded sample, SM clocks sampled during the timed region, and
-the number of kernel launches.
+per-stage CUDA events; a tensor-bound kernel is divided by the measured burst bf16
+figure when the timed region ran at the maximum SM clock, else by the sustained one,
+and the other fractions are kept as extra keys), the same metric end to end through
+dsmoe_forward_host with pinned host buffers (copies inside the timed region), the
+oracle timed on the host's cores over a bounded sample, SM clocks sampled during the
+timed region, and the number of kernel launches. At N=1 a "decode" block follows:
+the V4-shaped decode batches (T=256 and T=16), timed the same way after the main
+workload's tensors are released, with the HBM bytes they must move per step and their
+fraction of the measured copy bandwidth.
 """
 from __future__ import annotations
 
@@ -52,7 +57,27 @@ def parse_args():
     ap.add_argument("--cpu-sample", type=int, default=None, help="tokens in the oracle's timed sample")
     ap.add_argument("--gemm", default="single", choices=["single", "pair"],
                     help="grouped-GEMM kernel: one CTA per tile (default) or CTA pairs")
+    ap.add_argument("--decode", default="v4_decode_t256,v4_decode_t16",
+                    help="decode workloads timed after the main one at N=1 (comma list; empty: none)")
+    ap.add_argument("--decode-steps", type=int, default=20)
     return ap.parse_args()
+
+
+SPEC_BF16_TFLOPS = 2250.0  # B200 dense bf16, nominal
+SPEC_HBM_GBS = 8000.0      # B200 HBM3e, nominal
+PEAK_CHOICE = ("tensor frac is against the burst cuBLAS figure when the timed region ran at the "
+               "maximum SM clock (median within 3% of clocks.max.sm), else against the sustained one")
+
+
+def tensor_peak_key(clock_info):
+    """The measured bf16 peak to divide by: the burst figure (a GEMM timed alone, at full
+    clock) when the timed region's median SM clock was at the maximum, else the
+    sustained, power-capped one."""
+    if clock_info and clock_info.get("sm_mhz") and clock_info.get("sm_max_mhz"):
+        if clock_info["sm_mhz"] >= 0.97 * clock_info["sm_max_mhz"]:
+            return "bf16_tflops"
+        return "bf16_tflops_sustained"
+    return "bf16_tflops"
 
 
 def load_peaks():
@@ -341,18 +366,24 @@ def run_native(args, cfg):
                     "gemm_down": 2 * cfg.d_model * (touched * cfg.d_ff + cfg.n_shared * cfg.d_ff_shared)}
     dom_ms = stage_ms[dom]
     intensity = flops[dom] / max(weight_bytes[dom], 1)
-    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    tensor_key = tensor_peak_key(clock_info)
+    ridge = peaks[tensor_key] * 1e12 / (peaks["hbm_gbs"] * 1e9)
     if intensity >= ridge:
         achieved = flops[dom] / (dom_ms / 1e3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak}
+        peak = peaks[tensor_key]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "frac_of_burst": achieved / peaks["bf16_tflops"],
+                "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+                "frac_of_spec": achieved / SPEC_BF16_TFLOPS}
     else:
         achieved = weight_bytes[dom] / (dom_ms / 1e3) / 1e9
         peak = peaks["hbm_gbs"]
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak}
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "frac_of_spec": achieved / SPEC_HBM_GBS}
     traffic = captured_traffic(dom, weight_bytes[dom], args.gemm)
     roof.update({"kernel": dom, "kernel_ms": dom_ms, "traffic": traffic,
-                 "peak_source": f"{peak_src} ({'bf16_tflops_sustained' if roof['bound'] == 'tensor' else 'hbm_gbs'})",
+                 "peak_source": f"{peak_src} ({tensor_key if roof['bound'] == 'tensor' else 'hbm_gbs'})",
+                 "peak_choice": PEAK_CHOICE,
                  "algorithmic": {"flops": flops[dom], "weight_bytes": weight_bytes[dom]}})
     layer_flops = cfg.flops_per_token() * cfg.T
     layer_tflops = layer_flops / (ms_per_step / 1e3) / 1e12
@@ -412,19 +443,81 @@ def run_native(args, cfg):
         cpu_base = {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                     "sample": f"{m} tokens of the workload as one batch, full layer, float64 oracle, {dt:.1f} s"}
 
+    layer.close()
+    # ---- decode (weight-streaming) workloads, N=1 only: the main workload's tensors are
+    # released first; each is timed on its own with the same event and clock method
+    decode = None
+    if world == 1 and args.decode.strip():
+        del inp, w, layer, out, xh, hh, th, gh, ch, fh, ph
+        torch.cuda.empty_cache()
+        decode = {}
+        for name in [n.strip() for n in args.decode.split(",") if n.strip()]:
+            decode[name] = time_decode(M, W, name, dev, stream, args.decode_steps, max(args.warmup, 3), peaks,
+                                       peak_src)
+
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; random weights of the layer's shape)",
-                "config": dict(config_block(cfg, world), gemm_kernel=args.gemm), "roofline": roof, "cpu_baseline": cpu_base, "e2e": e2e,
-                "gpu_launches": int(launches), "clocks": clock_info,
-                "layer_tflops": layer_tflops, "stage_ms": stage_ms, "experts_touched": touched}
+                "config": dict(config_block(cfg, world), gemm_kernel=args.gemm), "roofline": roof,
+                "cpu_baseline": cpu_base, "e2e": e2e, "gpu_launches": int(launches), "clocks": clock_info,
+                "layer_tflops": layer_tflops, "stage_ms": stage_ms, "experts_touched": touched, "decode": decode}
         print(json.dumps(line), flush=True)
-    layer.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def time_decode(M, W, name, dev, stream, steps, warmup, peaks, peak_src):
+    """One decode-shaped workload (few tokens, hundreds of experts): the layer streams the
+    weights of every expert some token picked, so it is HBM-bound. Returns its step time,
+    tokens/s and the bytes that must cross HBM per step (weights of the touched routed
+    experts and the shared experts, the router matrix, x read and h written) as GB/s and
+    as fractions of the measured copy bandwidth and of the 8 TB/s nominal figure, plus
+    the same for the gate/up GEMM alone (its weights over its event time)."""
+    import torch
+    cfg = W.get_config(name)
+    inp = W.make_inputs(cfg, seed=0, device=dev, with_weights=True)
+    layer = M.DSMoE(M.cfg_from(cfg, cfg.T), inp, device=dev.index)
+    out = layer.alloc_outputs(cfg.T)
+    for _ in range(warmup):
+        layer.forward(inp["x"], token_ids=inp["token_ids"], out=out, stream=stream)
+    torch.cuda.synchronize(dev)
+    M.dsmoe_set_timing(layer.handle, True)
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        layer.forward(inp["x"], token_ids=inp["token_ids"], out=out, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    clock_info = clocks.stop()
+    stage_ms = M.dsmoe_stage_times(layer.handle)
+    st = M.dsmoe_get_status(layer.handle)
+    if st != M.DSMOE_OK:
+        raise SystemExit(f"device status after the {name} timed region: {M.dsmoe_last_error()}")
+    touched = int((out["counts"] > 0).sum())
+    layer.close()
+    d, F, Fs, Ks = cfg.d_model, cfg.d_ff, cfg.d_ff_shared, cfg.n_shared
+    w_gate_up = 2 * d * 2 * (touched * F + Ks * Fs)
+    w_down = 2 * d * (touched * F + Ks * Fs)
+    router = 0 if cfg.score == W.ROUTE_HASH else cfg.n_routed * d * 2
+    step_bytes = w_gate_up + w_down + router + 2 * cfg.T * d * 2
+    gbs = step_bytes / (ms / 1e3) / 1e9
+    gu_gbs = w_gate_up / (stage_ms["gemm_gate_up"] / 1e3) / 1e9
+    del inp, out
+    torch.cuda.empty_cache()
+    return {"T": cfg.T, "ms_per_step": ms, "tokens_per_s": cfg.T / (ms / 1e3), "experts_touched": touched,
+            "bytes_per_step": step_bytes, "achieved_gbs": gbs, "frac": gbs / peaks["hbm_gbs"],
+            "frac_of_spec": gbs / SPEC_HBM_GBS, "peak_gbs": peaks["hbm_gbs"], "peak_source": f"{peak_src} (hbm_gbs)",
+            "gate_up": {"ms": stage_ms["gemm_gate_up"], "weight_bytes": w_gate_up, "achieved_gbs": gu_gbs,
+                        "frac": gu_gbs / peaks["hbm_gbs"]},
+            "stage_ms": stage_ms, "clocks": clock_info, "steps": steps, "warmup": warmup}
 
 
 def main():

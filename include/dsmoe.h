@@ -133,6 +133,7 @@ void dsmoe_destroy(dsmoe_handle* h);
  * cfg.top_k unless dsmoe_set_selection changed it):
  *
  *   h          bf16 [T, d]        layer output, accumulated in fp32, rounded once
+ *                                 (fp32 partial sums under dsmoe_set_expert_range PARTIAL)
  *   topk_idx   int32 [T, K']      selected experts, by descending selection key,
  *                                 ties to the lower index
  *   gates      fp32 [T, K']       g_{i,t} of the selected experts, same order
@@ -218,7 +219,13 @@ dsmoe_status dsmoe_bias_update(dsmoe_handle* h, int64_t T, const int32_t* counts
  * DSMOE_OK, or DSMOE_ERR_DEVICE_TIMEOUT if a kernel gave up a bounded wait. */
 dsmoe_status dsmoe_get_status(dsmoe_handle* h);
 
-/* Bound on every in-kernel wait, in nanoseconds (default 2e9). */
+/* Bound on the in-kernel waits of later forwards, in nanoseconds (default 2e9): a kernel
+ * role (TMA producer, MMA issuer, epilogue) that waits longer for its operands or its
+ * accumulator gives up, the kernel records it in the status word (dsmoe_get_status then
+ * returns DSMOE_ERR_DEVICE_TIMEOUT) and that forward's outputs are undefined. Before the
+ * kernel exits it still waits for the copies and MMAs it already started, for at least
+ * one second whatever this limit, so that no asynchronous write outlives its CTA.
+ * ns = 0 returns DSMOE_ERR_INVALID_ARG and keeps the previous limit. */
 dsmoe_status dsmoe_set_wait_limit(dsmoe_handle* h, uint64_t ns);
 
 /* Which kernel computes the two grouped expert GEMMs of dsmoe_forward (the gate/up
@@ -251,6 +258,37 @@ int32_t dsmoe_get_gemm_kernel(dsmoe_handle* h);
  * dsmoe_route_noalloc always uses the configuration's plain selection. */
 dsmoe_status dsmoe_set_selection(dsmoe_handle* h, int32_t mask_top, int32_t k_active);
 dsmoe_status dsmoe_get_selection(dsmoe_handle* h, int32_t* mask_top, int32_t* k_active);
+
+/*
+ * Expert range: the part of the layer this handle applies, for expert parallelism
+ * (DeepSeek-MoE interview card, deep dive on engineering trade-offs, item 5: the shared
+ * experts are dense and replicated on every GPU while the routed experts are sharded
+ * across GPUs; "MoE architecture" page, memory section: with expert parallelism each GPU
+ * stores only part of the experts). Later forwards route every token over all N'
+ * experts exactly as before (topk_idx, gates, counts, f, P are the whole layer's), but
+ * apply only the routed experts e_begin <= e < e_end:
+ *   W_gate, W_up [e_end - e_begin, F, d] and W_down [e_end - e_begin, d, F] hold those
+ *   experts only (expert e_begin first); W_router and b stay [N', d] and [N'].
+ * flags:
+ *   DSMOE_RANGE_PARTIAL     h is fp32 [T, d] (not bf16): the partial sum
+ *                           sum_{k : e(t,k) in range} g_{t,k} FFN_{e(t,k)}(u_t), never rounded,
+ *                           for the ranks of an expert-parallel group to add;
+ *   DSMOE_RANGE_ADD_SHARED  add the residual u_t and the shared experts'
+ *                           sum_{i<=K_s} FFN_i(u_t) (one rank of the group does this; Ws_*
+ *                           may be NULL on the others).
+ * The default, (0, N', DSMOE_RANGE_ADD_SHARED), is the whole layer with bf16 h. Any other
+ * part needs DSMOE_RANGE_PARTIAL; a full range with PARTIAL | ADD_SHARED gives the whole
+ * layer unrounded in fp32. Errors: an empty or out-of-bounds range, unknown flags, or a
+ * part without DSMOE_RANGE_PARTIAL return DSMOE_ERR_INVALID_ARG and leave the handle as
+ * it was. dsmoe_forward_host supports the default only (DSMOE_ERR_UNSUPPORTED otherwise).
+ *
+ * dsmoe_round_bf16: dst[i] = bf16(src[i]) (round to nearest even) for n fp32 values,
+ * n a multiple of 8, both device pointers 16-byte aligned; for summed partials.
+ */
+enum { DSMOE_RANGE_PARTIAL = 1, DSMOE_RANGE_ADD_SHARED = 2 };
+dsmoe_status dsmoe_set_expert_range(dsmoe_handle* h, int32_t e_begin, int32_t e_end, int32_t flags);
+dsmoe_status dsmoe_get_expert_range(dsmoe_handle* h, int32_t* e_begin, int32_t* e_end, int32_t* flags);
+dsmoe_status dsmoe_round_bf16(dsmoe_handle* h, int64_t n, const float* src, void* dst, void* stream);
 
 /* Per-stage timing: while enabled, each forward with T > 0 records CUDA events on its
  * stream at every stage boundary (no synchronisation). dsmoe_stage_times waits for
@@ -308,7 +346,9 @@ dsmoe_status dsmoe_workspace_tensor(dsmoe_handle* h, const char* name, void** pt
  * does N' > 512; T > cfg->max_tokens returns DSMOE_ERR_WORKSPACE (dsmoe_last_error
  * says which). The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current); make that first call before
- * any stream capture. Work runs on `stream` of the current device. Every call
+ * any stream capture. Later calls whose stream is not capturing look it up again, so
+ * the address stays valid after cudaDeviceReset; after a reset, make one such call
+ * before capturing again. Work runs on `stream` of the current device. Every call
  * shares the array: each call clears the counters it needs on its stream first,
  * and calls that overlap on the GPU (other streams or threads) race and must be
  * serialised by the caller.

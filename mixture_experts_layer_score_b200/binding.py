@@ -20,6 +20,7 @@ DSMOE_OK, DSMOE_ERR_INVALID_ARG, DSMOE_ERR_UNSUPPORTED, DSMOE_ERR_WORKSPACE, DSM
 DSMOE_SCORE_SOFTMAX, DSMOE_SCORE_SIGMOID, DSMOE_SCORE_SQRT_SOFTPLUS, DSMOE_ROUTE_HASH = range(4)
 DSMOE_BIAS_NONE, DSMOE_BIAS_SELECT_ONLY, DSMOE_BIAS_IN_LOGITS = range(3)
 DSMOE_GEMM_PAIR, DSMOE_GEMM_SINGLE = range(2)
+DSMOE_RANGE_PARTIAL, DSMOE_RANGE_ADD_SHARED = 1, 2
 
 ABI_FUNCTIONS = (
     "dsmoe_abi_version", "dsmoe_status_string", "dsmoe_last_error", "dsmoe_check_config",
@@ -28,7 +29,8 @@ ABI_FUNCTIONS = (
     "dsmoe_stage_times", "dsmoe_stage_name", "dsmoe_launch_count", "dsmoe_workspace_tensor",
     "dsmoe_balance_losses", "dsmoe_sequence_balance", "dsmoe_bias_update",
     "dsmoe_route_noalloc", "dsmoe_set_gemm_kernel", "dsmoe_get_gemm_kernel",
-    "dsmoe_set_selection", "dsmoe_get_selection",
+    "dsmoe_set_selection", "dsmoe_get_selection", "dsmoe_set_expert_range", "dsmoe_get_expert_range",
+    "dsmoe_round_bf16",
 )
 
 
@@ -81,6 +83,10 @@ def _load():
         "dsmoe_workspace_tensor": (ctypes.c_int, [vp, ctypes.c_char_p, ctypes.POINTER(vp),
                                                   ctypes.POINTER(i64), ctypes.POINTER(i64)]),
         "dsmoe_route_noalloc": (ctypes.c_int, [cfgp, i32] + [vp] * 8 + [vp]),
+        "dsmoe_set_expert_range": (ctypes.c_int, [vp, i32, i32, i32]),
+        "dsmoe_get_expert_range": (ctypes.c_int, [vp, ctypes.POINTER(i32), ctypes.POINTER(i32),
+                                                  ctypes.POINTER(i32)]),
+        "dsmoe_round_bf16": (ctypes.c_int, [vp, i64, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -211,6 +217,21 @@ def dsmoe_get_selection(handle):
     return m.value, k.value
 
 
+def dsmoe_set_expert_range(handle, e_begin: int, e_end: int, flags: int) -> None:
+    _check(_lib.dsmoe_set_expert_range(handle, int(e_begin), int(e_end), int(flags)), "dsmoe_set_expert_range")
+
+
+def dsmoe_get_expert_range(handle):
+    b, e, f = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    _check(_lib.dsmoe_get_expert_range(handle, ctypes.byref(b), ctypes.byref(e), ctypes.byref(f)),
+           "dsmoe_get_expert_range")
+    return b.value, e.value, f.value
+
+
+def dsmoe_round_bf16(handle, n: int, src, dst, stream=None) -> None:
+    _check(_lib.dsmoe_round_bf16(handle, int(n), _ptr(src), _ptr(dst), _stream(stream)), "dsmoe_round_bf16")
+
+
 def dsmoe_set_timing(handle, enable: bool) -> None:
     _check(_lib.dsmoe_set_timing(handle, int(bool(enable))), "dsmoe_set_timing")
 
@@ -311,12 +332,21 @@ class DSMoE:
         self.w = weights
         self.handle = dsmoe_create(cfg, device)
         self.mask_top, self.k_active = 0, cfg.top_k
+        self.range_flags = DSMOE_RANGE_ADD_SHARED
 
     def set_selection(self, mask_top: int = 0, k_active: Optional[int] = None):
         """Selection variant for later forwards (see dsmoe_set_selection)."""
         k = self.cfg.top_k if k_active is None else int(k_active)
         dsmoe_set_selection(self.handle, mask_top, k)
         self.mask_top, self.k_active = int(mask_top), k
+
+    def set_expert_range(self, e_begin: int, e_end: int, partial: bool = True, add_shared: bool = False):
+        """Apply only routed experts [e_begin, e_end) in later forwards (see
+        dsmoe_set_expert_range); the weights given at construction must then hold those
+        experts only. With partial, forward() returns h as fp32 partial sums."""
+        flags = (DSMOE_RANGE_PARTIAL if partial else 0) | (DSMOE_RANGE_ADD_SHARED if add_shared else 0)
+        dsmoe_set_expert_range(self.handle, e_begin, e_end, flags)
+        self.range_flags = flags
 
     def close(self):
         if self.handle:
@@ -333,7 +363,8 @@ class DSMoE:
         import torch
         dev = torch.device("cuda", self.device)
         c = self.cfg
-        out = dict(h=torch.empty((T, c.d_model), dtype=torch.bfloat16, device=dev),
+        h_dtype = torch.float32 if self.range_flags & DSMOE_RANGE_PARTIAL else torch.bfloat16
+        out = dict(h=torch.empty((T, c.d_model), dtype=h_dtype, device=dev),
                    topk_idx=torch.empty((T, self.k_active), dtype=torch.int32, device=dev),
                    gates=torch.empty((T, self.k_active), dtype=torch.float32, device=dev),
                    counts=torch.empty((c.n_routed,), dtype=torch.int32, device=dev),

@@ -173,6 +173,11 @@ struct dsmoe_handle {
   int32_t gemm_kernel = DSMOE_GEMM_SINGLE;
   int32_t mask_top = 0;  // selection variant: top-ranked experts masked before the choice
   int32_t k_active = 0;  // selection variant: experts kept per token (cfg.top_k by default)
+  // expert range: the routed experts whose weights this handle applies ([0, N') by
+  // default), whether h is an fp32 partial sum, and whether the residual and the
+  // shared experts are added
+  int32_t e_begin = 0, e_end = 0;
+  bool partial = false, add_shared = true;
   uint64_t wait_ns = kDefaultWaitNs;
   char* ws = nullptr;
   Layout L;
@@ -293,6 +298,7 @@ DSMOE_EXPORT dsmoe_status dsmoe_create(const dsmoe_cfg* cfg, int32_t device, dsm
   if (h->cfg.score == DSMOE_ROUTE_HASH && h->cfg.hash_mod == 0) h->cfg.hash_mod = h->cfg.n_routed;
   h->device = device;
   h->k_active = h->cfg.top_k;
+  h->e_end = h->cfg.n_routed;
   h->num_sms = prop.multiProcessorCount;
   h->pair_clusters[0] = dsmoe::grouped_gemm_pair_max_clusters(false);
   h->pair_clusters[1] = dsmoe::grouped_gemm_pair_max_clusters(true);
@@ -394,7 +400,7 @@ dsmoe_status check_forward(dsmoe_handle* h, const FwdArgs& a) {
   if (hash && !a.token_ids) return fail(DSMOE_ERR_INVALID_ARG, "hash routing needs token_ids");
   if (!hash && !a.W_router) return fail(DSMOE_ERR_INVALID_ARG, "W_router is required");
   if (c.bias_mode != DSMOE_BIAS_NONE && !a.b) return fail(DSMOE_ERR_INVALID_ARG, "bias b is required by bias_mode");
-  if (c.n_shared > 0 && (!a.Ws_gate || !a.Ws_up || !a.Ws_down))
+  if (h->add_shared && c.n_shared > 0 && (!a.Ws_gate || !a.Ws_up || !a.Ws_down))
     return fail(DSMOE_ERR_INVALID_ARG, "shared expert weights are required (n_shared = %d)", c.n_shared);
   const void* must_align[] = {a.x, a.W_router, a.W_gate, a.W_up, a.W_down, a.Ws_gate, a.Ws_up, a.Ws_down, a.h};
   for (const void* p : must_align)
@@ -402,21 +408,24 @@ dsmoe_status check_forward(dsmoe_handle* h, const FwdArgs& a) {
   return DSMOE_OK;
 }
 
+// Tensor maps of the weights, cached per pointer (the routed maps span the handle's
+// expert range; dsmoe_set_expert_range clears the cache).
 const CUtensorMap* weight_map(dsmoe_handle* h, int which, const void* ptr, bool* ok) {
   if (h->wkey[which] != ptr) {
     const dsmoe_cfg& c = h->cfg;
+    const int n_local = h->e_end - h->e_begin;
     bool r = false;
     switch (which) {
       case 0:
-      case 1: r = map_3d(&h->tm_w[which], ptr, c.d_model, c.d_ff, c.n_routed, 128); break;
-      case 2: r = map_3d(&h->tm_w[which], ptr, c.d_ff, c.d_model, c.n_routed, 256); break;
+      case 1: r = map_3d(&h->tm_w[which], ptr, c.d_model, c.d_ff, n_local, 128); break;
+      case 2: r = map_3d(&h->tm_w[which], ptr, c.d_ff, c.d_model, n_local, 256); break;
       case 3:
       case 4: r = map_3d(&h->tm_w[which], ptr, c.d_model, c.d_ff_shared, c.n_shared, 128); break;
       case 5: r = map_3d(&h->tm_w[which], ptr, c.d_ff_shared, c.d_model, c.n_shared, 256); break;
       case 6: r = map_2d(&h->tm_w[which], ptr, c.d_model, c.n_routed, static_cast<uint32_t>(h->rt_nc)); break;
       case 7:
-      case 8: r = map_3d(&h->tm_w[which], ptr, c.d_model, c.d_ff, c.n_routed, dsmoe::kGemmPairGateUpRows); break;
-      case 9: r = map_3d(&h->tm_w[which], ptr, c.d_ff, c.d_model, c.n_routed, 128); break;
+      case 8: r = map_3d(&h->tm_w[which], ptr, c.d_model, c.d_ff, n_local, dsmoe::kGemmPairGateUpRows); break;
+      case 9: r = map_3d(&h->tm_w[which], ptr, c.d_ff, c.d_model, n_local, 128); break;
       case 10:
       case 11:
         r = map_3d(&h->tm_w[which], ptr, c.d_model, c.d_ff_shared, c.n_shared, dsmoe::kGemmPairGateUpRows);
@@ -438,7 +447,9 @@ int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
   const dsmoe_cfg& c = h->cfg;
   const int T = a.T, N = c.n_routed, K = h->k_active, d = c.d_model, F = c.d_ff;
-  const int Ks = c.n_shared, Fs = c.d_ff_shared;
+  // shared experts (and the residual) only where this handle adds them
+  const int Ks = h->add_shared ? c.n_shared : 0, Fs = c.d_ff_shared;
+  const int e0 = h->e_begin, NL = h->e_end - h->e_begin;  // routed experts applied here
   const bool hash = c.score == DSMOE_ROUTE_HASH;
   const bool timing = h->timing && T > 0;
   cudaEvent_t* evs = h->ev[h->timed_forwards % kTimingSlots];
@@ -542,12 +553,14 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
   sc.P_sum = a.P_sum;
   sc.offsets = h->offsets;
   sc.cursor = h->cursor;
+  sc.e_begin = e0;
+  sc.e_end = e0 + NL;
   CUDA_TRY(dsmoe::launch_scan_stats(sc, s));
   h->launches += 1;
   CUDA_TRY(mark(3));
 
-  CUDA_TRY(dsmoe::launch_permute_gather(static_cast<const bf16*>(a.x), a.topk_idx, h->offsets, h->cursor, T, K, N, d,
-                                        h->slot_of, h->Xp, h->status, h->num_sms, s));
+  CUDA_TRY(dsmoe::launch_permute_gather(static_cast<const bf16*>(a.x), a.topk_idx, h->offsets, h->cursor, T, K, N,
+                                        e0, e0 + NL, d, h->slot_of, h->Xp, h->status, h->num_sms, s));
   h->launches += 1;
   CUDA_TRY(mark(4));
 
@@ -562,8 +575,8 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
     g.b1_routed = *m_wu;
     g.b0_shared = *m_swg;
     g.b1_shared = *m_swu;
-    g.offsets = h->offsets;
-    g.n_routed = N;
+    g.offsets = h->offsets + e0;
+    g.n_routed = NL;
     g.n_shared_groups = Ks;
     g.m_shared = T;
     g.n_tiles_routed = cdiv(F, 128);
@@ -581,7 +594,7 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
     g.status = h->status;
     g.wait_limit_ns = h->wait_ns;
     const int64_t tt = pair ? dsmoe::kGemmPairTokenTile : dsmoe::kGemmGateUpTokenTile;
-    const int64_t bound = (cdiv(S, tt) + N) * static_cast<int64_t>(g.n_tiles_routed) +
+    const int64_t bound = (cdiv(S, tt) + NL) * static_cast<int64_t>(g.n_tiles_routed) +
                           static_cast<int64_t>(Ks) * cdiv(T, tt) * g.n_tiles_shared;
     if (pair) {
       const int clusters = static_cast<int>(bound < h->pair_clusters[1] ? bound : h->pair_clusters[1]);
@@ -603,8 +616,8 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
     g.b1_routed = *m_wd;
     g.b0_shared = *m_swd;
     g.b1_shared = *m_swd;
-    g.offsets = h->offsets;
-    g.n_routed = N;
+    g.offsets = h->offsets + e0;
+    g.n_routed = NL;
     g.n_shared_groups = Ks ? 1 : 0;
     g.m_shared = T;
     g.n_tiles_routed = cdiv(d, 256);
@@ -624,7 +637,7 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
     g.status = h->status;
     g.wait_limit_ns = h->wait_ns;
     const int64_t tt = pair ? dsmoe::kGemmPairTokenTile : dsmoe::kGemmDownTokenTile;
-    const int64_t bound = (cdiv(S, tt) + N) * static_cast<int64_t>(g.n_tiles_routed) +
+    const int64_t bound = (cdiv(S, tt) + NL) * static_cast<int64_t>(g.n_tiles_routed) +
                           static_cast<int64_t>(g.n_shared_groups) * cdiv(T, tt) * g.n_tiles_shared;
     if (pair) {
       const int clusters = static_cast<int>(bound < h->pair_clusters[0] ? bound : h->pair_clusters[0]);
@@ -636,8 +649,21 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
     h->launches += 1;
   }
   CUDA_TRY(mark(6));
-  CUDA_TRY(dsmoe::launch_combine(static_cast<const bf16*>(a.x), Ks ? h->Hs : nullptr, h->Y, h->slot_of, a.gates, T,
-                                 K, d, static_cast<bf16*>(a.h), h->num_sms, s));
+  {
+    dsmoe::CombineArgs ca;
+    ca.x = static_cast<const bf16*>(a.x);
+    ca.Hs = Ks ? h->Hs : nullptr;
+    ca.add_x = h->add_shared ? 1 : 0;
+    ca.Y = h->Y;
+    ca.slot_of = h->slot_of;
+    ca.gates = a.gates;
+    ca.T = T;
+    ca.K = K;
+    ca.d = d;
+    ca.h = h->partial ? nullptr : static_cast<bf16*>(a.h);
+    ca.h32 = h->partial ? static_cast<float*>(a.h) : nullptr;
+    CUDA_TRY(dsmoe::launch_combine(ca, h->num_sms, s));
+  }
   h->launches += 1;
   CUDA_TRY(mark(7));
   if (timing) h->timed_forwards += 1;
@@ -670,6 +696,7 @@ DSMOE_EXPORT dsmoe_status dsmoe_forward_host(dsmoe_handle* h, int32_t T, const v
                                              int32_t* counts_host, float* f_host, float* P_host, void* stream) {
   if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
   const dsmoe_cfg& c = h->cfg;
+  if (h->partial) return fail(DSMOE_ERR_UNSUPPORTED, "the host entry point runs the whole layer only");
   if (T < 0) return fail(DSMOE_ERR_INVALID_ARG, "T = %d is negative", T);
   if (T > c.max_tokens) return fail(DSMOE_ERR_WORKSPACE, "T = %d exceeds max_tokens = %d", T, c.max_tokens);
   if (!counts_host || !f_host || !P_host) return fail(DSMOE_ERR_INVALID_ARG, "counts, f and P are required");
@@ -733,6 +760,7 @@ DSMOE_EXPORT dsmoe_status dsmoe_get_status(dsmoe_handle* h) {
 
 DSMOE_EXPORT dsmoe_status dsmoe_set_wait_limit(dsmoe_handle* h, uint64_t ns) {
   if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  if (ns == 0) return fail(DSMOE_ERR_INVALID_ARG, "the wait limit must be at least 1 ns");
   h->wait_ns = ns;
   return DSMOE_OK;
 }
@@ -768,6 +796,48 @@ DSMOE_EXPORT dsmoe_status dsmoe_get_selection(dsmoe_handle* h, int32_t* mask_top
   if (!h || !mask_top || !k_active) return fail(DSMOE_ERR_INVALID_ARG, "NULL argument");
   *mask_top = h->mask_top;
   *k_active = h->k_active;
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_set_expert_range(dsmoe_handle* h, int32_t e_begin, int32_t e_end, int32_t flags) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  const dsmoe_cfg& c = h->cfg;
+  if (e_begin < 0 || e_end <= e_begin || e_end > c.n_routed)
+    return fail(DSMOE_ERR_INVALID_ARG, "expert range [%d, %d) is not a non-empty part of [0, %d)", e_begin, e_end,
+                c.n_routed);
+  if (flags & ~(DSMOE_RANGE_PARTIAL | DSMOE_RANGE_ADD_SHARED))
+    return fail(DSMOE_ERR_INVALID_ARG, "unknown expert-range flags 0x%x", flags);
+  const bool partial = (flags & DSMOE_RANGE_PARTIAL) != 0, add_shared = (flags & DSMOE_RANGE_ADD_SHARED) != 0;
+  if (!partial && (e_begin != 0 || e_end != c.n_routed || !add_shared))
+    return fail(DSMOE_ERR_INVALID_ARG, "a part of the layer (an expert sub-range, or no residual and shared "
+                "experts) needs DSMOE_RANGE_PARTIAL: its output is an fp32 partial sum");
+  if (e_begin != h->e_begin || e_end != h->e_end)
+    for (int i = 0; i < dsmoe_handle::kMaps; ++i) h->wkey[i] = nullptr;  // routed maps span the range
+  h->e_begin = e_begin;
+  h->e_end = e_end;
+  h->partial = partial;
+  h->add_shared = add_shared;
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_get_expert_range(dsmoe_handle* h, int32_t* e_begin, int32_t* e_end, int32_t* flags) {
+  if (!h || !e_begin || !e_end || !flags) return fail(DSMOE_ERR_INVALID_ARG, "NULL argument");
+  *e_begin = h->e_begin;
+  *e_end = h->e_end;
+  *flags = (h->partial ? DSMOE_RANGE_PARTIAL : 0) | (h->add_shared ? DSMOE_RANGE_ADD_SHARED : 0);
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_round_bf16(dsmoe_handle* h, int64_t n, const float* src, void* dst, void* stream) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  if (n < 0 || n % 8) return fail(DSMOE_ERR_INVALID_ARG, "n = %lld is not a non-negative multiple of 8",
+                                  static_cast<long long>(n));
+  if (n > 0 && (!src || !dst)) return fail(DSMOE_ERR_INVALID_ARG, "NULL argument");
+  if (!aligned16(src) || !aligned16(dst)) return fail(DSMOE_ERR_INVALID_ARG, "src and dst must be 16-byte aligned");
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
+  CUDA_TRY(dsmoe::launch_round_bf16(src, static_cast<bf16*>(dst), n, h->num_sms, static_cast<cudaStream_t>(stream)));
+  if (n > 0) h->launches += 1;
   return DSMOE_OK;
 }
 

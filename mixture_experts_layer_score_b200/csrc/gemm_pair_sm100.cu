@@ -375,13 +375,15 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair_kernel(const __
       for (int s = 0; s < kStages; ++s) {
         const uint32_t n_peer = pair::ld_cluster_u32(pair::map_to(smem_addr(&issued_n[s]), 1));
         const uint32_t n = max(issued_n[s], n_peer);
-        if (n > 0 && !pair::mbar_wait_bounded_cl(&landed[s], (n - 1) & 1u, a.wait_limit_ns, never_flag))
+        if (n > 0 &&
+            !pair::mbar_wait_bounded_cl(&landed[s], (n - 1) & 1u, drain_wait_limit(a.wait_limit_ns), never_flag))
           atomicOr(a.status, kStatusTimeoutDrain);
       }
     }
     if (warp == 1 && lane == 0) {
       pair::mma_commit_local(drain);
-      if (!pair::mbar_wait_bounded_cl(drain, 0, a.wait_limit_ns, never_flag)) atomicOr(a.status, kStatusTimeoutDrain);
+      if (!pair::mbar_wait_bounded_cl(drain, 0, drain_wait_limit(a.wait_limit_ns), never_flag))
+        atomicOr(a.status, kStatusTimeoutDrain);
     }
   }
   tc_fence_before();

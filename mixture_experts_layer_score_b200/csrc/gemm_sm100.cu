@@ -34,7 +34,8 @@
 //
 // Every wait is bounded (wait_limit_ns); a role that gives up raises a CTA-wide abort
 // flag and a bit of the device status word, the CTA lets in-flight TMA loads and MMAs
-// finish (again bounded), frees its TMEM and returns.
+// finish (a wait bounded by at least one second, whatever the caller's limit), frees its
+// TMEM and returns.
 #include "grouped_tiles.cuh"
 #include "sm100_ptx.cuh"
 
@@ -313,12 +314,13 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
     if (warp == 0 && lane == 0) {
       for (int s = 0; s < G_::kStages; ++s)
         if ((issued_mask >> s) & 1u)
-          if (!mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, a.wait_limit_ns, never_flag))
+          if (!mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, drain_wait_limit(a.wait_limit_ns), never_flag))
             atomicOr(a.status, kStatusTimeoutDrain);
     }
     if (warp == 1 && lane == 0) {
       mma_commit(drain);
-      if (!mbar_wait_bounded(drain, 0, a.wait_limit_ns, never_flag)) atomicOr(a.status, kStatusTimeoutDrain);
+      if (!mbar_wait_bounded(drain, 0, drain_wait_limit(a.wait_limit_ns), never_flag))
+        atomicOr(a.status, kStatusTimeoutDrain);
     }
   }
   tc_fence_before();

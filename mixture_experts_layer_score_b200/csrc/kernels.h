@@ -86,6 +86,7 @@ struct ScanArgs {
   float* P_sum;              // [N] out or nullptr
   int32_t* offsets;          // [N+1] out, or nullptr
   int32_t* cursor;           // [N] zeroed, or nullptr
+  int32_t e_begin, e_end;    // experts that get slots; the others' segments are empty
 };
 cudaError_t launch_scan_stats(const ScanArgs& a, cudaStream_t s);
 
@@ -93,10 +94,11 @@ cudaError_t launch_scan_stats(const ScanArgs& a, cudaStream_t s);
 cudaError_t launch_balance_stats(const int32_t* counts, const float* P_sum, int64_t T, int N, int K,
                                  float* f, float* P, cudaStream_t s);
 
-// slot positions + gather of token rows into expert-contiguous order.
+// slot positions + gather of token rows into expert-contiguous order. Only experts in
+// [e_begin, e_end) get slots; a (token, k) whose expert lies outside has slot -1.
 cudaError_t launch_permute_gather(const bf16* x, const int32_t* topk_idx, const int32_t* offsets,
-                                  int32_t* cursor, int T, int K, int N, int d, int32_t* slot_of, bf16* Xp,
-                                  uint32_t* status, int num_sms, cudaStream_t s);
+                                  int32_t* cursor, int T, int K, int N, int e_begin, int e_end, int d,
+                                  int32_t* slot_of, bf16* Xp, uint32_t* status, int num_sms, cudaStream_t s);
 
 // ---------------------------------------------------------------- balance control (balance.cu)
 cudaError_t launch_balance_losses(const float* f, const float* P, int N, int G, const int32_t* group_of,
@@ -109,10 +111,23 @@ cudaError_t launch_bias_update(const int32_t* counts, int64_t T, int N, int K, f
                                cudaStream_t s);
 
 // ---------------------------------------------------------------- combine (combine.cu)
-// h = base + sum_k gates[t,k] Y[slot_of[t,k]], where base is Hs (fp32 x + shared experts)
-// when Hs is not null, else x.
-cudaError_t launch_combine(const bf16* x, const float* Hs, const bf16* Y, const int32_t* slot_of,
-                           const float* gates, int T, int K, int d, bf16* h, int num_sms, cudaStream_t s);
+// h = base + sum_k gates[t,k] Y[slot_of[t,k]] over the k whose slot is not -1, where base
+// is Hs (fp32 x + shared experts) when Hs is not null, else x when add_x, else 0; written
+// as bf16 h (rounded once) or, when h32 is not null, as fp32 h32.
+struct CombineArgs {
+  const bf16* x;
+  const float* Hs;
+  int add_x;
+  const bf16* Y;
+  const int32_t* slot_of;
+  const float* gates;
+  int T, K, d;
+  bf16* h;
+  float* h32;
+};
+cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s);
+// dst[i] = bf16(src[i]) (round to nearest even), n a multiple of 8, both 16-byte aligned.
+cudaError_t launch_round_bf16(const float* src, bf16* dst, int64_t n, int num_sms, cudaStream_t s);
 
 // ---------------------------------------------------------------- grouped GEMM (gemm_sm100.cu)
 // Tokens per grouped-GEMM tile of each projection (the row box of its token-side

@@ -15,6 +15,8 @@ __global__ void __launch_bounds__(kScanThreads) scan_stats_kernel(const ScanArgs
   __shared__ int32_t warp_tot[kScanThreads / 32];
   const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
   const int32_t c = (i < a.N) ? a.counts_ws[i] : 0;
+  // slots exist only for the experts in [e_begin, e_end); the statistics use every count
+  const int32_t c_slots = (i >= a.e_begin && i < a.e_end) ? c : 0;
   if (i < a.N) {
     a.counts[i] = c;
     a.f[i] = (a.T > 0) ? static_cast<float>(static_cast<double>(a.N) * c / (static_cast<double>(a.K) * a.T)) : 0.f;
@@ -26,8 +28,8 @@ __global__ void __launch_bounds__(kScanThreads) scan_stats_kernel(const ScanArgs
     if (a.cursor) a.cursor[i] = 0;
   }
   if (!a.offsets) return;
-  // exclusive scan of the counts -> slot offset of each expert's segment
-  int32_t v = c;
+  // exclusive scan of the slot counts -> slot offset of each expert's segment
+  int32_t v = c_slots;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int32_t n = __shfl_up_sync(0xffffffffu, v, o);
@@ -46,7 +48,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_stats_kernel(const ScanArgs
   }
   __syncthreads();
   const int32_t incl = v + (warp > 0 ? warp_tot[warp - 1] : 0);
-  if (i < a.N) a.offsets[i] = incl - c;
+  if (i < a.N) a.offsets[i] = incl - c_slots;
   if (i == a.N - 1) a.offsets[a.N] = incl;
 }
 
@@ -58,13 +60,15 @@ __global__ void balance_stats_kernel(const int32_t* __restrict__ counts, const f
   }
 }
 
-// One warp per token: lanes k < K' claim a slot in expert topk_idx[t,k]'s segment, then
-// the warp copies the token's row (16-byte vectors) to each claimed slot.
+// One warp per token: lanes k < K' claim a slot in expert topk_idx[t,k]'s segment (experts
+// in [e_begin, e_end) only; the others get slot -1), then the warp copies the token's row
+// (16-byte vectors) to each claimed slot.
 __global__ void __launch_bounds__(256) permute_gather_kernel(const bf16* __restrict__ x,
                                                              const int32_t* __restrict__ topk_idx,
                                                              const int32_t* __restrict__ offsets,
                                                              int32_t* __restrict__ cursor, int T, int K, int N,
-                                                             int d, int32_t* __restrict__ slot_of,
+                                                             int e_begin, int e_end, int d,
+                                                             int32_t* __restrict__ slot_of,
                                                              bf16* __restrict__ Xp, uint32_t* status) {
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, nw = (gridDim.x * blockDim.x) >> 5;
@@ -75,10 +79,10 @@ __global__ void __launch_bounds__(256) permute_gather_kernel(const bf16* __restr
     int pos = -1;
     if (lane < K) {
       const int e = topk_idx[static_cast<int64_t>(t) * K + lane];
-      if (e >= 0 && e < N) {
-        pos = offsets[e] + atomicAdd(&cursor[e], 1);
-      } else {
+      if (e < 0 || e >= N) {
         atomicOr(status, kStatusBadIndex);
+      } else if (e >= e_begin && e < e_end) {
+        pos = offsets[e] + atomicAdd(&cursor[e], 1);
       }
       slot_of[static_cast<int64_t>(t) * K + lane] = pos;
     }
@@ -121,14 +125,14 @@ cudaError_t launch_balance_stats(const int32_t* counts, const float* P_sum, int6
 }
 
 cudaError_t launch_permute_gather(const bf16* x, const int32_t* topk_idx, const int32_t* offsets,
-                                  int32_t* cursor, int T, int K, int N, int d, int32_t* slot_of, bf16* Xp,
-                                  uint32_t* status, int num_sms, cudaStream_t s) {
+                                  int32_t* cursor, int T, int K, int N, int e_begin, int e_end, int d,
+                                  int32_t* slot_of, bf16* Xp, uint32_t* status, int num_sms, cudaStream_t s) {
   const int warps_per_block = 8;
   int grid = (T + warps_per_block - 1) / warps_per_block;
   if (grid > 8 * num_sms) grid = 8 * num_sms;
   if (grid < 1) grid = 1;
-  permute_gather_kernel<<<grid, warps_per_block * 32, 0, s>>>(x, topk_idx, offsets, cursor, T, K, N, d, slot_of,
-                                                              Xp, status);
+  permute_gather_kernel<<<grid, warps_per_block * 32, 0, s>>>(x, topk_idx, offsets, cursor, T, K, N, e_begin,
+                                                              e_end, d, slot_of, Xp, status);
   return cudaGetLastError();
 }
 

@@ -260,10 +260,20 @@ DSMOE_EXPORT dsmoe_status dsmoe_route_noalloc(const dsmoe_cfg* cfg, int32_t T, c
     dsmoe::note_error("dsmoe_route_noalloc: no usable current device");
     return DSMOE_ERR_CUDA;
   }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // The array's device address is looked up with the device current and kept per
+  // device. A call whose stream is not being captured looks it up again, so that the
+  // address stays right after cudaDeviceReset reloads the library's device image; a
+  // call under capture uses the address an earlier call found.
+  cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &capture) != cudaSuccess) {
+    dsmoe::note_error("dsmoe_route_noalloc: cudaStreamIsCapturing failed on the given stream");
+    return DSMOE_ERR_CUDA;
+  }
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_setup_mu);
-    if (!g_scratch_addr[dev]) {
+    if (!g_scratch_addr[dev] || capture == cudaStreamCaptureStatusNone) {
       void* p = nullptr;
       const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
       if (e != cudaSuccess || !p) {
@@ -274,7 +284,6 @@ DSMOE_EXPORT dsmoe_status dsmoe_route_noalloc(const dsmoe_cfg* cfg, int32_t T, c
     }
     scratch = g_scratch_addr[dev];
   }
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int N = cfg->n_routed;
   if (T == 0) {
     if (cudaMemsetAsync(counts, 0, N * sizeof(int32_t), s) != cudaSuccess ||

@@ -214,12 +214,13 @@ __global__ void __launch_bounds__(kThreads, 1) router_tc_kernel(const __grid_con
     if (warp == 0 && lane == 0) {
       for (int s = 0; s < stages; ++s)
         if ((issued_mask >> s) & 1u)
-          if (!mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, a.wait_limit_ns, never_flag))
+          if (!mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, drain_wait_limit(a.wait_limit_ns), never_flag))
             atomicOr(a.status, kStatusTimeoutDrain);
     }
     if (warp == 1 && lane == 0) {
       mma_commit(drain);
-      if (!mbar_wait_bounded(drain, 0, a.wait_limit_ns, never_flag)) atomicOr(a.status, kStatusTimeoutDrain);
+      if (!mbar_wait_bounded(drain, 0, drain_wait_limit(a.wait_limit_ns), never_flag))
+        atomicOr(a.status, kStatusTimeoutDrain);
     }
   }
   tc_fence_before();

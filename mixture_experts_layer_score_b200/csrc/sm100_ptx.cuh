@@ -68,6 +68,15 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// Limit of the waits of an abort drain: after a role gave up, the CTA waits for the TMA
+// copies and MMAs it already started before it releases their shared and tensor memory.
+// Those always finish on their own, so this wait must not be cut short by a small
+// caller-chosen limit: it takes the larger of that limit and one second.
+constexpr uint64_t kDrainWaitFloorNs = 1000000000ull;
+__host__ __device__ __forceinline__ uint64_t drain_wait_limit(uint64_t limit_ns) {
+  return limit_ns > kDrainWaitFloorNs ? limit_ns : kDrainWaitFloorNs;
+}
+
 // The same wait for a whole warp that is not on the critical path (an epilogue waiting
 // for an accumulator): only lane 0 polls, backing off with __nanosleep so that the
 // polling does not compete with the TMA and MMA traffic on the barrier's shared-memory

@@ -1,12 +1,23 @@
-"""Token-sharded data parallelism for the layer forward, one process per GPU.
+"""Multi-GPU forms of the layer forward, one process per GPU.
 
-Tokens are independent through the whole layer, so each rank runs the forward on
-its own contiguous shard of the batch with a full copy of the weights and no
-data-path exchange. The one step that spans ranks is the expert-level balance
-statistics f_i and P_i (DeepSeekMoE summary, "Expert-level balance loss"),
-which are defined over every token of the batch: each rank's token counts and
-score sums are summed across ranks (one all-reduce of 2 N' words) and the
+Token sharding (prefill): tokens are independent through the whole layer, so each
+rank runs the forward on its own contiguous shard of the batch with a full copy of
+the weights and no data-path exchange. The one step that spans ranks is the
+expert-level balance statistics f_i and P_i (DeepSeekMoE summary, "Expert-level
+balance loss"), which are defined over every token of the batch: each rank's token
+counts and score sums are summed across ranks (one all-reduce of 2 N' words) and the
 library turns the sums into f and P (dsmoe_balance_stats).
+
+Expert sharding (decode): with few tokens and hundreds of experts, token shards would
+each stream almost every expert's weights. Instead each rank holds a contiguous block
+of the routed experts and all ranks replicate the router and the shared experts (the
+DeepSeek-MoE interview card's deployment trade-off: shared experts on every GPU,
+routed experts sharded). Every rank gathers all ranks' tokens (all-gather of x),
+routes them all (the router is replicated, so every rank makes the same choice),
+applies its own experts into an fp32 partial sum, one rank also adds the residual and
+the shared experts, and a reduce-scatter sums the partials and hands each rank its own
+tokens' rows, which the library rounds to bf16 once. Each expert's weights are then
+read on one GPU only.
 """
 from __future__ import annotations
 
@@ -37,3 +48,49 @@ def global_balance_stats(handle, T_total: int, counts: torch.Tensor, P_sum: torc
     from .binding import dsmoe_balance_stats
     reduce_balance_sums(counts, P_sum, group)
     dsmoe_balance_stats(handle, T_total, counts, P_sum, f, P, stream)
+
+
+def expert_block(n_routed: int, rank: int, world: int) -> Tuple[int, int]:
+    """[e_begin, e_end) of the routed experts rank holds: contiguous blocks, sizes
+    differing by at most one."""
+    return shard_rows(n_routed, rank, world)
+
+
+def configure_expert_shard(layer, rank: int, world: int) -> Tuple[int, int]:
+    """Set a layer (binding.DSMoE built with this rank's block of expert weights) to apply
+    its block and write fp32 partial sums; rank 0 also adds the residual and the shared
+    experts."""
+    e0, e1 = expert_block(layer.cfg.n_routed, rank, world)
+    layer.set_expert_range(e0, e1, partial=True, add_shared=(rank == 0))
+    return e0, e1
+
+
+def expert_sharded_forward(layer, x_local: torch.Tensor, token_ids_local: torch.Tensor = None, group=None,
+                           stream=None, round_bf16=None):
+    """The layer on this rank's tokens in the expert-sharded form. Every rank must pass the
+    same number of tokens. Returns h (bf16, this rank's rows), this rank's topk_idx and
+    gates, and the whole batch's counts, f and P (identical on every rank).
+
+    round_bf16(src, dst) turns the summed fp32 rows into bf16; by default the library's
+    kernel (dsmoe_round_bf16) on `stream`."""
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    T, d = x_local.shape
+    x_all = torch.empty((world * T, d), dtype=x_local.dtype, device=x_local.device)
+    dist.all_gather_into_tensor(x_all, x_local.contiguous(), group=group)
+    ids_all = None
+    if token_ids_local is not None:
+        ids_all = torch.empty((world * T,), dtype=token_ids_local.dtype, device=token_ids_local.device)
+        dist.all_gather_into_tensor(ids_all, token_ids_local.contiguous(), group=group)
+    out = layer.forward(x_all, token_ids=ids_all, stream=stream)
+    mine = torch.empty((T, d), dtype=torch.float32, device=x_local.device)
+    dist.reduce_scatter_tensor(mine, out["h"], op=dist.ReduceOp.SUM, group=group)
+    h = torch.empty((T, d), dtype=torch.bfloat16, device=x_local.device)
+    if round_bf16 is None:
+        from .binding import dsmoe_round_bf16
+        dsmoe_round_bf16(layer.handle, T * d, mine, h, stream)
+    else:
+        round_bf16(mine, h)
+    rows = slice(rank * T, (rank + 1) * T)
+    return dict(h=h, topk_idx=out["topk_idx"][rows], gates=out["gates"][rows], counts=out["counts"], f=out["f"],
+                P=out["P"])

@@ -126,16 +126,38 @@ def ep_gather_forward_rank(cfg, local_inputs: Dict, local_experts: Dict[int, tup
     r = O.route(cfg, full)
     idx = np.asarray(r["idx"], dtype=np.int64)
     g = np.asarray(r["gates"], dtype=np.float64)
-    partial = np.zeros_like(X)
-    for e in np.unique(idx):
-        if int(expert_owner(e, cfg.n_routed, world)) != rank:
-            continue
-        rows, ks = np.nonzero(idx == e)
-        Wg, Wu, Wd = local_experts[int(e)]
-        partial[rows] += g[rows, ks][:, None] * O.swiglu_ffn(X[rows], Wg, Wu, Wd)
+    owned = [e for e in range(cfg.n_routed) if int(expert_owner(e, cfg.n_routed, world)) == rank]
+    partial = gather_partial(X, idx, g, local_experts, owned)
     total = allreduce_sum(partial)
     n = X_local.shape[0]
     h = X_local + total[start:start + n]
     for (Wg, Wu, Wd) in shared:
         h += O.swiglu_ffn(X_local, Wg, Wu, Wd)
     return dict(h=h, idx=idx[start:start + n], gates=g[start:start + n])
+
+
+def gather_partial(X, idx, gates, local_experts: Dict[int, tuple], owned, shared: List[tuple] = None,
+                   rows=None) -> np.ndarray:
+    """One rank's share of the decode-shaped expert-parallel form, before the sum over
+    ranks: for every gathered token t (or the given rows), sum over its picks k whose
+    expert the rank owns of g_{t,k} FFN_e(u_t); with `shared` given (the one rank that
+    adds them), plus u_t and the shared experts' outputs. The sum of all ranks' partials
+    is the layer output (the shared-expert layer equation split by expert owner)."""
+    X = O._as_f64(X)
+    idx = np.asarray(idx, dtype=np.int64)
+    gates = np.asarray(gates, dtype=np.float64)
+    rows = np.arange(X.shape[0]) if rows is None else np.asarray(rows, dtype=np.int64)
+    Xr, ir, gr = X[rows], idx[rows], gates[rows]
+    partial = np.zeros_like(Xr)
+    owned = set(int(e) for e in owned)
+    for e in np.unique(ir):
+        if int(e) not in owned:
+            continue
+        rr, ks = np.nonzero(ir == e)
+        Wg, Wu, Wd = local_experts[int(e)]
+        partial[rr] += gr[rr, ks][:, None] * O.swiglu_ffn(Xr[rr], Wg, Wu, Wd)
+    if shared is not None:
+        partial += Xr
+        for (Wg, Wu, Wd) in shared:
+            partial += O.swiglu_ffn(Xr, Wg, Wu, Wd)
+    return partial

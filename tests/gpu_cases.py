@@ -28,8 +28,18 @@ class LazyExperts:
         return self.t.shape[0]
 
 
-def make_case(cfg: W.MoEConfig, T: int, seed: int = 0, gen_device: str = "cpu"):
-    """Inputs drawn on gen_device; returns (inputs on cuda:0, CPU view for the oracle)."""
+# Layers whose expert weights exceed this are drawn on the GPU (the oracle then copies
+# only the experts it needs); drawing 20-35 GB of V3/V4-shaped weights with the CPU
+# generator takes over a minute per case.
+GPU_DRAW_BYTES = 1 << 30
+
+
+def make_case(cfg: W.MoEConfig, T: int, seed: int = 0, gen_device: str = None):
+    """Inputs drawn on gen_device (default: the GPU for layers whose weights exceed
+    GPU_DRAW_BYTES, else the CPU); returns (inputs on cuda:0, CPU view for the oracle)."""
+    if gen_device is None:
+        big = cfg.routed_weight_bytes() + cfg.shared_weight_bytes() > GPU_DRAW_BYTES
+        gen_device = "cuda" if big else "cpu"
     inp = W.make_inputs(cfg, seed=seed, device=gen_device, T=T)
     gpu, cpu = {}, {}
     for k, v in inp.items():

@@ -120,3 +120,30 @@ def test_expert_parallel_oracle_equals_single_device(name, world):
         np.testing.assert_allclose(h, ref["h"][a:b], rtol=1e-12, atol=1e-12)
         np.testing.assert_allclose(h_gather, ref["h"][a:b], rtol=1e-12, atol=1e-12)
         assert loads.sum() == cfg.T * cfg.top_k
+
+
+@pytest.mark.parametrize("world", [1, 2, 3])
+def test_gather_partials_sum_to_the_layer(world):
+    """The decode form's per-rank partial sums (uneven contiguous expert blocks, one rank
+    adding the residual and the shared experts) add up to the single-device layer."""
+    import workloads as W
+    from oracle import dsmoe_oracle as O
+    from oracle import dsmoe_ep as EP
+    cfg = _cfg("tiny")
+    inp = W.make_inputs(cfg, seed=2)
+    ref = O.forward(cfg, inp)
+    N = cfg.n_routed
+    shared = [(inp["Ws_gate"][i], inp["Ws_up"][i], inp["Ws_down"][i]) for i in range(cfg.n_shared)]
+    total = 0.0
+    for rank in range(world):
+        e0 = (N // world) * rank + min(rank, N % world)
+        e1 = e0 + N // world + (1 if rank < N % world else 0)
+        local = {e: (inp["W_gate"][e], inp["W_up"][e], inp["W_down"][e]) for e in range(e0, e1)}
+        part = EP.gather_partial(inp["x"], ref["idx"], ref["gates"], local, range(e0, e1),
+                                 shared if rank == 0 else None)
+        rows = np.array([3, 0, 150])
+        sub = EP.gather_partial(inp["x"], ref["idx"], ref["gates"], local, range(e0, e1),
+                                shared if rank == 0 else None, rows=rows)
+        np.testing.assert_allclose(sub, part[rows], rtol=1e-12, atol=1e-12)
+        total = total + part
+    np.testing.assert_allclose(total, ref["h"], rtol=1e-12, atol=1e-12)

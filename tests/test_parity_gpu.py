@@ -19,7 +19,7 @@ if not torch.cuda.is_available():
     pytest.skip("no GPU", allow_module_level=True)
 
 
-def _check(cfg, T, rows_n=None, gen_device="cpu", seed=0, gemm_kernel=None):
+def _check(cfg, T, rows_n=None, gen_device=None, seed=0, gemm_kernel=None):
     gpu, cpu = make_case(cfg, T, seed=seed, gen_device=gen_device)
     out = run_cuda(cfg, gpu, T, gemm_kernel=gemm_kernel)
     ref = PAR.reference_selection(cfg, cpu, out["topk_idx"], out["scores"])
@@ -66,8 +66,8 @@ def test_gemm_kernels_agree():
     assert float(d.max()) == 0.0
 
 
-FULL = [("gshard_a", 128), ("gshard_b", 128), ("gshard_c", 128), ("ds2b", 128), ("v3_prefill", 32),
-        ("v4_decode_t256", 32), ("v4_hash_t256", 32)]
+# (the V3 prefill and V4 decode T=256 layers at full size are in test_fullsize_stages_gpu.py)
+FULL = [("gshard_a", 128), ("gshard_b", 128), ("gshard_c", 128), ("ds2b", 128), ("v4_hash_t256", 64)]
 
 
 @pytest.mark.parametrize("name,rows", FULL, ids=[n for n, _ in FULL])
