@@ -290,6 +290,85 @@ dsmoe_status dsmoe_set_expert_range(dsmoe_handle* h, int32_t e_begin, int32_t e_
 dsmoe_status dsmoe_get_expert_range(dsmoe_handle* h, int32_t* e_begin, int32_t* e_end, int32_t* flags);
 dsmoe_status dsmoe_round_bf16(dsmoe_handle* h, int64_t n, const float* src, void* dst, void* stream);
 
+/*
+ * Expert parallelism with token dispatch: routed experts split over `world` ranks in
+ * contiguous blocks (rank j holds experts [j*B + min(j, R), ...) with B = N' / world,
+ * R = N' % world, the first R blocks one larger), the router and the shared experts
+ * replicated on every rank (DeepSeek-MoE interview card, deep dive on engineering
+ * trade-offs, item 5; "MoE: sparse activation" page, training-cost section: tokens travel
+ * by all-to-all to the GPUs that hold their experts). Each rank calls, in order:
+ *
+ * dsmoe_ep_route -- route its T tokens (as dsmoe_forward: topk_idx, gates, counts, f, P,
+ *   P_sum, scores_dbg over its own tokens) and gather their rows into the expert-
+ *   contiguous slot order, which is also destination order: workspace "Xp" rows
+ *   [0, T K') are what this rank sends. send_rows int32 [world] (device, out) = rows
+ *   bound for each rank. The per-expert row counts to send are `counts` (rank j's block).
+ * (the caller exchanges the per-expert counts and the rows, e.g. NCCL all-to-all)
+ * dsmoe_ep_experts -- the owner's experts on the rows it received: rows bf16
+ *   [n_rows, d] grouped by source rank, and within a source by expert; recv_counts int32
+ *   [n_src, e_end - e_begin] (device) rows per (source, local expert); W_gate, W_up
+ *   [e_end - e_begin, F, d] and W_down [e_end - e_begin, d, F] this rank's experts.
+ *   Writes Y bf16 [n_rows, d], row for row. n_rows <= max_tokens * top_k and
+ *   n_src * (e_end - e_begin) <= 512 (DSMOE_ERR_WORKSPACE / DSMOE_ERR_UNSUPPORTED).
+ * (the caller sends Y back along the reverse exchange, so that it arrives in the order
+ *  the rows left)
+ * dsmoe_ep_combine -- the shared experts on the rank's own tokens and the combine
+ *   h_t = u_t + sum_shared FFN(u_t) + sum_k g_{t,k} Y[slot(t,k)], Y bf16 [T K', d] in
+ *   this rank's slot order (the returned rows); h bf16 [T, d]. Uses the slot table of the
+ *   handle's last dsmoe_ep_route (T must match, else DSMOE_ERR_INVALID_ARG).
+ * The three calls use the handle's workspace (dsmoe_ep_experts overwrites the expert
+ * offsets and the A1 rows); a handle serves one rank, one layer call at a time.
+ */
+dsmoe_status dsmoe_ep_route(dsmoe_handle* h, int32_t T, const void* x, const int32_t* token_ids,
+                            const void* W_router, const float* b, int32_t* topk_idx, float* gates,
+                            int32_t* counts, float* f, float* P, float* P_sum, float* scores_dbg, int32_t world,
+                            int32_t* send_rows, void* stream);
+dsmoe_status dsmoe_ep_experts(dsmoe_handle* h, int32_t n_src, int32_t e_begin, int32_t e_end,
+                              const int32_t* recv_counts, int64_t n_rows, const void* rows, const void* W_gate,
+                              const void* W_up, const void* W_down, void* Y, void* stream);
+dsmoe_status dsmoe_ep_combine(dsmoe_handle* h, int32_t T, const void* x, const void* Ws_gate, const void* Ws_up,
+                              const void* Ws_down, const float* gates, const void* Y, void* h_out, void* stream);
+
+/*
+ * First steps of the backward pass, for an upstream gradient dh = dL/dh of the layer
+ * output h_t = u_t + sum_shared FFN(u_t) + sum_k g_{t,k} y_{t,k} (DeepSeekMoE summary,
+ * shared-expert layer equation), the top-K' selection held fixed (its indicator has no
+ * gradient).
+ *
+ * dsmoe_backward_gates -- uses the expert outputs y and the slot table of this handle's
+ *   last forward (call it after that forward, on the same stream, with the same T):
+ *     dh     bf16 [T, d]        upstream gradient (device, 16-byte aligned)
+ *     gates  fp32 [T, K']       the forward's gates
+ *     dg     fp32 [T, K'] out   dg_{t,k} = <dh_t, y_{t,k}>, fp32 accumulation of bf16 terms
+ *     dY     bf16 [T K', d] out the routed experts' output gradient g_{t,k} dh_t, in the
+ *                               forward's slot order (expert-contiguous; workspace "slot_of"
+ *                               maps (t, k) to its row)
+ *   Under an expert range, picks of experts outside it get dg = 0 and no dY row.
+ *
+ * dsmoe_backward_router -- the router's backward with the expert-level balance term
+ *   alpha sum_i f_i P_i (same page, "Expert-level balance loss": P_i carries the
+ *   gradient to the router, f_i is a constant). Not for hash routing (UNSUPPORTED).
+ *     x, W_router        the forward's bf16 inputs
+ *     topk_idx, gates    the forward's picks and gates [T, K']
+ *     scores             fp32 [T, N'], the forward's raw scores (its scores_dbg output)
+ *     dg                 fp32 [T, K'] from dsmoe_backward_gates
+ *     f, alpha           the balance term's f_i [N'] and factor (f may be NULL iff alpha = 0)
+ *     dlogits fp32 [T, N'] out  dL/dl: ds = alpha f_i / T + the gate terms (dg at the kept
+ *                               experts, or (dg_k - sum_j dg_j g_j) / sum_kept s when the
+ *                               gates are renormalised), then the score function's
+ *                               derivative (softmax, sigmoid, or sqrt(softplus), whose slope
+ *                               sigma(l) / (2 s) uses sigma(l) = 1 - exp(-s^2))
+ *     dx      fp32 [T, d] out   dlogits W_router (the router's part of dL/du)
+ *     dW_router fp32 [N', d] out dlogits^T x
+ *   All sums run in a fixed order (deterministic).
+ */
+dsmoe_status dsmoe_backward_gates(dsmoe_handle* h, int32_t T, const void* dh, const float* gates, float* dg,
+                                  void* dY, void* stream);
+dsmoe_status dsmoe_backward_router(dsmoe_handle* h, int32_t T, const void* x, const void* W_router,
+                                   const int32_t* topk_idx, const float* gates, const float* scores,
+                                   const float* dg, const float* f, float alpha, float* dlogits, float* dx,
+                                   float* dW_router, void* stream);
+
 /* Per-stage timing: while enabled, each forward with T > 0 records CUDA events on its
  * stream at every stage boundary (no synchronisation). dsmoe_stage_times waits for
  * the recorded events and writes, per stage, the mean duration in ms over the last

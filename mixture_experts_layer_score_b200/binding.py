@@ -30,7 +30,8 @@ ABI_FUNCTIONS = (
     "dsmoe_balance_losses", "dsmoe_sequence_balance", "dsmoe_bias_update",
     "dsmoe_route_noalloc", "dsmoe_set_gemm_kernel", "dsmoe_get_gemm_kernel",
     "dsmoe_set_selection", "dsmoe_get_selection", "dsmoe_set_expert_range", "dsmoe_get_expert_range",
-    "dsmoe_round_bf16",
+    "dsmoe_round_bf16", "dsmoe_backward_gates", "dsmoe_backward_router", "dsmoe_ep_route", "dsmoe_ep_experts",
+    "dsmoe_ep_combine",
 )
 
 
@@ -87,6 +88,12 @@ def _load():
         "dsmoe_get_expert_range": (ctypes.c_int, [vp, ctypes.POINTER(i32), ctypes.POINTER(i32),
                                                   ctypes.POINTER(i32)]),
         "dsmoe_round_bf16": (ctypes.c_int, [vp, i64, vp, vp, vp]),
+        "dsmoe_backward_gates": (ctypes.c_int, [vp, i32, vp, vp, vp, vp, vp]),
+        "dsmoe_ep_route": (ctypes.c_int, [vp, i32] + [vp] * 11 + [i32, vp, vp]),
+        "dsmoe_ep_experts": (ctypes.c_int, [vp, i32, i32, i32, vp, i64, vp, vp, vp, vp, vp, vp]),
+        "dsmoe_ep_combine": (ctypes.c_int, [vp, i32] + [vp] * 7 + [vp]),
+        "dsmoe_backward_router": (ctypes.c_int, [vp, i32, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp,
+                                                 vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -230,6 +237,37 @@ def dsmoe_get_expert_range(handle):
 
 def dsmoe_round_bf16(handle, n: int, src, dst, stream=None) -> None:
     _check(_lib.dsmoe_round_bf16(handle, int(n), _ptr(src), _ptr(dst), _stream(stream)), "dsmoe_round_bf16")
+
+
+def dsmoe_ep_route(handle, T, x, token_ids, W_router, b, topk_idx, gates, counts, f, P, P_sum, scores_dbg, world,
+                   send_rows, stream=None) -> None:
+    _check(_lib.dsmoe_ep_route(handle, int(T), *[_ptr(t) for t in (
+        x, token_ids, W_router, b, topk_idx, gates, counts, f, P, P_sum, scores_dbg)], int(world), _ptr(send_rows),
+        _stream(stream)), "dsmoe_ep_route")
+
+
+def dsmoe_ep_experts(handle, n_src, e_begin, e_end, recv_counts, n_rows, rows, W_gate, W_up, W_down, Y,
+                     stream=None) -> None:
+    _check(_lib.dsmoe_ep_experts(handle, int(n_src), int(e_begin), int(e_end), _ptr(recv_counts), int(n_rows),
+                                 *[_ptr(t) for t in (rows, W_gate, W_up, W_down, Y)], _stream(stream)),
+           "dsmoe_ep_experts")
+
+
+def dsmoe_ep_combine(handle, T, x, Ws_gate, Ws_up, Ws_down, gates, Y, h, stream=None) -> None:
+    _check(_lib.dsmoe_ep_combine(handle, int(T), *[_ptr(t) for t in (x, Ws_gate, Ws_up, Ws_down, gates, Y, h)],
+                                 _stream(stream)), "dsmoe_ep_combine")
+
+
+def dsmoe_backward_gates(handle, T, dh, gates, dg, dY, stream=None) -> None:
+    _check(_lib.dsmoe_backward_gates(handle, int(T), _ptr(dh), _ptr(gates), _ptr(dg), _ptr(dY), _stream(stream)),
+           "dsmoe_backward_gates")
+
+
+def dsmoe_backward_router(handle, T, x, W_router, topk_idx, gates, scores, dg, f, alpha, dlogits, dx, dW_router,
+                          stream=None) -> None:
+    _check(_lib.dsmoe_backward_router(handle, int(T), *[_ptr(t) for t in (
+        x, W_router, topk_idx, gates, scores, dg, f)], float(alpha), _ptr(dlogits), _ptr(dx), _ptr(dW_router),
+        _stream(stream)), "dsmoe_backward_router")
 
 
 def dsmoe_set_timing(handle, enable: bool) -> None:

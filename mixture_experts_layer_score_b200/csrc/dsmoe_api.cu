@@ -13,6 +13,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <functional>
 #include <mutex>
 #include <string>
 
@@ -32,6 +33,7 @@ constexpr int kSelectMaxBlocks = 1024;  // rows of the statistics partials
 constexpr int kTimingSlots = 64;        // forwards whose stage events are kept
 constexpr int kTcRouterMinTokens = 256; // below this the CUDA-core router spreads over more SMs
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+constexpr int kEpMaxGroups = 512;       // (source rank, local expert) groups of dsmoe_ep_experts
 
 thread_local std::string g_last_error;
 
@@ -130,7 +132,7 @@ Layout plan(const dsmoe_cfg& c) {
   L.logits = take(hash ? 0 : logit_floats * 4);
   L.counts_ws = take(N * 4);
   L.cursor = take(N * 4);
-  L.offsets = take((N + 1) * 4);
+  L.offsets = take((std::max<size_t>(N, kEpMaxGroups) + 1) * 4);  // also the expert-parallel groups
   L.P_part = take(hash ? 0 : static_cast<size_t>(kSelectMaxBlocks) * N * 4);
   L.slot_of = take(S * 4);
   L.Xp = take(S * d * 2);
@@ -196,6 +198,7 @@ struct dsmoe_handle {
   // for the one-CTA GEMM and the router, then the six expert weights for the pair GEMM
   static constexpr int kMaps = 13;
   const void* wkey[kMaps] = {};
+  int wkey_n[kMaps] = {};  // experts each cached routed map spans
   CUtensorMap tm_w[kMaps];
   int rt_chunks = 1, rt_nc = 16;
   uint32_t rt_cols = 32;
@@ -203,6 +206,7 @@ struct dsmoe_handle {
   int timed_forwards = 0;               // forwards recorded since timing was enabled
   cudaEvent_t ev[kTimingSlots][kNumStages + 1] = {};
   int64_t launches = 0;
+  int32_t ep_T = -1;  // tokens of the last dsmoe_ep_route (its slot table is in the workspace)
 };
 
 // ========================================================================================
@@ -388,6 +392,23 @@ struct FwdArgs {
   float *f, *P, *P_sum, *scores_dbg;
 };
 
+// The routing half's arguments (router inputs and routing outputs).
+dsmoe_status check_route(dsmoe_handle* h, const FwdArgs& a) {
+  const dsmoe_cfg& c = h->cfg;
+  if (a.T < 0) return fail(DSMOE_ERR_INVALID_ARG, "T = %d is negative", a.T);
+  if (a.T > c.max_tokens) return fail(DSMOE_ERR_WORKSPACE, "T = %d exceeds max_tokens = %d", a.T, c.max_tokens);
+  if (!a.counts || !a.f || !a.P) return fail(DSMOE_ERR_INVALID_ARG, "counts, f and P are required");
+  if (a.T == 0) return DSMOE_OK;
+  const bool hash = c.score == DSMOE_ROUTE_HASH;
+  if (!a.x || !a.topk_idx || !a.gates) return fail(DSMOE_ERR_INVALID_ARG, "x, topk_idx and gates are required");
+  if (hash && !a.token_ids) return fail(DSMOE_ERR_INVALID_ARG, "hash routing needs token_ids");
+  if (!hash && !a.W_router) return fail(DSMOE_ERR_INVALID_ARG, "W_router is required");
+  if (c.bias_mode != DSMOE_BIAS_NONE && !a.b) return fail(DSMOE_ERR_INVALID_ARG, "bias b is required by bias_mode");
+  if (!aligned16(a.x) || (a.W_router && !aligned16(a.W_router)))
+    return fail(DSMOE_ERR_INVALID_ARG, "x and W_router must be 16-byte aligned");
+  return DSMOE_OK;
+}
+
 dsmoe_status check_forward(dsmoe_handle* h, const FwdArgs& a) {
   const dsmoe_cfg& c = h->cfg;
   if (a.T < 0) return fail(DSMOE_ERR_INVALID_ARG, "T = %d is negative", a.T);
@@ -408,12 +429,13 @@ dsmoe_status check_forward(dsmoe_handle* h, const FwdArgs& a) {
   return DSMOE_OK;
 }
 
-// Tensor maps of the weights, cached per pointer (the routed maps span the handle's
-// expert range; dsmoe_set_expert_range clears the cache).
-const CUtensorMap* weight_map(dsmoe_handle* h, int which, const void* ptr, bool* ok) {
-  if (h->wkey[which] != ptr) {
+// Tensor maps of the weights, cached per pointer and expert count. The routed maps
+// (0-2, 7-9) span n_local experts: the handle's expert range unless the caller says.
+const CUtensorMap* weight_map(dsmoe_handle* h, int which, const void* ptr, bool* ok, int n_local = -1) {
+  if (n_local < 0) n_local = h->e_end - h->e_begin;
+  if (h->wkey[which] != ptr || h->wkey_n[which] != n_local) {
     const dsmoe_cfg& c = h->cfg;
-    const int n_local = h->e_end - h->e_begin;
+    h->wkey_n[which] = n_local;
     bool r = false;
     switch (which) {
       case 0:
@@ -444,105 +466,92 @@ const CUtensorMap* weight_map(dsmoe_handle* h, int which, const void* ptr, bool*
 
 int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
-dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
+// ---- stages of the forward, shared by dsmoe_forward and the expert-parallel entry points
+
+// Router affinities, scores, top-K', gates and statistics partials (or hash routing) for
+// a.T > 0 tokens. Writes the routing outputs and h->counts_ws; *sel_grid = rows of score
+// partials (0 for hash routing).
+dsmoe_status route_stage(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s, int* sel_grid,
+                         const std::function<cudaError_t(int)>& mark) {
   const dsmoe_cfg& c = h->cfg;
-  const int T = a.T, N = c.n_routed, K = h->k_active, d = c.d_model, F = c.d_ff;
-  // shared experts (and the residual) only where this handle adds them
-  const int Ks = h->add_shared ? c.n_shared : 0, Fs = c.d_ff_shared;
-  const int e0 = h->e_begin, NL = h->e_end - h->e_begin;  // routed experts applied here
+  const int T = a.T, N = c.n_routed, K = h->k_active, d = c.d_model;
   const bool hash = c.score == DSMOE_ROUTE_HASH;
-  const bool timing = h->timing && T > 0;
-  cudaEvent_t* evs = h->ev[h->timed_forwards % kTimingSlots];
-  auto mark = [&](int i) -> cudaError_t { return timing ? cudaEventRecord(evs[i], s) : cudaSuccess; };
-
-  if (T == 0) {
-    CUDA_TRY(cudaMemsetAsync(a.counts, 0, N * sizeof(int32_t), s));
-    CUDA_TRY(cudaMemsetAsync(a.f, 0, N * sizeof(float), s));
-    CUDA_TRY(cudaMemsetAsync(a.P, 0, N * sizeof(float), s));
-    if (a.P_sum) CUDA_TRY(cudaMemsetAsync(a.P_sum, 0, N * sizeof(float), s));
-    return DSMOE_OK;
-  }
-
-  // tensor maps that depend on the call's pointers
   bool ok = true;
-  const bool pair = h->gemm_kernel == DSMOE_GEMM_PAIR;
-  const int wm = pair ? 7 : 0;  // first weight map of the chosen GEMM kernel
-  const CUtensorMap* m_wg = weight_map(h, wm + 0, a.W_gate, &ok);
-  const CUtensorMap* m_wu = weight_map(h, wm + 1, a.W_up, &ok);
-  const CUtensorMap* m_wd = weight_map(h, wm + 2, a.W_down, &ok);
-  const CUtensorMap* m_swg = Ks ? weight_map(h, wm + 3, a.Ws_gate, &ok) : m_wg;
-  const CUtensorMap* m_swu = Ks ? weight_map(h, wm + 4, a.Ws_up, &ok) : m_wu;
-  const CUtensorMap* m_swd = Ks ? weight_map(h, wm + 5, a.Ws_down, &ok) : m_wd;
-  CUtensorMap m_x, m_x_router;  // token rows of x: GEMM tiles, and the router's 128-token tiles
-  ok = ok && map_2d(&m_x, a.x, d, T, dsmoe::kGemmGateUpTokenTile) && map_2d(&m_x_router, a.x, d, T, 128);
-  if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map of this call");
-
-  CUDA_TRY(mark(0));
   CUDA_TRY(cudaMemsetAsync(h->counts_ws, 0, N * sizeof(int32_t), s));
-  int sel_grid = 0;
+  *sel_grid = 0;
   if (hash) {
     CUDA_TRY(dsmoe::launch_hash_route(a.token_ids, T, N, c.hash_mult, c.hash_mod, a.topk_idx, a.gates, h->counts_ws,
                                       h->status, s));
     h->launches += 1;
     CUDA_TRY(mark(1));
-  } else {
-    // router affinities as split-K partial sums: tensor cores for larger batches,
-    // CUDA cores below kTcRouterMinTokens tokens; then scores, top-K', gates, partials
-    int splits;
-    if (T >= kTcRouterMinTokens) {
-      dsmoe::RouterTcArgs ra;
-      memset(&ra, 0, sizeof(ra));
-      const CUtensorMap* m_wr = weight_map(h, 6, a.W_router, &ok);
-      if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected the router tensor map");
-      splits = dsmoe::router_tc_splits(T, d, h->num_sms);
-      ra.tm_x = m_x_router;
-      ra.tm_w = *m_wr;
-      ra.T = T;
-      ra.N = N;
-      ra.d = d;
-      ra.splits = splits;
-      ra.n_chunks = h->rt_chunks;
-      ra.nc = h->rt_nc;
-      ra.tmem_cols = h->rt_cols;
-      ra.partial = h->logits;
-      ra.status = h->status;
-      ra.wait_limit_ns = h->wait_ns;
-      const int work = cdiv(T, 128) * splits;
-      CUDA_TRY(dsmoe::launch_router_tc(ra, work < h->num_sms ? work : h->num_sms, s));
-    } else {
-      splits = dsmoe::router_logits_splits(T, N, d, h->num_sms);
-      CUDA_TRY(dsmoe::launch_router_logits(static_cast<const bf16*>(a.x), static_cast<const bf16*>(a.W_router), T,
-                                           N, d, splits, h->logits, s));
-    }
-    CUDA_TRY(mark(1));
-    dsmoe::SelectArgs sa;
-    sa.logits = h->logits;
-    sa.splits = splits;
-    sa.b = a.b;
-    sa.T = T;
-    sa.N = N;
-    sa.K = K;
-    sa.mask_top = h->mask_top;
-    sa.score = c.score;
-    sa.bias_select = c.bias_mode == DSMOE_BIAS_SELECT_ONLY;
-    sa.bias_in_logits = c.bias_mode == DSMOE_BIAS_IN_LOGITS;
-    sa.renormalize = c.renormalize;
-    sa.topk_idx = a.topk_idx;
-    sa.gates = a.gates;
-    sa.counts = h->counts_ws;
-    sa.P_part = h->P_part;
-    sa.scores_dbg = a.scores_dbg;
-    sa.status = h->status;
-    // two blocks per SM: enough warps for the tokens, few partial rows for the scan
-    sel_grid = dsmoe::select_grid(T, h->num_sms / 2 > 0 ? h->num_sms / 2 : 1);
-    CUDA_TRY(dsmoe::launch_select(sa, sel_grid, s));
-    h->launches += 2;
+    return DSMOE_OK;
   }
-  CUDA_TRY(mark(2));
+  // router affinities as split-K partial sums: tensor cores for larger batches,
+  // CUDA cores below kTcRouterMinTokens tokens; then scores, top-K', gates, partials
+  int splits;
+  if (T >= kTcRouterMinTokens) {
+    CUtensorMap m_x_router;  // token rows of x in the router's 128-token tiles
+    if (!map_2d(&m_x_router, a.x, d, T, 128))
+      return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected the router's token map");
+    dsmoe::RouterTcArgs ra;
+    memset(&ra, 0, sizeof(ra));
+    const CUtensorMap* m_wr = weight_map(h, 6, a.W_router, &ok);
+    if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected the router tensor map");
+    splits = dsmoe::router_tc_splits(T, d, h->num_sms);
+    ra.tm_x = m_x_router;
+    ra.tm_w = *m_wr;
+    ra.T = T;
+    ra.N = N;
+    ra.d = d;
+    ra.splits = splits;
+    ra.n_chunks = h->rt_chunks;
+    ra.nc = h->rt_nc;
+    ra.tmem_cols = h->rt_cols;
+    ra.partial = h->logits;
+    ra.status = h->status;
+    ra.wait_limit_ns = h->wait_ns;
+    const int work = cdiv(T, 128) * splits;
+    CUDA_TRY(dsmoe::launch_router_tc(ra, work < h->num_sms ? work : h->num_sms, s));
+  } else {
+    splits = dsmoe::router_logits_splits(T, N, d, h->num_sms);
+    CUDA_TRY(dsmoe::launch_router_logits(static_cast<const bf16*>(a.x), static_cast<const bf16*>(a.W_router), T, N,
+                                         d, splits, h->logits, s));
+  }
+  CUDA_TRY(mark(1));
+  dsmoe::SelectArgs sa;
+  sa.logits = h->logits;
+  sa.splits = splits;
+  sa.b = a.b;
+  sa.T = T;
+  sa.N = N;
+  sa.K = K;
+  sa.mask_top = h->mask_top;
+  sa.score = c.score;
+  sa.bias_select = c.bias_mode == DSMOE_BIAS_SELECT_ONLY;
+  sa.bias_in_logits = c.bias_mode == DSMOE_BIAS_IN_LOGITS;
+  sa.renormalize = c.renormalize;
+  sa.topk_idx = a.topk_idx;
+  sa.gates = a.gates;
+  sa.counts = h->counts_ws;
+  sa.P_part = h->P_part;
+  sa.scores_dbg = a.scores_dbg;
+  sa.status = h->status;
+  // two blocks per SM: enough warps for the tokens, few partial rows for the scan
+  *sel_grid = dsmoe::select_grid(T, h->num_sms / 2 > 0 ? h->num_sms / 2 : 1);
+  CUDA_TRY(dsmoe::launch_select(sa, *sel_grid, s));
+  h->launches += 2;
+  return DSMOE_OK;
+}
 
+// Counts, f, P (and P_sum), the slot offsets of the experts in [e0, e1), and the
+// permutation + gather of the token rows into h->Xp.
+dsmoe_status scan_permute_stage(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s, int sel_grid, int e0, int e1,
+                                const std::function<cudaError_t(int)>& mark) {
+  const dsmoe_cfg& c = h->cfg;
+  const int T = a.T, N = c.n_routed, K = h->k_active, d = c.d_model;
   dsmoe::ScanArgs sc;
   sc.counts_ws = h->counts_ws;
-  sc.P_part = hash ? nullptr : h->P_part;
+  sc.P_part = c.score == DSMOE_ROUTE_HASH ? nullptr : h->P_part;
   sc.n_part = sel_grid;
   sc.N = N;
   sc.K = K;
@@ -554,32 +563,53 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
   sc.offsets = h->offsets;
   sc.cursor = h->cursor;
   sc.e_begin = e0;
-  sc.e_end = e0 + NL;
+  sc.e_end = e1;
   CUDA_TRY(dsmoe::launch_scan_stats(sc, s));
   h->launches += 1;
   CUDA_TRY(mark(3));
-
   CUDA_TRY(dsmoe::launch_permute_gather(static_cast<const bf16*>(a.x), a.topk_idx, h->offsets, h->cursor, T, K, N,
-                                        e0, e0 + NL, d, h->slot_of, h->Xp, h->status, h->num_sms, s));
+                                        e0, e1, d, h->slot_of, h->Xp, h->status, h->num_sms, s));
   h->launches += 1;
-  CUDA_TRY(mark(4));
+  return DSMOE_OK;
+}
 
-  const int64_t S = static_cast<int64_t>(T) * K;
+// The grouped GEMMs of one projection pair over `n_groups` routed groups (device offsets
+// [n_groups + 1], rows of `rows_map`, weights expert_mod-mapped) and Ks shared experts on
+// the T token rows of `x_map` (gate/up) / h->A1s (down). Gate/up writes A1 (routed) and
+// A1s (shared); down writes Y_out (routed) and Hs = residual + shared outputs (fp32).
+struct GemmPlan {
+  const CUtensorMap* rows_map;      // routed token rows (Xp or received rows), gate/up A operand
+  const CUtensorMap* x_map;         // x rows of the shared groups
+  const int32_t* offsets;
+  int n_groups, expert_mod;
+  int64_t routed_rows;              // rows the routed groups cover (tile bound)
+  int T, Ks;
+  const CUtensorMap *wg, *wu, *wd, *swg, *swu, *swd;
+  const bf16* residual;             // x, added to the shared rows of the down GEMM
+  bf16* Y_out;                      // [routed_rows, d] routed expert outputs
+};
+
+dsmoe_status gemm_stage(dsmoe_handle* h, const GemmPlan& p, cudaStream_t s,
+                        const std::function<cudaError_t(int)>& mark) {
+  const dsmoe_cfg& c = h->cfg;
+  const int d = c.d_model, F = c.d_ff, Fs = c.d_ff_shared, Ks = p.Ks, T = p.T;
+  const bool pair = h->gemm_kernel == DSMOE_GEMM_PAIR;
   // ---- gate/up GEMM with SiLU(gate) * up
   {
     dsmoe::GemmArgs g;
     memset(&g, 0, sizeof(g));
-    g.a_routed = h->tm_xp;
-    g.a_shared = m_x;
-    g.b0_routed = *m_wg;
-    g.b1_routed = *m_wu;
-    g.b0_shared = *m_swg;
-    g.b1_shared = *m_swu;
-    g.offsets = h->offsets + e0;
-    g.n_routed = NL;
+    g.a_routed = *p.rows_map;
+    g.a_shared = *p.x_map;
+    g.b0_routed = *p.wg;
+    g.b1_routed = *p.wu;
+    g.b0_shared = *p.swg;
+    g.b1_shared = *p.swu;
+    g.offsets = p.offsets;
+    g.n_routed = p.n_groups;
+    g.expert_mod = p.expert_mod;
     g.n_shared_groups = Ks;
     g.m_shared = T;
-    g.n_tiles_routed = cdiv(F, 128);
+    g.n_tiles_routed = p.n_groups ? cdiv(F, 128) : 0;
     g.n_tiles_shared = Ks ? cdiv(Fs, 128) : 0;
     g.kb_routed = d / 64;
     g.kb_shared = d / 64;
@@ -594,16 +624,18 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
     g.status = h->status;
     g.wait_limit_ns = h->wait_ns;
     const int64_t tt = pair ? dsmoe::kGemmPairTokenTile : dsmoe::kGemmGateUpTokenTile;
-    const int64_t bound = (cdiv(S, tt) + NL) * static_cast<int64_t>(g.n_tiles_routed) +
+    const int64_t bound = (cdiv(p.routed_rows, tt) + p.n_groups) * static_cast<int64_t>(g.n_tiles_routed) +
                           static_cast<int64_t>(Ks) * cdiv(T, tt) * g.n_tiles_shared;
-    if (pair) {
-      const int clusters = static_cast<int>(bound < h->pair_clusters[1] ? bound : h->pair_clusters[1]);
-      CUDA_TRY(dsmoe::launch_grouped_gemm_pair(true, g, clusters, s));
-    } else {
-      const int grid = static_cast<int>(bound < h->num_sms ? bound : h->num_sms);
-      CUDA_TRY(dsmoe::launch_grouped_gemm(true, g, grid, s));
+    if (bound > 0) {
+      if (pair) {
+        const int clusters = static_cast<int>(bound < h->pair_clusters[1] ? bound : h->pair_clusters[1]);
+        CUDA_TRY(dsmoe::launch_grouped_gemm_pair(true, g, clusters, s));
+      } else {
+        const int grid = static_cast<int>(bound < h->num_sms ? bound : h->num_sms);
+        CUDA_TRY(dsmoe::launch_grouped_gemm(true, g, grid, s));
+      }
+      h->launches += 1;
     }
-    h->launches += 1;
   }
   CUDA_TRY(mark(5));
   // ---- down GEMM; the shared experts accumulate into one output row per token
@@ -612,59 +644,129 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
     memset(&g, 0, sizeof(g));
     g.a_routed = h->tm_a1;
     g.a_shared = h->tm_a1s;
-    g.b0_routed = *m_wd;
-    g.b1_routed = *m_wd;
-    g.b0_shared = *m_swd;
-    g.b1_shared = *m_swd;
-    g.offsets = h->offsets + e0;
-    g.n_routed = NL;
+    g.b0_routed = *p.wd;
+    g.b1_routed = *p.wd;
+    g.b0_shared = *p.swd;
+    g.b1_shared = *p.swd;
+    g.offsets = p.offsets;
+    g.n_routed = p.n_groups;
+    g.expert_mod = p.expert_mod;
     g.n_shared_groups = Ks ? 1 : 0;
     g.m_shared = T;
-    g.n_tiles_routed = cdiv(d, 256);
+    g.n_tiles_routed = p.n_groups ? cdiv(d, 256) : 0;
     g.n_tiles_shared = Ks ? cdiv(d, 256) : 0;
     g.kb_routed = F / 64;
     g.kb_shared = Ks ? Ks * Fs / 64 : 0;
     g.kb_per_b_expert_shared = Ks ? Fs / 64 : 1;
     g.n_valid_routed = d;
     g.n_valid_shared = d;
-    g.out_routed = h->Y;
+    g.out_routed = p.Y_out;
     g.ld_routed = d;
     g.out_shared = nullptr;
     g.out_shared_f32 = h->Hs;
-    g.residual = static_cast<const bf16*>(a.x);
+    g.residual = p.residual;
     g.ld_shared = d;
     g.shared_col_stride = 0;
     g.status = h->status;
     g.wait_limit_ns = h->wait_ns;
     const int64_t tt = pair ? dsmoe::kGemmPairTokenTile : dsmoe::kGemmDownTokenTile;
-    const int64_t bound = (cdiv(S, tt) + NL) * static_cast<int64_t>(g.n_tiles_routed) +
+    const int64_t bound = (cdiv(p.routed_rows, tt) + p.n_groups) * static_cast<int64_t>(g.n_tiles_routed) +
                           static_cast<int64_t>(g.n_shared_groups) * cdiv(T, tt) * g.n_tiles_shared;
-    if (pair) {
-      const int clusters = static_cast<int>(bound < h->pair_clusters[0] ? bound : h->pair_clusters[0]);
-      CUDA_TRY(dsmoe::launch_grouped_gemm_pair(false, g, clusters, s));
-    } else {
-      const int grid = static_cast<int>(bound < h->num_sms ? bound : h->num_sms);
-      CUDA_TRY(dsmoe::launch_grouped_gemm(false, g, grid, s));
+    if (bound > 0) {
+      if (pair) {
+        const int clusters = static_cast<int>(bound < h->pair_clusters[0] ? bound : h->pair_clusters[0]);
+        CUDA_TRY(dsmoe::launch_grouped_gemm_pair(false, g, clusters, s));
+      } else {
+        const int grid = static_cast<int>(bound < h->num_sms ? bound : h->num_sms);
+        CUDA_TRY(dsmoe::launch_grouped_gemm(false, g, grid, s));
+      }
+      h->launches += 1;
     }
-    h->launches += 1;
   }
   CUDA_TRY(mark(6));
-  {
-    dsmoe::CombineArgs ca;
-    ca.x = static_cast<const bf16*>(a.x);
-    ca.Hs = Ks ? h->Hs : nullptr;
-    ca.add_x = h->add_shared ? 1 : 0;
-    ca.Y = h->Y;
-    ca.slot_of = h->slot_of;
-    ca.gates = a.gates;
-    ca.T = T;
-    ca.K = K;
-    ca.d = d;
-    ca.h = h->partial ? nullptr : static_cast<bf16*>(a.h);
-    ca.h32 = h->partial ? static_cast<float*>(a.h) : nullptr;
-    CUDA_TRY(dsmoe::launch_combine(ca, h->num_sms, s));
-  }
+  return DSMOE_OK;
+}
+
+// h = base + sum_k g Y[slot_of], base = Hs (Ks > 0), x (add_x) or 0; bf16 or fp32 out.
+dsmoe_status combine_stage(dsmoe_handle* h, const FwdArgs& a, const bf16* Y, int Ks, bool add_x, bool partial,
+                           cudaStream_t s) {
+  dsmoe::CombineArgs ca;
+  ca.x = static_cast<const bf16*>(a.x);
+  ca.Hs = Ks ? h->Hs : nullptr;
+  ca.add_x = add_x ? 1 : 0;
+  ca.Y = Y;
+  ca.slot_of = h->slot_of;
+  ca.gates = a.gates;
+  ca.T = a.T;
+  ca.K = h->k_active;
+  ca.d = h->cfg.d_model;
+  ca.h = partial ? nullptr : static_cast<bf16*>(a.h);
+  ca.h32 = partial ? static_cast<float*>(a.h) : nullptr;
+  CUDA_TRY(dsmoe::launch_combine(ca, h->num_sms, s));
   h->launches += 1;
+  return DSMOE_OK;
+}
+
+dsmoe_status zero_stats(const FwdArgs& a, int N, cudaStream_t s) {
+  CUDA_TRY(cudaMemsetAsync(a.counts, 0, N * sizeof(int32_t), s));
+  CUDA_TRY(cudaMemsetAsync(a.f, 0, N * sizeof(float), s));
+  CUDA_TRY(cudaMemsetAsync(a.P, 0, N * sizeof(float), s));
+  if (a.P_sum) CUDA_TRY(cudaMemsetAsync(a.P_sum, 0, N * sizeof(float), s));
+  return DSMOE_OK;
+}
+
+#define STAGE_TRY(expr)                        \
+  do {                                         \
+    const dsmoe_status st_ = (expr);           \
+    if (st_ != DSMOE_OK) return st_;           \
+  } while (0)
+
+dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
+  const dsmoe_cfg& c = h->cfg;
+  const int T = a.T, N = c.n_routed, K = h->k_active, d = c.d_model;
+  // shared experts (and the residual) only where this handle adds them
+  const int Ks = h->add_shared ? c.n_shared : 0;
+  const int e0 = h->e_begin, NL = h->e_end - h->e_begin;  // routed experts applied here
+  const bool timing = h->timing && T > 0;
+  cudaEvent_t* evs = h->ev[h->timed_forwards % kTimingSlots];
+  const std::function<cudaError_t(int)> mark = [&](int i) -> cudaError_t {
+    return timing ? cudaEventRecord(evs[i], s) : cudaSuccess;
+  };
+
+  if (T == 0) return zero_stats(a, N, s);
+
+  // tensor maps that depend on the call's pointers
+  bool ok = true;
+  const int wm = h->gemm_kernel == DSMOE_GEMM_PAIR ? 7 : 0;  // first weight map of the chosen GEMM kernel
+  GemmPlan p;
+  p.wg = weight_map(h, wm + 0, a.W_gate, &ok);
+  p.wu = weight_map(h, wm + 1, a.W_up, &ok);
+  p.wd = weight_map(h, wm + 2, a.W_down, &ok);
+  p.swg = Ks ? weight_map(h, wm + 3, a.Ws_gate, &ok) : p.wg;
+  p.swu = Ks ? weight_map(h, wm + 4, a.Ws_up, &ok) : p.wu;
+  p.swd = Ks ? weight_map(h, wm + 5, a.Ws_down, &ok) : p.wd;
+  CUtensorMap m_x;  // token rows of x in GEMM tiles (shared groups)
+  ok = ok && map_2d(&m_x, a.x, d, T, dsmoe::kGemmGateUpTokenTile);
+  if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map of this call");
+
+  CUDA_TRY(mark(0));
+  int sel_grid = 0;
+  STAGE_TRY(route_stage(h, a, s, &sel_grid, mark));
+  CUDA_TRY(mark(2));
+  STAGE_TRY(scan_permute_stage(h, a, s, sel_grid, e0, e0 + NL, mark));
+  CUDA_TRY(mark(4));
+  p.rows_map = &h->tm_xp;
+  p.x_map = &m_x;
+  p.offsets = h->offsets + e0;
+  p.n_groups = NL;
+  p.expert_mod = 0;
+  p.routed_rows = static_cast<int64_t>(T) * K;
+  p.T = T;
+  p.Ks = Ks;
+  p.residual = static_cast<const bf16*>(a.x);
+  p.Y_out = h->Y;
+  STAGE_TRY(gemm_stage(h, p, s, mark));
+  STAGE_TRY(combine_stage(h, a, h->Y, Ks, h->add_shared, h->partial, s));
   CUDA_TRY(mark(7));
   if (timing) h->timed_forwards += 1;
   return DSMOE_OK;
@@ -729,6 +831,143 @@ DSMOE_EXPORT dsmoe_status dsmoe_forward_host(dsmoe_handle* h, int32_t T, const v
   CUDA_TRY(cudaMemcpyAsync(P_host, h->P_stage, nb, cudaMemcpyDeviceToHost, s));
   CUDA_TRY(cudaStreamSynchronize(s));
   return DSMOE_OK;
+}
+
+// ========================================================================================
+// expert parallelism with token dispatch (route -> exchange rows -> owners' experts ->
+// exchange back -> combine); the exchanges are the caller's collectives
+// ========================================================================================
+DSMOE_EXPORT dsmoe_status dsmoe_ep_route(dsmoe_handle* h, int32_t T, const void* x, const int32_t* token_ids,
+                                         const void* W_router, const float* b, int32_t* topk_idx, float* gates,
+                                         int32_t* counts, float* f, float* P, float* P_sum, float* scores_dbg,
+                                         int32_t world, int32_t* send_rows, void* stream) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  const dsmoe_cfg& c = h->cfg;
+  if (world < 1 || world > c.n_routed) return fail(DSMOE_ERR_INVALID_ARG, "world = %d outside [1, N']", world);
+  if (!send_rows) return fail(DSMOE_ERR_INVALID_ARG, "send_rows is required");
+  FwdArgs a{T, x, W_router, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, token_ids, b, nullptr, topk_idx,
+            gates, counts, f, P, P_sum, scores_dbg};
+  const dsmoe_status st = check_route(h, a);
+  if (st != DSMOE_OK) return st;
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const std::function<cudaError_t(int)> mark = [](int) { return cudaSuccess; };
+  if (T == 0) {
+    STAGE_TRY(zero_stats(a, c.n_routed, s));
+    CUDA_TRY(cudaMemsetAsync(send_rows, 0, world * sizeof(int32_t), s));
+    return DSMOE_OK;
+  }
+  int sel_grid = 0;
+  STAGE_TRY(route_stage(h, a, s, &sel_grid, mark));
+  STAGE_TRY(scan_permute_stage(h, a, s, sel_grid, 0, c.n_routed, mark));
+  CUDA_TRY(dsmoe::launch_block_rows(h->offsets, c.n_routed, world, send_rows, s));
+  h->launches += 1;
+  h->ep_T = T;
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_ep_experts(dsmoe_handle* h, int32_t n_src, int32_t e_begin, int32_t e_end,
+                                           const int32_t* recv_counts, int64_t n_rows, const void* rows,
+                                           const void* W_gate, const void* W_up, const void* W_down, void* Y,
+                                           void* stream) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  const dsmoe_cfg& c = h->cfg;
+  const int n_local = e_end - e_begin;
+  if (e_begin < 0 || n_local < 1 || e_end > c.n_routed)
+    return fail(DSMOE_ERR_INVALID_ARG, "expert block [%d, %d) is not a non-empty part of [0, %d)", e_begin, e_end,
+                c.n_routed);
+  if (n_src < 1 || static_cast<int64_t>(n_src) * n_local > kEpMaxGroups)
+    return fail(DSMOE_ERR_UNSUPPORTED, "n_src * local experts = %lld outside [1, %d]",
+                static_cast<long long>(n_src) * n_local, kEpMaxGroups);
+  if (n_rows < 0 || n_rows > static_cast<int64_t>(c.max_tokens) * c.top_k)
+    return fail(DSMOE_ERR_WORKSPACE, "n_rows = %lld outside [0, max_tokens * top_k = %lld]",
+                static_cast<long long>(n_rows), static_cast<long long>(c.max_tokens) * c.top_k);
+  if (!recv_counts || (n_rows > 0 && (!rows || !W_gate || !W_up || !W_down || !Y)))
+    return fail(DSMOE_ERR_INVALID_ARG, "NULL argument");
+  const void* must_align[] = {rows, W_gate, W_up, W_down, Y};
+  for (const void* p : must_align)
+    if (p && !aligned16(p)) return fail(DSMOE_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", p);
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (n_rows == 0) return DSMOE_OK;
+  const int groups = n_src * n_local;
+  CUDA_TRY(dsmoe::launch_group_offsets(recv_counts, groups, h->offsets, h->status, s));
+  h->launches += 1;
+  bool ok = true;
+  const int wm = h->gemm_kernel == DSMOE_GEMM_PAIR ? 7 : 0;
+  GemmPlan p;
+  p.wg = weight_map(h, wm + 0, W_gate, &ok, n_local);
+  p.wu = weight_map(h, wm + 1, W_up, &ok, n_local);
+  p.wd = weight_map(h, wm + 2, W_down, &ok, n_local);
+  p.swg = p.wg;
+  p.swu = p.wu;
+  p.swd = p.wd;
+  CUtensorMap m_rows;
+  const uint32_t box = h->gemm_kernel == DSMOE_GEMM_PAIR ? 128 : dsmoe::kGemmGateUpTokenTile;
+  ok = ok && map_2d(&m_rows, rows, c.d_model, static_cast<uint64_t>(n_rows), box);
+  if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map of this call");
+  p.rows_map = &m_rows;
+  p.x_map = &m_rows;
+  p.offsets = h->offsets;
+  p.n_groups = groups;
+  p.expert_mod = n_local;
+  p.routed_rows = n_rows;
+  p.T = 0;
+  p.Ks = 0;
+  p.residual = nullptr;
+  p.Y_out = static_cast<bf16*>(Y);
+  const std::function<cudaError_t(int)> mark = [](int) { return cudaSuccess; };
+  return gemm_stage(h, p, s, mark);
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_ep_combine(dsmoe_handle* h, int32_t T, const void* x, const void* Ws_gate,
+                                           const void* Ws_up, const void* Ws_down, const float* gates, const void* Y,
+                                           void* h_out, void* stream) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  const dsmoe_cfg& c = h->cfg;
+  if (T != h->ep_T) return fail(DSMOE_ERR_INVALID_ARG, "T = %d differs from the last dsmoe_ep_route (%d)", T, h->ep_T);
+  if (T == 0) return DSMOE_OK;
+  if (!x || !gates || !Y || !h_out) return fail(DSMOE_ERR_INVALID_ARG, "NULL argument");
+  const int Ks = c.n_shared;
+  if (Ks > 0 && (!Ws_gate || !Ws_up || !Ws_down))
+    return fail(DSMOE_ERR_INVALID_ARG, "shared expert weights are required (n_shared = %d)", Ks);
+  const void* must_align[] = {x, Ws_gate, Ws_up, Ws_down, Y, h_out};
+  for (const void* p : must_align)
+    if (p && !aligned16(p)) return fail(DSMOE_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", p);
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const std::function<cudaError_t(int)> mark = [](int) { return cudaSuccess; };
+  if (Ks > 0) {
+    bool ok = true;
+    const int wm = h->gemm_kernel == DSMOE_GEMM_PAIR ? 7 : 0;
+    GemmPlan p;
+    p.swg = weight_map(h, wm + 3, Ws_gate, &ok);
+    p.swu = weight_map(h, wm + 4, Ws_up, &ok);
+    p.swd = weight_map(h, wm + 5, Ws_down, &ok);
+    p.wg = p.swg;
+    p.wu = p.swu;
+    p.wd = p.swd;
+    CUtensorMap m_x;
+    ok = ok && map_2d(&m_x, x, c.d_model, T, dsmoe::kGemmGateUpTokenTile);
+    if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map of this call");
+    p.rows_map = &m_x;
+    p.x_map = &m_x;
+    p.offsets = h->offsets;
+    p.n_groups = 0;
+    p.expert_mod = 0;
+    p.routed_rows = 0;
+    p.T = T;
+    p.Ks = Ks;
+    p.residual = static_cast<const bf16*>(x);
+    p.Y_out = nullptr;
+    STAGE_TRY(gemm_stage(h, p, s, mark));
+  }
+  FwdArgs a{T, x, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, h_out, nullptr,
+            const_cast<float*>(gates), nullptr, nullptr, nullptr, nullptr, nullptr};
+  return combine_stage(h, a, static_cast<const bf16*>(Y), Ks, true, false, s);
 }
 
 DSMOE_EXPORT dsmoe_status dsmoe_balance_stats(dsmoe_handle* h, int64_t T_total, const int32_t* counts,
@@ -811,8 +1050,6 @@ DSMOE_EXPORT dsmoe_status dsmoe_set_expert_range(dsmoe_handle* h, int32_t e_begi
   if (!partial && (e_begin != 0 || e_end != c.n_routed || !add_shared))
     return fail(DSMOE_ERR_INVALID_ARG, "a part of the layer (an expert sub-range, or no residual and shared "
                 "experts) needs DSMOE_RANGE_PARTIAL: its output is an fp32 partial sum");
-  if (e_begin != h->e_begin || e_end != h->e_end)
-    for (int i = 0; i < dsmoe_handle::kMaps; ++i) h->wkey[i] = nullptr;  // routed maps span the range
   h->e_begin = e_begin;
   h->e_end = e_end;
   h->partial = partial;
@@ -838,6 +1075,94 @@ DSMOE_EXPORT dsmoe_status dsmoe_round_bf16(dsmoe_handle* h, int64_t n, const flo
   if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
   CUDA_TRY(dsmoe::launch_round_bf16(src, static_cast<bf16*>(dst), n, h->num_sms, static_cast<cudaStream_t>(stream)));
   if (n > 0) h->launches += 1;
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_backward_gates(dsmoe_handle* h, int32_t T, const void* dh, const float* gates,
+                                               float* dg, void* dY, void* stream) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  if (T < 0 || T > h->cfg.max_tokens) return fail(DSMOE_ERR_INVALID_ARG, "T = %d outside [0, max_tokens]", T);
+  if (T == 0) return DSMOE_OK;
+  if (!dh || !gates || !dg || !dY) return fail(DSMOE_ERR_INVALID_ARG, "NULL argument");
+  if (!aligned16(dh) || !aligned16(dY)) return fail(DSMOE_ERR_INVALID_ARG, "dh and dY must be 16-byte aligned");
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
+  dsmoe::GateGradArgs a;
+  a.dh = static_cast<const bf16*>(dh);
+  a.Y = h->Y;
+  a.slot_of = h->slot_of;
+  a.gates = gates;
+  a.T = T;
+  a.K = h->k_active;
+  a.d = h->cfg.d_model;
+  a.dg = dg;
+  a.dY = static_cast<bf16*>(dY);
+  CUDA_TRY(dsmoe::launch_gate_grad(a, h->num_sms, static_cast<cudaStream_t>(stream)));
+  h->launches += 1;
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_backward_router(dsmoe_handle* h, int32_t T, const void* x, const void* W_router,
+                                                const int32_t* topk_idx, const float* gates, const float* scores,
+                                                const float* dg, const float* f, float alpha, float* dlogits,
+                                                float* dx, float* dW_router, void* stream) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  const dsmoe_cfg& c = h->cfg;
+  if (c.score == DSMOE_ROUTE_HASH) return fail(DSMOE_ERR_UNSUPPORTED, "hash routing has no router to differentiate");
+  if (T < 0 || T > c.max_tokens) return fail(DSMOE_ERR_INVALID_ARG, "T = %d outside [0, max_tokens]", T);
+  if (!dW_router) return fail(DSMOE_ERR_INVALID_ARG, "dW_router is required");
+  if (T > 0 && (!x || !W_router || !topk_idx || !gates || !scores || !dg || !dlogits || !dx))
+    return fail(DSMOE_ERR_INVALID_ARG, "NULL argument");
+  if (alpha != 0.f && !f) return fail(DSMOE_ERR_INVALID_ARG, "a balance term (alpha != 0) needs f");
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int N = c.n_routed, d = c.d_model;
+  if (T == 0) {
+    CUDA_TRY(cudaMemsetAsync(dW_router, 0, static_cast<size_t>(N) * d * sizeof(float), st));
+    return DSMOE_OK;
+  }
+  dsmoe::RouterBwdArgs r;
+  r.scores = scores;
+  r.topk_idx = topk_idx;
+  r.gates = gates;
+  r.dg = dg;
+  r.f = alpha != 0.f ? f : nullptr;
+  r.alpha = alpha;
+  r.T = T;
+  r.N = N;
+  r.K = h->k_active;
+  r.score = c.score;
+  r.renormalize = c.renormalize;
+  r.dlogits = dlogits;
+  r.status = h->status;
+  CUDA_TRY(dsmoe::launch_router_backward(r, h->num_sms, st));
+  // dx = dlogits W_router  (M = T, K = N', N = d)
+  dsmoe::GemmF32Args a;
+  a.A = dlogits;
+  a.a_sm = N;
+  a.a_sk = 1;
+  a.B = static_cast<const bf16*>(W_router);
+  a.ldb = d;
+  a.C = dx;
+  a.ldc = d;
+  a.M = T;
+  a.N = d;
+  a.K = N;
+  CUDA_TRY(dsmoe::launch_gemm_f32_bf16(a, st));
+  // dW_router = dlogits^T x  (M = N', K = T, N = d)
+  a.A = dlogits;
+  a.a_sm = 1;
+  a.a_sk = N;
+  a.B = static_cast<const bf16*>(x);
+  a.ldb = d;
+  a.C = dW_router;
+  a.ldc = d;
+  a.M = N;
+  a.N = d;
+  a.K = T;
+  CUDA_TRY(dsmoe::launch_gemm_f32_bf16(a, st));
+  h->launches += 3;
   return DSMOE_OK;
 }
 

@@ -1,8 +1,9 @@
 // grouped_tiles.cuh -- the tile schedule shared by the grouped-GEMM kernels.
 //
 // Groups are the shared experts (dense, m_shared rows each) followed by the routed
-// experts (their segments of the expert-contiguous slot order, from the device-side
-// offsets). A group of M rows has ceil(M / kTok) token tiles times n_tiles output tiles;
+// groups (segments of the expert-contiguous slot order, from the device-side offsets).
+// A routed group is one expert, or, with expert_mod = n > 0, group g applies expert
+// g mod n (rows received from several ranks, grouped by source and then by expert). A group of M rows has ceil(M / kTok) token tiles times n_tiles output tiles;
 // tiles are numbered group by group, token tiles fastest, so that the CTAs working at
 // the same time share each weight tile through L2. The per-group prefix lives in shared
 // memory and is built by every CTA from the offsets (no host synchronisation).
@@ -76,9 +77,10 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int32_t* ti
     t.kb_n = a.kb_shared;
   } else {
     t.shared = 0;
-    t.expert = lo - a.n_shared_groups;
-    base = a.offsets[t.expert];
-    M = a.offsets[t.expert + 1] - base;
+    const int gi = lo - a.n_shared_groups;  // routed group: its segment of the offsets
+    t.expert = a.expert_mod > 0 ? gi % a.expert_mod : gi;  // its weights
+    base = a.offsets[gi];
+    M = a.offsets[gi + 1] - base;
     t.kb_n = a.kb_routed;
   }
   const int mt = (M + kTok - 1) / kTok;

@@ -100,6 +100,14 @@ cudaError_t launch_permute_gather(const bf16* x, const int32_t* topk_idx, const 
                                   int32_t* cursor, int T, int K, int N, int e_begin, int e_end, int d,
                                   int32_t* slot_of, bf16* Xp, uint32_t* status, int num_sms, cudaStream_t s);
 
+// Expert parallelism. block_rows: out[j] = rows of the slot order that fall in rank j's
+// contiguous block of experts (blocks of N / world, the first N % world one larger).
+// group_offsets: offsets[0..groups] = exclusive scan of counts[groups] (negative counts
+// are recorded in the status word and taken as 0).
+cudaError_t launch_block_rows(const int32_t* offsets, int N, int world, int32_t* out, cudaStream_t s);
+cudaError_t launch_group_offsets(const int32_t* counts, int groups, int32_t* offsets, uint32_t* status,
+                                 cudaStream_t s);
+
 // ---------------------------------------------------------------- balance control (balance.cu)
 cudaError_t launch_balance_losses(const float* f, const float* P, int N, int G, const int32_t* group_of,
                                   float alpha1, float alpha2, float* f_dev, float* P_dev, float* losses,
@@ -129,6 +137,46 @@ cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s);
 // dst[i] = bf16(src[i]) (round to nearest even), n a multiple of 8, both 16-byte aligned.
 cudaError_t launch_round_bf16(const float* src, bf16* dst, int64_t n, int num_sms, cudaStream_t s);
 
+// ---------------------------------------------------------------- backward (backward.cu)
+// dg[t,k] = <dh_t, Y[slot_of[t,k]]> and dY[slot_of[t,k]] = bf16(gates[t,k] dh_t).
+struct GateGradArgs {
+  const bf16* dh;          // [T, d]
+  const bf16* Y;           // [slots, d] the forward's expert outputs in slot order
+  const int32_t* slot_of;  // [T, K]
+  const float* gates;      // [T, K]
+  int T, K, d;
+  float* dg;               // [T, K]
+  bf16* dY;                // [slots, d]
+};
+cudaError_t launch_gate_grad(const GateGradArgs& a, int num_sms, cudaStream_t s);
+
+// dlogits [T, N] from the forward's scores, picks and gates, dg, and the balance term
+// alpha f_i / T (f may be null: no balance term).
+struct RouterBwdArgs {
+  const float* scores;     // [T, N]
+  const int32_t* topk_idx; // [T, K]
+  const float* gates;      // [T, K]
+  const float* dg;         // [T, K]
+  const float* f;          // [N] or nullptr
+  float alpha;
+  int T, N, K, score, renormalize;
+  float* dlogits;          // [T, N]
+  uint32_t* status;
+};
+cudaError_t launch_router_backward(const RouterBwdArgs& a, int num_sms, cudaStream_t s);
+
+// C[M, N] = A(M x K, fp32, element (m, k) at A[m a_sm + k a_sk]) * B (bf16 [K, ldb]), fp32 out.
+struct GemmF32Args {
+  const float* A;
+  int64_t a_sm, a_sk;
+  const bf16* B;
+  int64_t ldb;
+  float* C;
+  int64_t ldc;
+  int M, N, K;
+};
+cudaError_t launch_gemm_f32_bf16(const GemmF32Args& a, cudaStream_t s);
+
 // ---------------------------------------------------------------- grouped GEMM (gemm_sm100.cu)
 // Tokens per grouped-GEMM tile of each projection (the row box of its token-side
 // tensor maps).
@@ -142,8 +190,9 @@ struct GemmArgs {
   CUtensorMap b1_routed;  // 3D up-projection weights (SwiGLU only)
   CUtensorMap b0_shared;
   CUtensorMap b1_shared;
-  const int32_t* offsets;         // [n_routed + 1] slot offset of each routed expert
+  const int32_t* offsets;         // [n_routed + 1] slot offset of each routed group
   int32_t n_routed;               // routed groups
+  int32_t expert_mod;             // 0: routed group g is expert g; n > 0: expert g mod n
   int32_t n_shared_groups;        // shared groups (tiles run before the routed ones)
   int32_t m_shared;               // rows of every shared group (T)
   int32_t n_tiles_routed, n_tiles_shared;  // output tiles along N

@@ -111,7 +111,60 @@ __global__ void __launch_bounds__(256) permute_gather_kernel(const bf16* __restr
     }
   }
 }
+__global__ void block_rows_kernel(const int32_t* __restrict__ offsets, int N, int world, int32_t* __restrict__ out) {
+  for (int j = threadIdx.x; j < world; j += blockDim.x) {
+    const int base = N / world, extra = N % world;
+    const int e0 = j * base + min(j, extra), e1 = e0 + base + (j < extra ? 1 : 0);
+    out[j] = offsets[e1] - offsets[e0];
+  }
+}
+
+// One block of kScanThreads threads: an exclusive scan of up to kScanThreads counts.
+__global__ void __launch_bounds__(kScanThreads) group_offsets_kernel(const int32_t* __restrict__ counts, int groups,
+                                                                      int32_t* __restrict__ offsets,
+                                                                      uint32_t* status) {
+  __shared__ int32_t warp_tot[kScanThreads / 32];
+  const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
+  int32_t c = (i < groups) ? counts[i] : 0;
+  if (c < 0) {
+    atomicOr(status, kStatusBadIndex);
+    c = 0;
+  }
+  int32_t v = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) warp_tot[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t w = (lane < kScanThreads / 32) ? warp_tot[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t n = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += n;
+    }
+    if (lane < kScanThreads / 32) warp_tot[lane] = w;
+  }
+  __syncthreads();
+  const int32_t incl = v + (warp > 0 ? warp_tot[warp - 1] : 0);
+  if (i < groups) offsets[i] = incl - c;
+  if (i == groups - 1) offsets[groups] = incl;
+}
 }  // namespace
+
+cudaError_t launch_block_rows(const int32_t* offsets, int N, int world, int32_t* out, cudaStream_t s) {
+  block_rows_kernel<<<1, 256, 0, s>>>(offsets, N, world, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_group_offsets(const int32_t* counts, int groups, int32_t* offsets, uint32_t* status,
+                                 cudaStream_t s) {
+  if (groups < 1 || groups > kScanThreads) return cudaErrorInvalidValue;
+  group_offsets_kernel<<<1, kScanThreads, 0, s>>>(counts, groups, offsets, status);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_scan_stats(const ScanArgs& a, cudaStream_t s) {
   scan_stats_kernel<<<1, kScanThreads, 0, s>>>(a);

@@ -94,3 +94,62 @@ def expert_sharded_forward(layer, x_local: torch.Tensor, token_ids_local: torch.
     rows = slice(rank * T, (rank + 1) * T)
     return dict(h=h, topk_idx=out["topk_idx"][rows], gates=out["gates"][rows], counts=out["counts"], f=out["f"],
                 P=out["P"])
+
+
+def token_dispatch_forward(layer, x_local: torch.Tensor, token_ids_local: torch.Tensor = None, group=None,
+                           stream=None, lib=None):
+    """The layer on this rank's tokens in the token-dispatch expert-parallel form (the
+    "MoE: sparse activation" page's training-cost section: tokens travel by all-to-all to
+    the GPUs that hold their experts; the interview card's deployment trade-off: routed
+    experts sharded, shared experts replicated).
+
+    layer: binding.DSMoE whose W_gate / W_up / W_down hold this rank's contiguous block of
+    routed experts (expert_block) and whose router and shared experts are full copies;
+    its handle's max_tokens must cover the rows this rank may receive (world * T at
+    most). Steps: dsmoe_ep_route (route, gather the rows into expert order, which is
+    destination order) -> all-to-all of the per-expert counts, then of the rows ->
+    dsmoe_ep_experts (this rank's experts on what it received) -> all-to-all back ->
+    dsmoe_ep_combine (shared experts, gate-weighted sum, residual). Returns h (bf16) and
+    this rank's routing; counts, f and P are this rank's tokens' statistics (reduce them
+    with global_balance_stats for the whole batch).
+
+    lib: the object providing the library calls (the binding module by default)."""
+    if lib is None:
+        from . import binding as lib
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    cfg = layer.cfg
+    T, d = x_local.shape
+    N = cfg.n_routed
+    dev = x_local.device
+    K = layer.k_active
+    out = layer.alloc_outputs(T)
+    send_rows = torch.empty((world,), dtype=torch.int32, device=dev)
+    w = layer.w
+    lib.dsmoe_ep_route(layer.handle, T, x_local, token_ids_local, w.get("W_router"), w.get("b"), out["topk_idx"],
+                       out["gates"], out["counts"], out["f"], out["P"], out["P_sum"], None, world, send_rows, stream)
+    # per-expert counts to each expert's owner
+    blocks = [expert_block(N, j, world) for j in range(world)]
+    e0, e1 = blocks[rank]
+    n_local = e1 - e0
+    recv_counts = torch.empty((world * n_local,), dtype=torch.int32, device=dev)
+    dist.all_to_all_single(recv_counts, out["counts"], output_split_sizes=[n_local] * world,
+                           input_split_sizes=[b - a for a, b in blocks], group=group)
+    # the row exchange needs its split sizes on the host
+    send_splits = [int(v) for v in send_rows.cpu().tolist()]
+    per_src = recv_counts.view(world, n_local).cpu().numpy().sum(axis=1)
+    recv_splits = [int(v) for v in per_src]
+    xp = lib.workspace_view(layer.handle, "Xp", layer.device)[:T * K]
+    rows = torch.empty((sum(recv_splits), d), dtype=torch.bfloat16, device=dev)
+    dist.all_to_all_single(rows, xp, output_split_sizes=recv_splits, input_split_sizes=send_splits, group=group)
+    y_rows = torch.empty_like(rows)
+    lib.dsmoe_ep_experts(layer.handle, world, e0, e1, recv_counts, rows.shape[0], rows, w["W_gate"], w["W_up"],
+                         w["W_down"], y_rows, stream)
+    y_back = torch.empty((T * K, d), dtype=torch.bfloat16, device=dev)
+    dist.all_to_all_single(y_back, y_rows, output_split_sizes=send_splits, input_split_sizes=recv_splits,
+                           group=group)
+    h = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+    lib.dsmoe_ep_combine(layer.handle, T, x_local, w.get("Ws_gate"), w.get("Ws_up"), w.get("Ws_down"), out["gates"],
+                         y_back, h, stream)
+    out["h"] = h
+    return out

@@ -133,14 +133,12 @@ def layer_backward(cfg, inputs: Dict, dh, routing: Optional[Dict] = None, alpha_
         out["dWs_gate"][i], out["dWs_up"][i], out["dWs_down"][i] = dWg, dWu, dWd
 
     # routed experts: the rows that kept each expert, output gradient g * dh; the gate
-    # gradient dg = <dh, FFN(u)> on the same rows
-    dg = np.zeros_like(gates)
+    # gradient dg = <dh, FFN(u)> on the same rows (gate_grads)
+    dg = gate_grads(inputs, idx, dh)
     for e in np.unique(idx):
         rows, ks = np.nonzero(idx == e)
         U = X[rows]
         Wg, Wu, Wd = inputs["W_gate"][e], inputs["W_up"][e], inputs["W_down"][e]
-        y = O.swiglu_ffn(U, Wg, Wu, Wd)
-        dg[rows, ks] = (dh[rows] * y).sum(axis=1)
         dU, dWg, dWu, dWd = swiglu_backward(U, Wg, Wu, Wd, gates[rows, ks][:, None] * dh[rows])
         np.add.at(dx, rows, dU)
         out["dW_gate"][e], out["dW_up"][e], out["dW_down"][e] = dWg, dWu, dWd
@@ -149,13 +147,37 @@ def layer_backward(cfg, inputs: Dict, dh, routing: Optional[Dict] = None, alpha_
         out.update(dx=dx, dW_router=None, dg=dg, dlogits=None)
         return out
 
-    # router: gates and the balance term reach the scores, then the logits
-    s = np.asarray(r["scores"], dtype=np.float64)
-    ds = gate_backward(s, idx, gates, dg, cfg.renormalize)
-    if alpha_bal:
-        ds += alpha_bal * np.asarray(r["f"], dtype=np.float64)[None, :] / T
-    dl = score_backward(r["logits"], s, ds, cfg.score)
-    W_r = O._as_f64(inputs["W_router"])
-    dx += dl @ W_r
-    out.update(dx=dx, dW_router=dl.T @ X, dg=dg, dlogits=dl)
+    dl, dx_router, dW_router = router_grads(cfg, r, inputs["x"], inputs["W_router"], dg, alpha_bal)
+    dx += dx_router
+    out.update(dx=dx, dW_router=dW_router, dg=dg, dlogits=dl)
     return out
+
+
+def gate_grads(inputs: Dict, idx, dh) -> np.ndarray:
+    """dg_{t,k} = <dh_t, FFN_{e(t,k)}(u_t)> [T, K'] for the picks idx, each expert
+    evaluated on the rows that kept it (inputs as for dsmoe_oracle.forward)."""
+    X = O._as_f64(inputs["x"])
+    dh = np.asarray(dh, dtype=np.float64)
+    idx = np.asarray(idx, dtype=np.int64)
+    dg = np.zeros(idx.shape)
+    for e in np.unique(idx):
+        rows, ks = np.nonzero(idx == e)
+        y = O.swiglu_ffn(X[rows], inputs["W_gate"][e], inputs["W_up"][e], inputs["W_down"][e])
+        dg[rows, ks] = (dh[rows] * y).sum(axis=1)
+    return dg
+
+
+def router_grads(cfg, routing: Dict, x, W_router, dg, alpha_bal: float = 0.0):
+    """The router's backward: the gate gradients dg and the balance term reach the scores
+    (gate_backward, plus alpha f_i / T), then the logits (score_backward), then
+    du = dl W_router and dW_router = dl^T u. Returns (dlogits, du, dW_router)."""
+    X = O._as_f64(x)
+    T = X.shape[0]
+    idx = np.asarray(routing["idx"], dtype=np.int64)
+    s = np.asarray(routing["scores"], dtype=np.float64)
+    ds = gate_backward(s, idx, routing["gates"], dg, cfg.renormalize)
+    if alpha_bal:
+        ds += alpha_bal * np.asarray(routing["f"], dtype=np.float64)[None, :] / T
+    dl = score_backward(routing["logits"], s, ds, cfg.score)
+    W_r = O._as_f64(W_router)
+    return dl, dl @ W_r, dl.T @ X

@@ -1,0 +1,106 @@
+"""The first backward kernels against the float64 backward oracle (oracle/dsmoe_backward.py,
+pinned there by finite differences, float64 autograd and closed forms): for an upstream
+gradient dh, the gate gradients dg = <dh, y>, the routed experts' output gradient
+g dh in slot order, and the router's backward with the expert-level balance term
+(DeepSeekMoE summary, "Expert-level balance loss": P_i carries the gradient).
+
+Bounds (max |err| / RMS(ref)):
+* dg against the oracle: 1e-2 (the kernel dots dh with the forward's bf16 expert rows,
+  the oracle with the exact float64 FFN outputs);
+* dlogits, dx and dW_router against the oracle fed the kernel's own dg: 1e-4 (fp32
+  arithmetic on fp32 scores); dlogits against the oracle end to end: 2e-2;
+* dY rows equal bf16(g * dh) exactly (one fp32 product, rounded to nearest even)."""
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_layer_score_b200 as M
+import workloads as W
+from oracle import dsmoe_backward as DB
+from tests import parity as PAR
+from tests.gpu_cases import make_case
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("no GPU", allow_module_level=True)
+
+# (workload, T, alpha of the balance term, mask_top, k_active or None)
+CASES = [("tiny", 300, 0.01, 0, None), ("gshard_b", 1000, 0.01, 0, None), ("v3_prefill", 300, 0.003, 0, None),
+         ("v4_decode_t64", 64, 0.0, 0, None), ("ds2b", 700, 0.01, 0, None), ("gshard_c", 500, 0.02, 2, 5)]
+
+
+def _rel(got, ref):
+    return float(np.abs(np.asarray(got, dtype=np.float64) - ref).max() / max(np.sqrt(np.mean(ref ** 2)), 1e-30))
+
+
+@pytest.mark.parametrize("name,T,alpha,mask,k", CASES, ids=[f"{c[0]}-T{c[1]}" + (f"-m{c[3]}k{c[4]}" if c[3] else "")
+                                                           for c in CASES])
+def test_gate_and_router_backward(name, T, alpha, mask, k):
+    cfg = W.get_config(name)
+    gpu, cpu = make_case(cfg, T)
+    dh = W.normal_bf16((T, cfg.d_model), 1.0, 0, "dh", 0, "cuda")
+    layer = M.DSMoE(M.cfg_from(cfg, T), gpu)
+    try:
+        if mask or k:
+            layer.set_selection(mask, k or cfg.top_k)
+        K = layer.k_active
+        out = layer.forward(gpu["x"], with_scores=True)
+        dg = torch.empty((T, K), dtype=torch.float32, device="cuda")
+        dY = torch.empty((T * K, cfg.d_model), dtype=torch.bfloat16, device="cuda")
+        M.dsmoe_backward_gates(layer.handle, T, dh, out["gates"], dg, dY)
+        slot = M.workspace_view(layer.handle, "slot_of")[:T, :K].clone()
+        dl = torch.empty((T, cfg.n_routed), dtype=torch.float32, device="cuda")
+        dx = torch.empty((T, cfg.d_model), dtype=torch.float32, device="cuda")
+        dWr = torch.empty((cfg.n_routed, cfg.d_model), dtype=torch.float32, device="cuda")
+        M.dsmoe_backward_router(layer.handle, T, gpu["x"], gpu["W_router"], out["topk_idx"], out["gates"],
+                                out["scores"], dg, out["f"], alpha, dl, dx, dWr)
+        torch.cuda.synchronize()
+        assert M.dsmoe_get_status(layer.handle) == M.DSMOE_OK, M.dsmoe_last_error()
+    finally:
+        layer.close()
+    cfg_v = cfg.replace(top_k=K, mask_top=mask)
+    ref = PAR.reference_selection(cfg_v, cpu, out["topk_idx"], out["scores"])
+    PAR.check_routing(cfg_v, ref, out, T)
+    # dY: g * dh in the slot of each pick, exactly
+    want = (out["gates"][:, :, None] * dh.float()[:, None, :]).to(torch.bfloat16)
+    got = dY[slot.view(-1).long()].view(T, K, cfg.d_model)
+    assert torch.equal(got, want)
+    dh64 = dh.float().cpu().numpy().astype(np.float64)
+    # dg against the oracle (exact float64 expert outputs)
+    dg_ref = DB.gate_grads(cpu, ref["idx"], dh64)
+    e_dg = _rel(dg.cpu().numpy(), dg_ref)
+    # the router's backward fed the kernel's own dg, and end to end
+    routing = dict(ref, f=out["f"].cpu().numpy().astype(np.float64))
+    dl_k, dx_k, dW_k = DB.router_grads(cfg_v, routing, cpu["x"], cpu["W_router"], dg.cpu().numpy().astype(np.float64),
+                                       alpha)
+    e_dl = _rel(dl.cpu().numpy(), dl_k)
+    dl64 = dl.cpu().numpy().astype(np.float64)
+    x64 = cpu["x"].float().numpy().astype(np.float64)
+    Wr64 = cpu["W_router"].float().numpy().astype(np.float64)
+    e_dx = _rel(dx.cpu().numpy(), dl64 @ Wr64)
+    e_dW = _rel(dWr.cpu().numpy(), dl64.T @ x64)
+    dl_ref, _, _ = DB.router_grads(cfg_v, routing, cpu["x"], cpu["W_router"], dg_ref, alpha)
+    e_dl_e2e = _rel(dl.cpu().numpy(), dl_ref)
+    for k_ in ("W_gate", "W_up", "W_down"):
+        if hasattr(cpu[k_], "cache"):
+            cpu[k_].cache.clear()
+    print(name, T, dict(dg=e_dg, dl=e_dl, dx=e_dx, dW=e_dW, dl_e2e=e_dl_e2e))
+    assert e_dg <= 1e-2 and e_dl_e2e <= 2e-2
+    assert e_dl <= 1e-4 and e_dx <= 1e-4 and e_dW <= 1e-4
+
+
+def test_backward_argument_errors():
+    cfg = W.get_config("v4_hash_t16")
+    gpu, _ = make_case(cfg, 16)
+    layer = M.DSMoE(M.cfg_from(cfg, 16), gpu)
+    try:
+        with pytest.raises(M.DsmoeError) as ei:
+            M.dsmoe_backward_router(layer.handle, 16, gpu["x"], None, None, None, None, None, None, 0.0, None, None,
+                                    torch.empty(1, device="cuda"))
+        assert ei.value.status == M.DSMOE_ERR_UNSUPPORTED
+        with pytest.raises(M.DsmoeError) as ei:
+            M.dsmoe_backward_gates(layer.handle, 17, None, None, None, None)
+        assert ei.value.status == M.DSMOE_ERR_INVALID_ARG
+    finally:
+        layer.close()
