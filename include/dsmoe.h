@@ -175,6 +175,27 @@ dsmoe_status dsmoe_forward_host(dsmoe_handle* h, int32_t T,
                                 void* stream);
 
 /*
+ * The host forward pipelined for serving loops: the same arguments and results as
+ * dsmoe_forward_host, but the call only enqueues work and returns. Input copies and
+ * output copies run on a copy stream the handle owns, the forward on `stream`, through
+ * two staging slots used in turn, so the copies of one call overlap the forward of the
+ * next or previous one. The caller must keep each call's host buffers alive and
+ * untouched until that call has finished: dsmoe_host_sync blocks until every enqueued
+ * host call is done; dsmoe_host_join makes `stream` wait for them without blocking the
+ * host. All host entry points of a handle share its workspace: issue them from one host
+ * thread with one `stream`.
+ */
+dsmoe_status dsmoe_forward_host_async(dsmoe_handle* h, int32_t T,
+                                      const void* x_host, const int32_t* token_ids_host,
+                                      const void* W_router, const float* b,
+                                      const void* W_gate, const void* W_up, const void* W_down,
+                                      const void* Ws_gate, const void* Ws_up, const void* Ws_down,
+                                      void* h_host, int32_t* topk_idx_host, float* gates_host,
+                                      int32_t* counts_host, float* f_host, float* P_host, void* stream);
+dsmoe_status dsmoe_host_join(dsmoe_handle* h, void* stream);
+dsmoe_status dsmoe_host_sync(dsmoe_handle* h);
+
+/*
  * Expert-level balance statistics from token counts and score sums gathered
  * over T_total tokens (e.g. summed across token shards on several GPUs):
  * f_i = N' / (K' T_total) * counts_i and P_i = P_sum_i / T_total

@@ -31,7 +31,7 @@ ABI_FUNCTIONS = (
     "dsmoe_route_noalloc", "dsmoe_set_gemm_kernel", "dsmoe_get_gemm_kernel",
     "dsmoe_set_selection", "dsmoe_get_selection", "dsmoe_set_expert_range", "dsmoe_get_expert_range",
     "dsmoe_round_bf16", "dsmoe_backward_gates", "dsmoe_backward_router", "dsmoe_ep_route", "dsmoe_ep_experts",
-    "dsmoe_ep_combine",
+    "dsmoe_ep_combine", "dsmoe_forward_host_async", "dsmoe_host_join", "dsmoe_host_sync",
 )
 
 
@@ -66,6 +66,9 @@ def _load():
         "dsmoe_destroy": (None, [vp]),
         "dsmoe_forward": (ctypes.c_int, [vp, i32] + [vp] * 18 + [vp]),
         "dsmoe_forward_host": (ctypes.c_int, [vp, i32] + [vp] * 16 + [vp]),
+        "dsmoe_forward_host_async": (ctypes.c_int, [vp, i32] + [vp] * 16 + [vp]),
+        "dsmoe_host_join": (ctypes.c_int, [vp, vp]),
+        "dsmoe_host_sync": (ctypes.c_int, [vp]),
         "dsmoe_balance_stats": (ctypes.c_int, [vp, i64, vp, vp, vp, vp, vp]),
         "dsmoe_get_status": (ctypes.c_int, [vp]),
         "dsmoe_set_wait_limit": (ctypes.c_int, [vp, u64]),
@@ -191,6 +194,23 @@ def dsmoe_forward_host(handle, T, x_host, token_ids_host, W_router, b, W_gate, W
         x_host, token_ids_host, W_router, b, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, h_host,
         topk_idx_host, gates_host, counts_host, f_host, P_host)], _stream(stream))
     _check(st, "dsmoe_forward_host")
+
+
+def dsmoe_forward_host_async(handle, T, x_host, token_ids_host, W_router, b, W_gate, W_up, W_down, Ws_gate, Ws_up,
+                             Ws_down, h_host, topk_idx_host, gates_host, counts_host, f_host, P_host,
+                             stream=None) -> None:
+    st = _lib.dsmoe_forward_host_async(handle, int(T), *[_ptr(t) for t in (
+        x_host, token_ids_host, W_router, b, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, h_host,
+        topk_idx_host, gates_host, counts_host, f_host, P_host)], _stream(stream))
+    _check(st, "dsmoe_forward_host_async")
+
+
+def dsmoe_host_join(handle, stream=None) -> None:
+    _check(_lib.dsmoe_host_join(handle, _stream(stream)), "dsmoe_host_join")
+
+
+def dsmoe_host_sync(handle) -> None:
+    _check(_lib.dsmoe_host_sync(handle), "dsmoe_host_sync")
 
 
 def dsmoe_balance_stats(handle, T_total, counts, P_sum, f, P, stream=None) -> None:

@@ -106,7 +106,8 @@ struct DeviceGuard {
 
 struct Layout {
   size_t logits, counts_ws, cursor, offsets, P_part, slot_of, Xp, A1, A1s, Y, Hs, status, seq_terms;
-  size_t x_stage, ids_stage, h_stage, topk_stage, gates_stage, counts_stage, f_stage, P_stage;
+  size_t x_stage[2], ids_stage[2], h_stage[2], topk_stage[2], gates_stage[2], counts_stage[2], f_stage[2],
+      P_stage[2];  // two staging slots for the host entry points
   size_t total;
 };
 
@@ -142,14 +143,16 @@ Layout plan(const dsmoe_cfg& c) {
   L.Hs = take(c.n_shared > 0 ? T * d * 4 : 0);
   L.status = take(4);
   L.seq_terms = take(T * 4);
-  L.x_stage = take(T * d * 2);
-  L.ids_stage = take(hash ? T * 4 : 0);
-  L.h_stage = take(T * d * 2);
-  L.topk_stage = take(S * 4);
-  L.gates_stage = take(S * 4);
-  L.counts_stage = take(N * 4);
-  L.f_stage = take(N * 4);
-  L.P_stage = take(N * 4);
+  for (int i = 0; i < 2; ++i) {
+    L.x_stage[i] = take(T * d * 2);
+    L.ids_stage[i] = take(hash ? T * 4 : 0);
+    L.h_stage[i] = take(T * d * 2);
+    L.topk_stage[i] = take(S * 4);
+    L.gates_stage[i] = take(S * 4);
+    L.counts_stage[i] = take(N * 4);
+    L.f_stage[i] = take(N * 4);
+    L.P_stage[i] = take(N * 4);
+  }
   L.total = off;
   return L;
 }
@@ -190,9 +193,16 @@ struct dsmoe_handle {
   float* Hs;
   uint32_t* status;
   float* seq_terms;
-  bf16 *x_stage, *h_stage;
-  int32_t *ids_stage, *topk_stage, *counts_stage;
-  float *gates_stage, *f_stage, *P_stage;
+  struct Stage {
+    bf16 *x, *h;
+    int32_t *ids, *topk, *counts;
+    float *gates, *f, *P;
+  } stage[2];
+  // the pipelined host entry point: its copy stream and, per staging slot, the events
+  // that order input copy -> forward -> output copy -> reuse of the slot
+  cudaStream_t copy_stream = nullptr;
+  cudaEvent_t ev_in[2] = {}, ev_out[2] = {}, ev_d2h[2] = {};
+  int64_t async_calls = 0;
   CUtensorMap tm_xp, tm_a1, tm_a1s;
   // weight maps, cached per pointer: W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, W_router
   // for the one-CTA GEMM and the router, then the six expert weights for the pair GEMM
@@ -276,6 +286,10 @@ static void release(dsmoe_handle* h) {
   for (auto& set : h->ev)
     for (auto& e : set)
       if (e) cudaEventDestroy(e);
+  for (int i = 0; i < 2; ++i)
+    for (cudaEvent_t e : {h->ev_in[i], h->ev_out[i], h->ev_d2h[i]})
+      if (e) cudaEventDestroy(e);
+  if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
   if (h->ws) cudaFree(h->ws);
   delete h;
 }
@@ -329,14 +343,16 @@ DSMOE_EXPORT dsmoe_status dsmoe_create(const dsmoe_cfg* cfg, int32_t device, dsm
   h->Hs = reinterpret_cast<float*>(w + L.Hs);
   h->status = reinterpret_cast<uint32_t*>(w + L.status);
   h->seq_terms = reinterpret_cast<float*>(w + L.seq_terms);
-  h->x_stage = reinterpret_cast<bf16*>(w + L.x_stage);
-  h->ids_stage = reinterpret_cast<int32_t*>(w + L.ids_stage);
-  h->h_stage = reinterpret_cast<bf16*>(w + L.h_stage);
-  h->topk_stage = reinterpret_cast<int32_t*>(w + L.topk_stage);
-  h->gates_stage = reinterpret_cast<float*>(w + L.gates_stage);
-  h->counts_stage = reinterpret_cast<int32_t*>(w + L.counts_stage);
-  h->f_stage = reinterpret_cast<float*>(w + L.f_stage);
-  h->P_stage = reinterpret_cast<float*>(w + L.P_stage);
+  for (int i = 0; i < 2; ++i) {
+    h->stage[i].x = reinterpret_cast<bf16*>(w + L.x_stage[i]);
+    h->stage[i].ids = reinterpret_cast<int32_t*>(w + L.ids_stage[i]);
+    h->stage[i].h = reinterpret_cast<bf16*>(w + L.h_stage[i]);
+    h->stage[i].topk = reinterpret_cast<int32_t*>(w + L.topk_stage[i]);
+    h->stage[i].gates = reinterpret_cast<float*>(w + L.gates_stage[i]);
+    h->stage[i].counts = reinterpret_cast<int32_t*>(w + L.counts_stage[i]);
+    h->stage[i].f = reinterpret_cast<float*>(w + L.f_stage[i]);
+    h->stage[i].P = reinterpret_cast<float*>(w + L.P_stage[i]);
+  }
   e = cudaMemset(h->ws, 0, h->L.total);
   if (e != cudaSuccess) {
     release(h);
@@ -362,6 +378,14 @@ DSMOE_EXPORT dsmoe_status dsmoe_create(const dsmoe_cfg* cfg, int32_t device, dsm
         return fail(DSMOE_ERR_CUDA, "cudaEventCreate failed: %s", cudaGetErrorString(e));
       }
     }
+  for (int i = 0; i < 2 && e == cudaSuccess; ++i)
+    for (cudaEvent_t* ev : {&h->ev_in[i], &h->ev_out[i], &h->ev_d2h[i]})
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking);
+  if (e != cudaSuccess) {
+    release(h);
+    return fail(DSMOE_ERR_CUDA, "event or stream creation failed: %s", cudaGetErrorString(e));
+  }
   *out = h;
   return DSMOE_OK;
 }
@@ -790,6 +814,74 @@ DSMOE_EXPORT dsmoe_status dsmoe_forward(dsmoe_handle* h, int32_t T, const void* 
   return run_forward(h, a, static_cast<cudaStream_t>(stream));
 }
 
+namespace {
+struct HostArgs {
+  int32_t T;
+  const void *x_host, *W_router, *W_gate, *W_up, *W_down, *Ws_gate, *Ws_up, *Ws_down;
+  const int32_t* token_ids_host;
+  const float* b;
+  void* h_host;
+  int32_t* topk_idx_host;
+  float* gates_host;
+  int32_t* counts_host;
+  float *f_host, *P_host;
+};
+
+dsmoe_status check_host(dsmoe_handle* h, const HostArgs& a) {
+  const dsmoe_cfg& c = h->cfg;
+  if (h->partial) return fail(DSMOE_ERR_UNSUPPORTED, "the host entry points run the whole layer only");
+  if (a.T < 0) return fail(DSMOE_ERR_INVALID_ARG, "T = %d is negative", a.T);
+  if (a.T > c.max_tokens) return fail(DSMOE_ERR_WORKSPACE, "T = %d exceeds max_tokens = %d", a.T, c.max_tokens);
+  if (!a.counts_host || !a.f_host || !a.P_host) return fail(DSMOE_ERR_INVALID_ARG, "counts, f and P are required");
+  if (a.T > 0 && (!a.x_host || !a.h_host || !a.topk_idx_host || !a.gates_host))
+    return fail(DSMOE_ERR_INVALID_ARG, "x, h, topk_idx and gates are required");
+  if (a.T > 0 && c.score == DSMOE_ROUTE_HASH && !a.token_ids_host)
+    return fail(DSMOE_ERR_INVALID_ARG, "hash routing needs token_ids");
+  return DSMOE_OK;
+}
+
+// One host forward through staging slot `slot`: input copies on `cin`, the forward on
+// `s`, output copies on `cout` (all three the same stream for the synchronous entry).
+dsmoe_status host_forward(dsmoe_handle* h, const HostArgs& a, int slot, cudaStream_t cin, cudaStream_t s,
+                          cudaStream_t cout, bool pipelined) {
+  const dsmoe_cfg& c = h->cfg;
+  const int T = a.T;
+  const bool hash = c.score == DSMOE_ROUTE_HASH;
+  dsmoe_handle::Stage& st = h->stage[slot];
+  const size_t xb = static_cast<size_t>(T) * c.d_model * 2, sb = static_cast<size_t>(T) * h->k_active * 4,
+               nb = static_cast<size_t>(c.n_routed) * 4;
+  if (T > 0) {
+    CUDA_TRY(cudaMemcpyAsync(st.x, a.x_host, xb, cudaMemcpyHostToDevice, cin));
+    if (hash) CUDA_TRY(cudaMemcpyAsync(st.ids, a.token_ids_host, static_cast<size_t>(T) * 4, cudaMemcpyHostToDevice, cin));
+  }
+  if (pipelined) {
+    CUDA_TRY(cudaEventRecord(h->ev_in[slot], cin));
+    CUDA_TRY(cudaStreamWaitEvent(s, h->ev_in[slot], 0));
+    CUDA_TRY(cudaStreamWaitEvent(s, h->ev_d2h[slot], 0));  // the slot's previous outputs have left
+  }
+  FwdArgs f{T, st.x, a.W_router, a.W_gate, a.W_up, a.W_down, a.Ws_gate, a.Ws_up, a.Ws_down,
+            hash ? st.ids : nullptr, a.b, st.h, st.topk, st.gates, st.counts, st.f, st.P, nullptr, nullptr};
+  dsmoe_status r = check_forward(h, f);
+  if (r != DSMOE_OK) return r;
+  r = run_forward(h, f, s);
+  if (r != DSMOE_OK) return r;
+  if (pipelined) {
+    CUDA_TRY(cudaEventRecord(h->ev_out[slot], s));
+    CUDA_TRY(cudaStreamWaitEvent(cout, h->ev_out[slot], 0));
+  }
+  if (T > 0) {
+    CUDA_TRY(cudaMemcpyAsync(a.h_host, st.h, xb, cudaMemcpyDeviceToHost, cout));
+    CUDA_TRY(cudaMemcpyAsync(a.topk_idx_host, st.topk, sb, cudaMemcpyDeviceToHost, cout));
+    CUDA_TRY(cudaMemcpyAsync(a.gates_host, st.gates, sb, cudaMemcpyDeviceToHost, cout));
+  }
+  CUDA_TRY(cudaMemcpyAsync(a.counts_host, st.counts, nb, cudaMemcpyDeviceToHost, cout));
+  CUDA_TRY(cudaMemcpyAsync(a.f_host, st.f, nb, cudaMemcpyDeviceToHost, cout));
+  CUDA_TRY(cudaMemcpyAsync(a.P_host, st.P, nb, cudaMemcpyDeviceToHost, cout));
+  if (pipelined) CUDA_TRY(cudaEventRecord(h->ev_d2h[slot], cout));
+  return DSMOE_OK;
+}
+}  // namespace
+
 DSMOE_EXPORT dsmoe_status dsmoe_forward_host(dsmoe_handle* h, int32_t T, const void* x_host,
                                              const int32_t* token_ids_host, const void* W_router, const float* b,
                                              const void* W_gate, const void* W_up, const void* W_down,
@@ -797,39 +889,51 @@ DSMOE_EXPORT dsmoe_status dsmoe_forward_host(dsmoe_handle* h, int32_t T, const v
                                              void* h_host, int32_t* topk_idx_host, float* gates_host,
                                              int32_t* counts_host, float* f_host, float* P_host, void* stream) {
   if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
-  const dsmoe_cfg& c = h->cfg;
-  if (h->partial) return fail(DSMOE_ERR_UNSUPPORTED, "the host entry point runs the whole layer only");
-  if (T < 0) return fail(DSMOE_ERR_INVALID_ARG, "T = %d is negative", T);
-  if (T > c.max_tokens) return fail(DSMOE_ERR_WORKSPACE, "T = %d exceeds max_tokens = %d", T, c.max_tokens);
-  if (!counts_host || !f_host || !P_host) return fail(DSMOE_ERR_INVALID_ARG, "counts, f and P are required");
-  if (T > 0 && (!x_host || !h_host || !topk_idx_host || !gates_host))
-    return fail(DSMOE_ERR_INVALID_ARG, "x, h, topk_idx and gates are required");
-  const bool hash = c.score == DSMOE_ROUTE_HASH;
-  if (T > 0 && hash && !token_ids_host) return fail(DSMOE_ERR_INVALID_ARG, "hash routing needs token_ids");
+  HostArgs a{T, x_host, W_router, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, token_ids_host, b, h_host,
+             topk_idx_host, gates_host, counts_host, f_host, P_host};
+  STAGE_TRY(check_host(h, a));
   DeviceGuard g(h->device);
   if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t xb = static_cast<size_t>(T) * c.d_model * 2, sb = static_cast<size_t>(T) * h->k_active * 4,
-               nb = static_cast<size_t>(c.n_routed) * 4;
-  if (T > 0) {
-    CUDA_TRY(cudaMemcpyAsync(h->x_stage, x_host, xb, cudaMemcpyHostToDevice, s));
-    if (hash) CUDA_TRY(cudaMemcpyAsync(h->ids_stage, token_ids_host, static_cast<size_t>(T) * 4, cudaMemcpyHostToDevice, s));
-  }
-  FwdArgs a{T, h->x_stage, W_router, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, hash ? h->ids_stage : nullptr,
-            b, h->h_stage, h->topk_stage, h->gates_stage, h->counts_stage, h->f_stage, h->P_stage, nullptr, nullptr};
-  dsmoe_status st = check_forward(h, a);
-  if (st != DSMOE_OK) return st;
-  st = run_forward(h, a, s);
-  if (st != DSMOE_OK) return st;
-  if (T > 0) {
-    CUDA_TRY(cudaMemcpyAsync(h_host, h->h_stage, xb, cudaMemcpyDeviceToHost, s));
-    CUDA_TRY(cudaMemcpyAsync(topk_idx_host, h->topk_stage, sb, cudaMemcpyDeviceToHost, s));
-    CUDA_TRY(cudaMemcpyAsync(gates_host, h->gates_stage, sb, cudaMemcpyDeviceToHost, s));
-  }
-  CUDA_TRY(cudaMemcpyAsync(counts_host, h->counts_stage, nb, cudaMemcpyDeviceToHost, s));
-  CUDA_TRY(cudaMemcpyAsync(f_host, h->f_stage, nb, cudaMemcpyDeviceToHost, s));
-  CUDA_TRY(cudaMemcpyAsync(P_host, h->P_stage, nb, cudaMemcpyDeviceToHost, s));
+  CUDA_TRY(cudaStreamSynchronize(h->copy_stream));  // no pipelined call still uses the staging
+  STAGE_TRY(host_forward(h, a, 0, s, s, s, false));
   CUDA_TRY(cudaStreamSynchronize(s));
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_forward_host_async(dsmoe_handle* h, int32_t T, const void* x_host,
+                                                   const int32_t* token_ids_host, const void* W_router,
+                                                   const float* b, const void* W_gate, const void* W_up,
+                                                   const void* W_down, const void* Ws_gate, const void* Ws_up,
+                                                   const void* Ws_down, void* h_host, int32_t* topk_idx_host,
+                                                   float* gates_host, int32_t* counts_host, float* f_host,
+                                                   float* P_host, void* stream) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  HostArgs a{T, x_host, W_router, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, token_ids_host, b, h_host,
+             topk_idx_host, gates_host, counts_host, f_host, P_host};
+  STAGE_TRY(check_host(h, a));
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
+  const int slot = static_cast<int>(h->async_calls & 1);
+  STAGE_TRY(host_forward(h, a, slot, h->copy_stream, static_cast<cudaStream_t>(stream), h->copy_stream, true));
+  h->async_calls += 1;
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_host_join(dsmoe_handle* h, void* stream) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (int i = 0; i < 2; ++i) CUDA_TRY(cudaStreamWaitEvent(s, h->ev_d2h[i], 0));
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_host_sync(dsmoe_handle* h) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
+  CUDA_TRY(cudaStreamSynchronize(h->copy_stream));
   return DSMOE_OK;
 }
 

@@ -177,6 +177,19 @@ def test_host_entry_point_matches_device_entry_point():
     assert torch.equal(hh, d["h"].cpu()) and torch.equal(th, d["topk_idx"].cpu())
     assert torch.equal(gh, d["gates"].cpu()) and torch.equal(ch, d["counts"].cpu())
     assert torch.equal(fh, d["f"].cpu()) and torch.equal(ph, d["P"].cpu())
+    # the pipelined entry point: three calls in flight through its two staging slots, with
+    # different inputs, give each call's own results
+    xs = [xh, (gpu["x"] * 0.5).cpu().pin_memory(), (gpu["x"] * 2.0).cpu().pin_memory()]
+    outs = [tuple(torch.empty_like(t).pin_memory() for t in (hh, th, gh, ch, fh, ph)) for _ in xs]
+    for xi, o in zip(xs, outs):
+        M.dsmoe_forward_host_async(layer.handle, T, xi, None, gpu["W_router"], None, gpu["W_gate"], gpu["W_up"],
+                                   gpu["W_down"], gpu["Ws_gate"], gpu["Ws_up"], gpu["Ws_down"], *o)
+    M.dsmoe_host_sync(layer.handle)
+    for xi, o in zip(xs, outs):
+        ref = layer.forward(xi.cuda())
+        torch.cuda.synchronize()
+        for got, k in zip(o, ("h", "topk_idx", "gates", "counts", "f", "P")):
+            assert torch.equal(got, ref[k].cpu()), k
     layer.close()
 
 
