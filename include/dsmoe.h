@@ -385,6 +385,37 @@ dsmoe_status dsmoe_ep_combine(dsmoe_handle* h, int32_t T, const void* x, const v
  */
 dsmoe_status dsmoe_backward_gates(dsmoe_handle* h, int32_t T, const void* dh, const float* gates, float* dg,
                                   void* dY, void* stream);
+
+/*
+ * The experts' part of dL/du (the input gradient through the expert FFNs), for the same
+ * upstream gradient:
+ *   dm = W_down^T dy, da = dm * b * SiLU'(a), db = dm * SiLU(a), du = W_gate^T da + W_up^T db
+ * with SiLU'(a) = sigma(a)(1 + a(1 - sigma(a))), dy = g dh for a routed pick (the dY of
+ * dsmoe_backward_gates) and dy = dh for a shared expert.
+ *
+ * dsmoe_set_training(h, 1) allocates the training buffers (about (4 F + d) T K' bf16 plus
+ * the shared experts' share, sized for max_tokens); from then on every forward of the
+ * handle also stores its pre-activations a = u W_gate^T and b = u W_up^T (bf16). (h, 0)
+ * frees them. Neither is called inside a forward.
+ *
+ * dsmoe_backward_experts -- after a training forward of T tokens on this handle (same T,
+ * else DSMOE_ERR_INVALID_ARG):
+ *     dh        bf16 [T, d]          upstream gradient
+ *     dY        bf16 [T K', d]       the routed experts' output gradients in slot order
+ *                                    (dsmoe_backward_gates)
+ *     W_*, Ws_* the forward's weights (the handle's expert range, as for the forward)
+ *     dx_add    fp32 [T, d] or NULL  added to the result (e.g. dsmoe_backward_router's dx)
+ *     dx        fp32 [T, d] out      dh + sum_shared du + sum_k du_{t,k} (+ dx_add): the
+ *                                    residual, shared-expert and routed-expert parts of dL/du
+ *   Two grouped GEMMs on the tensor cores (the weights read MN-major, in the forward's
+ *   layout) and one combine; fp32 accumulation, da | db and the per-slot du rows stored
+ *   as bf16, the shared experts' du summed in fp32. The weight gradients are not computed
+ *   here.
+ */
+dsmoe_status dsmoe_set_training(dsmoe_handle* h, int32_t enable);
+dsmoe_status dsmoe_backward_experts(dsmoe_handle* h, int32_t T, const void* dh, const void* dY, const void* W_gate,
+                                    const void* W_up, const void* W_down, const void* Ws_gate, const void* Ws_up,
+                                    const void* Ws_down, const float* dx_add, float* dx, void* stream);
 dsmoe_status dsmoe_backward_router(dsmoe_handle* h, int32_t T, const void* x, const void* W_router,
                                    const int32_t* topk_idx, const float* gates, const float* scores,
                                    const float* dg, const float* f, float alpha, float* dlogits, float* dx,
@@ -417,6 +448,13 @@ dsmoe_status dsmoe_launch_count(dsmoe_handle* h, int64_t* n);
  *   "A1s"     bf16 [T, K_s F_s]   the same for the shared experts, side by side
  *   "Y"       bf16 [T K', d]      routed expert outputs per slot
  *   "Hs"      fp32 [T, d]         u_t + sum of the shared experts' outputs
+ *   training buffers (dsmoe_set_training), absent otherwise:
+ *   "AB"      bf16 [T K', 2 F]    a | b pre-activations per slot (last training forward)
+ *   "ABs"     bf16 [T, 2 K_s F_s] a | b of the shared experts, [a_s | b_s] per expert
+ *   "dAB"     bf16 [T K', 2 F]    da | db per slot (last dsmoe_backward_experts)
+ *   "dABs"    bf16 [T, 2 K_s F_s] da | db of the shared experts
+ *   "dXp"     bf16 [T K', d]      du per slot (routed experts)
+ *   "dXs"     fp32 [T, d]         du summed over the shared experts
  * Rows/cols are given for max_tokens; the first T (or T K') rows are meaningful.
  * Returns DSMOE_ERR_INVALID_ARG for an unknown name or a buffer this cfg lacks.
  */

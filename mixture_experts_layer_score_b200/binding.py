@@ -31,7 +31,8 @@ ABI_FUNCTIONS = (
     "dsmoe_route_noalloc", "dsmoe_set_gemm_kernel", "dsmoe_get_gemm_kernel",
     "dsmoe_set_selection", "dsmoe_get_selection", "dsmoe_set_expert_range", "dsmoe_get_expert_range",
     "dsmoe_round_bf16", "dsmoe_backward_gates", "dsmoe_backward_router", "dsmoe_ep_route", "dsmoe_ep_experts",
-    "dsmoe_ep_combine", "dsmoe_forward_host_async", "dsmoe_host_join", "dsmoe_host_sync",
+    "dsmoe_ep_combine", "dsmoe_forward_host_async", "dsmoe_host_join", "dsmoe_host_sync", "dsmoe_set_training",
+    "dsmoe_backward_experts",
 )
 
 
@@ -69,6 +70,8 @@ def _load():
         "dsmoe_forward_host_async": (ctypes.c_int, [vp, i32] + [vp] * 16 + [vp]),
         "dsmoe_host_join": (ctypes.c_int, [vp, vp]),
         "dsmoe_host_sync": (ctypes.c_int, [vp]),
+        "dsmoe_set_training": (ctypes.c_int, [vp, i32]),
+        "dsmoe_backward_experts": (ctypes.c_int, [vp, i32] + [vp] * 10 + [vp]),
         "dsmoe_balance_stats": (ctypes.c_int, [vp, i64, vp, vp, vp, vp, vp]),
         "dsmoe_get_status": (ctypes.c_int, [vp]),
         "dsmoe_set_wait_limit": (ctypes.c_int, [vp, u64]),
@@ -278,6 +281,17 @@ def dsmoe_ep_combine(handle, T, x, Ws_gate, Ws_up, Ws_down, gates, Y, h, stream=
                                  _stream(stream)), "dsmoe_ep_combine")
 
 
+def dsmoe_set_training(handle, enable: bool) -> None:
+    _check(_lib.dsmoe_set_training(handle, int(bool(enable))), "dsmoe_set_training")
+
+
+def dsmoe_backward_experts(handle, T, dh, dY, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, dx_add, dx,
+                           stream=None) -> None:
+    _check(_lib.dsmoe_backward_experts(handle, int(T), *[_ptr(t) for t in (
+        dh, dY, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, dx_add, dx)], _stream(stream)),
+        "dsmoe_backward_experts")
+
+
 def dsmoe_backward_gates(handle, T, dh, gates, dg, dY, stream=None) -> None:
     _check(_lib.dsmoe_backward_gates(handle, int(T), _ptr(dh), _ptr(gates), _ptr(dg), _ptr(dY), _stream(stream)),
            "dsmoe_backward_gates")
@@ -347,7 +361,8 @@ def dsmoe_bias_update(handle, T, counts, alpha, b, stream=None):
 
 
 _WS_DTYPES = {"logits": "float32", "offsets": "int32", "slot_of": "int32", "Xp": "bfloat16",
-              "A1": "bfloat16", "A1s": "bfloat16", "Y": "bfloat16", "Hs": "float32"}
+              "A1": "bfloat16", "A1s": "bfloat16", "Y": "bfloat16", "Hs": "float32", "AB": "bfloat16",
+              "ABs": "bfloat16", "dAB": "bfloat16", "dABs": "bfloat16", "dXp": "bfloat16", "dXs": "float32"}
 
 
 def dsmoe_workspace_tensor(handle, name: str):

@@ -183,6 +183,65 @@ __global__ void __launch_bounds__(kRbWarps * 32) router_backward_kernel(const Ro
   }
 }
 
+// dx = dh + (shared experts' fp32 rows) + (router part) + sum of the token's slot rows,
+// accumulated in fp32 in that order; 8 elements (16 bytes of each bf16 source) per step.
+template <int KMAX>
+__global__ void __launch_bounds__(128) dx_combine_kernel(const bf16* __restrict__ dh, const float* __restrict__ dXs,
+                                                          const float* __restrict__ dx_add,
+                                                          const bf16* __restrict__ dXp,
+                                                          const int32_t* __restrict__ slot_of, int T, int K, int d,
+                                                          float* __restrict__ dx) {
+  __shared__ int32_t s_slot[16];
+  const int d8 = d >> 3;
+  const uint4* dh4 = reinterpret_cast<const uint4*>(dh);
+  const uint4* dp4 = reinterpret_cast<const uint4*>(dXp);
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    __syncthreads();
+    if (threadIdx.x < K) s_slot[threadIdx.x] = slot_of[static_cast<int64_t>(t) * K + threadIdx.x];
+    __syncthreads();
+    for (int c = threadIdx.x; c < d8; c += blockDim.x) {
+      uint4 pv[KMAX];
+#pragma unroll
+      for (int k = 0; k < KMAX; ++k) {
+        const int p = k < K ? s_slot[k] : -1;
+        pv[k] = p >= 0 ? dp4[static_cast<int64_t>(p) * d8 + c] : make_uint4(0u, 0u, 0u, 0u);
+      }
+      float acc[8];
+      const uint4 hv = dh4[static_cast<int64_t>(t) * d8 + c];
+      const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = unpack_bf16x2(hw[j]);
+        acc[2 * j] = f.x;
+        acc[2 * j + 1] = f.y;
+      }
+      const int64_t o = static_cast<int64_t>(t) * d + 8 * c;
+      if (dXs) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] += dXs[o + j];
+      }
+      if (dx_add) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] += dx_add[o + j];
+      }
+#pragma unroll
+      for (int k = 0; k < KMAX; ++k) {
+        if (k >= K || s_slot[k] < 0) continue;
+        const uint32_t w[4] = {pv[k].x, pv[k].y, pv[k].z, pv[k].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = unpack_bf16x2(w[j]);
+          acc[2 * j] += f.x;
+          acc[2 * j + 1] += f.y;
+        }
+      }
+      float4* o4 = reinterpret_cast<float4*>(dx + o);
+      o4[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      o4[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
+  }
+}
+
 // C[m, n] = sum_k A(m, k) B[k, n] on the CUDA cores: A fp32 with element (m, k) at
 // A[m * a_sm + k * a_sk], B bf16 row-major [K, ldb], C fp32 [M, ldc]. A block computes a
 // 64 x 128 tile from 32-deep slices staged in shared memory; each thread owns 4 x 8
@@ -262,6 +321,19 @@ cudaError_t launch_router_backward(const RouterBwdArgs& a, int num_sms, cudaStre
   else if (npl <= 8) router_backward_kernel<8><<<grid, kRbWarps * 32, 0, s>>>(a);
   else if (npl <= 12) router_backward_kernel<12><<<grid, kRbWarps * 32, 0, s>>>(a);
   else if (npl <= 16) router_backward_kernel<16><<<grid, kRbWarps * 32, 0, s>>>(a);
+  else return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dx_combine(const bf16* dh, const float* dXs, const float* dx_add, const bf16* dXp,
+                              const int32_t* slot_of, int T, int K, int d, float* dx, int num_sms, cudaStream_t s) {
+  int grid = T;
+  if (grid > 16 * num_sms) grid = 16 * num_sms;
+  if (grid < 1) grid = 1;
+  if (K <= 2) dx_combine_kernel<2><<<grid, 128, 0, s>>>(dh, dXs, dx_add, dXp, slot_of, T, K, d, dx);
+  else if (K <= 4) dx_combine_kernel<4><<<grid, 128, 0, s>>>(dh, dXs, dx_add, dXp, slot_of, T, K, d, dx);
+  else if (K <= 8) dx_combine_kernel<8><<<grid, 128, 0, s>>>(dh, dXs, dx_add, dXp, slot_of, T, K, d, dx);
+  else if (K <= 16) dx_combine_kernel<16><<<grid, 128, 0, s>>>(dh, dXs, dx_add, dXp, slot_of, T, K, d, dx);
   else return cudaErrorInvalidValue;
   return cudaGetLastError();
 }

@@ -92,6 +92,21 @@ bool map_3d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, uint
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 4D bf16 view (64, rows, cols / 64, experts) of an [experts, rows, cols] tensor whose
+// cols are contiguous, 128-byte swizzle, box (64, 64, 4, 1): one copy lands 256 cols x 64
+// rows as four MN-major atoms (the backward GEMMs' A operand).
+bool map_4d_mn(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint64_t experts) {
+  auto enc = tensor_map_encoder();
+  if (!enc || cols % 64) return false;
+  cuuint64_t dims[4] = {64, rows, cols / 64, experts};
+  cuuint64_t strides[3] = {cols * 2, 128, rows * cols * 2};
+  cuuint32_t box[4] = {64, 64, 4, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct DeviceGuard {
   int prev = -1, want;
   bool ok = false;
@@ -217,6 +232,12 @@ struct dsmoe_handle {
   cudaEvent_t ev[kTimingSlots][kNumStages + 1] = {};
   int64_t launches = 0;
   int32_t ep_T = -1;  // tokens of the last dsmoe_ep_route (its slot table is in the workspace)
+  // training buffers (dsmoe_set_training): the forward's saved pre-activations a | b, and
+  // the backward's da | db and per-slot / shared input gradients
+  char* tr = nullptr;
+  bf16 *AB = nullptr, *ABs = nullptr, *dAB = nullptr, *dABs = nullptr, *dXp = nullptr;
+  float* dXs = nullptr;
+  int32_t saved_T = -1;  // tokens of the last forward that saved a | b
 };
 
 // ========================================================================================
@@ -290,6 +311,7 @@ static void release(dsmoe_handle* h) {
     for (cudaEvent_t e : {h->ev_in[i], h->ev_out[i], h->ev_d2h[i]})
       if (e) cudaEventDestroy(e);
   if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
+  if (h->tr) cudaFree(h->tr);
   if (h->ws) cudaFree(h->ws);
   delete h;
 }
@@ -611,6 +633,7 @@ struct GemmPlan {
   const CUtensorMap *wg, *wu, *wd, *swg, *swu, *swd;
   const bf16* residual;             // x, added to the shared rows of the down GEMM
   bf16* Y_out;                      // [routed_rows, d] routed expert outputs
+  bool save_ab = false;             // also store the pre-activations a | b (training)
 };
 
 dsmoe_status gemm_stage(dsmoe_handle* h, const GemmPlan& p, cudaStream_t s,
@@ -645,6 +668,8 @@ dsmoe_status gemm_stage(dsmoe_handle* h, const GemmPlan& p, cudaStream_t s,
     g.out_shared = h->A1s;
     g.ld_shared = static_cast<int64_t>(Ks) * Fs;
     g.shared_col_stride = Fs;
+    g.save_ab_routed = p.save_ab ? h->AB : nullptr;
+    g.save_ab_shared = p.save_ab ? h->ABs : nullptr;
     g.status = h->status;
     g.wait_limit_ns = h->wait_ns;
     const int64_t tt = pair ? dsmoe::kGemmPairTokenTile : dsmoe::kGemmGateUpTokenTile;
@@ -789,7 +814,9 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
   p.Ks = Ks;
   p.residual = static_cast<const bf16*>(a.x);
   p.Y_out = h->Y;
+  p.save_ab = h->tr != nullptr;
   STAGE_TRY(gemm_stage(h, p, s, mark));
+  if (h->tr) h->saved_T = T;
   STAGE_TRY(combine_stage(h, a, h->Y, Ks, h->add_shared, h->partial, s));
   CUDA_TRY(mark(7));
   if (timing) h->timed_forwards += 1;
@@ -1270,6 +1297,153 @@ DSMOE_EXPORT dsmoe_status dsmoe_backward_router(dsmoe_handle* h, int32_t T, cons
   return DSMOE_OK;
 }
 
+DSMOE_EXPORT dsmoe_status dsmoe_set_training(dsmoe_handle* h, int32_t enable) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
+  if (!enable) {
+    if (h->tr) {
+      CUDA_TRY(cudaDeviceSynchronize());
+      CUDA_TRY(cudaFree(h->tr));
+    }
+    h->tr = nullptr;
+    h->AB = h->ABs = h->dAB = h->dABs = h->dXp = nullptr;
+    h->dXs = nullptr;
+    h->saved_T = -1;
+    return DSMOE_OK;
+  }
+  if (h->tr) return DSMOE_OK;
+  const dsmoe_cfg& c = h->cfg;
+  const size_t T = c.max_tokens, S = T * c.top_k, F = c.d_ff, d = c.d_model;
+  const size_t KsFs = static_cast<size_t>(c.n_shared) * c.d_ff_shared;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += up256(bytes > 0 ? bytes : 1);
+    return o;
+  };
+  const size_t oAB = take(S * 2 * F * 2), oABs = take(T * 2 * KsFs * 2), odAB = take(S * 2 * F * 2),
+               odABs = take(T * 2 * KsFs * 2), odXp = take(S * d * 2), odXs = take(c.n_shared ? T * d * 4 : 0);
+  char* p = nullptr;
+  const cudaError_t e = cudaMalloc(&p, off);
+  if (e != cudaSuccess) return fail(DSMOE_ERR_WORKSPACE, "cudaMalloc(%zu) of the training buffers failed: %s", off,
+                                    cudaGetErrorString(e));
+  h->tr = p;
+  h->AB = reinterpret_cast<bf16*>(p + oAB);
+  h->ABs = reinterpret_cast<bf16*>(p + oABs);
+  h->dAB = reinterpret_cast<bf16*>(p + odAB);
+  h->dABs = reinterpret_cast<bf16*>(p + odABs);
+  h->dXp = reinterpret_cast<bf16*>(p + odXp);
+  h->dXs = reinterpret_cast<float*>(p + odXs);
+  h->saved_T = -1;
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_backward_experts(dsmoe_handle* h, int32_t T, const void* dh, const void* dY,
+                                                 const void* W_gate, const void* W_up, const void* W_down,
+                                                 const void* Ws_gate, const void* Ws_up, const void* Ws_down,
+                                                 const float* dx_add, float* dx, void* stream) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  const dsmoe_cfg& c = h->cfg;
+  if (!h->tr) return fail(DSMOE_ERR_INVALID_ARG, "training buffers are not enabled (dsmoe_set_training)");
+  if (T != h->saved_T || T <= 0)
+    return fail(DSMOE_ERR_INVALID_ARG, "T = %d is not the token count of the last training forward (%d)", T,
+                h->saved_T);
+  const int Ks = h->add_shared ? c.n_shared : 0;
+  if (!dh || !dY || !W_gate || !W_up || !W_down || !dx || (Ks && (!Ws_gate || !Ws_up || !Ws_down)))
+    return fail(DSMOE_ERR_INVALID_ARG, "NULL argument");
+  const void* must_align[] = {dh, dY, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, dx, dx_add};
+  for (const void* q : must_align)
+    if (q && !aligned16(q)) return fail(DSMOE_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", q);
+  DeviceGuard gd(h->device);
+  if (!gd.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int d = c.d_model, F = c.d_ff, Fs = c.d_ff_shared, K = h->k_active;
+  const int NL = h->e_end - h->e_begin;
+  const int64_t S = static_cast<int64_t>(T) * K;
+  CUtensorMap m_dY, m_dh, m_dAB, m_dABs, m_wd, m_wg, m_wu, m_swd, m_swg, m_swu;
+  bool ok = map_2d(&m_dY, dY, d, S, 128) && map_2d(&m_dh, dh, d, T, 128) &&
+            map_2d(&m_dAB, h->dAB, 2 * F, S, 128) && map_4d_mn(&m_wd, W_down, d, F, NL) &&
+            map_4d_mn(&m_wg, W_gate, F, d, NL) && map_4d_mn(&m_wu, W_up, F, d, NL);
+  if (Ks)
+    ok = ok && map_2d(&m_dABs, h->dABs, 2 * static_cast<uint64_t>(Ks) * Fs, T, 128) &&
+         map_4d_mn(&m_swd, Ws_down, d, Fs, Ks) && map_4d_mn(&m_swg, Ws_gate, Fs, d, Ks) &&
+         map_4d_mn(&m_swu, Ws_up, Fs, d, Ks);
+  else
+    m_dABs = m_dAB, m_swd = m_wd, m_swg = m_wg, m_swu = m_wu;
+  if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map of the backward");
+  auto grid_for = [&](const dsmoe::GemmArgs& g) {
+    const int64_t bound = (cdiv(S, 128) + NL) * static_cast<int64_t>(g.n_tiles_routed) +
+                          static_cast<int64_t>(g.n_shared_groups) * cdiv(T, 128) * g.n_tiles_shared;
+    return static_cast<int>(bound < h->num_sms ? bound : h->num_sms);
+  };
+  // da | db from dy (routed: dY per slot; shared: dh) and W_down
+  {
+    dsmoe::GemmBwdArgs b;
+    memset(&b, 0, sizeof(b));
+    dsmoe::GemmArgs& g = b.g;
+    g.a_routed = m_dY;
+    g.a_shared = m_dh;
+    g.b0_routed = g.b1_routed = m_wd;
+    g.b0_shared = g.b1_shared = m_swd;
+    g.offsets = h->offsets + h->e_begin;
+    g.n_routed = NL;
+    g.n_shared_groups = Ks;
+    g.m_shared = T;
+    g.n_tiles_routed = cdiv(F, 256);
+    g.n_tiles_shared = Ks ? cdiv(Fs, 256) : 0;
+    g.kb_routed = d / 64;
+    g.kb_shared = d / 64;
+    g.n_valid_routed = F;
+    g.n_valid_shared = Fs;
+    g.status = h->status;
+    g.wait_limit_ns = h->wait_ns;
+    b.ab_routed = h->AB;
+    b.ab_shared = h->ABs;
+    b.dab_routed = h->dAB;
+    b.dab_shared = h->dABs;
+    b.ld_ab_routed = 2 * static_cast<int64_t>(F);
+    b.ld_ab_shared = 2 * static_cast<int64_t>(Ks) * Fs;
+    b.width_routed = F;
+    b.width_shared = Fs;
+    CUDA_TRY(dsmoe::launch_grouped_gemm_bwd(dsmoe::kBwdDM, b, grid_for(g), s));
+  }
+  // input gradients from da | db and W_gate, W_up (the shared experts summed in one group)
+  {
+    dsmoe::GemmBwdArgs b;
+    memset(&b, 0, sizeof(b));
+    dsmoe::GemmArgs& g = b.g;
+    g.a_routed = m_dAB;
+    g.a_shared = m_dABs;
+    g.b0_routed = m_wg;
+    g.b1_routed = m_wu;
+    g.b0_shared = m_swg;
+    g.b1_shared = m_swu;
+    g.offsets = h->offsets + h->e_begin;
+    g.n_routed = NL;
+    g.n_shared_groups = Ks ? 1 : 0;
+    g.m_shared = T;
+    g.n_tiles_routed = cdiv(d, 256);
+    g.n_tiles_shared = Ks ? cdiv(d, 256) : 0;
+    g.kb_routed = 2 * F / 64;
+    g.kb_shared = Ks ? 2 * Ks * Fs / 64 : 0;
+    g.n_valid_routed = d;
+    g.n_valid_shared = d;
+    g.status = h->status;
+    g.wait_limit_ns = h->wait_ns;
+    b.kb_half_routed = F / 64;
+    b.kb_half_shared = Fs / 64;
+    b.dx_routed = h->dXp;
+    b.dx_shared = h->dXs;
+    b.ld_dx = d;
+    CUDA_TRY(dsmoe::launch_grouped_gemm_bwd(dsmoe::kBwdDX, b, grid_for(g), s));
+  }
+  CUDA_TRY(dsmoe::launch_dx_combine(static_cast<const bf16*>(dh), Ks ? h->dXs : nullptr, dx_add, h->dXp, h->slot_of,
+                                    T, K, d, dx, h->num_sms, s));
+  h->launches += 3;
+  return DSMOE_OK;
+}
+
 DSMOE_EXPORT dsmoe_status dsmoe_set_timing(dsmoe_handle* h, int32_t enable) {
   if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
   h->timing = enable != 0;
@@ -1328,6 +1502,12 @@ DSMOE_EXPORT dsmoe_status dsmoe_workspace_tensor(dsmoe_handle* h, const char* na
       {"A1s", h->A1s, T, static_cast<int64_t>(c.n_shared) * c.d_ff_shared, c.n_shared > 0},
       {"Y", h->Y, S, c.d_model, true},
       {"Hs", h->Hs, T, c.d_model, c.n_shared > 0},
+      {"AB", h->AB, S, 2 * static_cast<int64_t>(c.d_ff), h->tr != nullptr},
+      {"dAB", h->dAB, S, 2 * static_cast<int64_t>(c.d_ff), h->tr != nullptr},
+      {"ABs", h->ABs, T, 2 * static_cast<int64_t>(c.n_shared) * c.d_ff_shared, h->tr != nullptr && c.n_shared > 0},
+      {"dABs", h->dABs, T, 2 * static_cast<int64_t>(c.n_shared) * c.d_ff_shared, h->tr != nullptr && c.n_shared > 0},
+      {"dXp", h->dXp, S, c.d_model, h->tr != nullptr},
+      {"dXs", h->dXs, T, c.d_model, h->tr != nullptr && c.n_shared > 0},
   };
   for (const Entry& e : table) {
     if (strcmp(e.n, name) == 0) {

@@ -255,6 +255,32 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         tmem_ld16(tb + G_::kChainCols + c0, *reinterpret_cast<uint32_t(*)[16]>(&v1[0]));
         tmem_ld16(tb + G_::kChainCols + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v1[16]));
         tmem_wait_ld();
+        // the backward pass's saved pre-activations: a (chain 0) and b (chain 1) as bf16
+        bf16* save = kSwiGLU ? (t.shared ? a.save_ab_shared : a.save_ab_routed) : nullptr;
+        if (kSwiGLU && save) {
+          const int width = t.shared ? a.shared_col_stride : a.n_valid_routed;  // F_s or F
+          const int64_t lds = 2 * (t.shared ? a.ld_shared : a.ld_routed);
+          const int64_t col0 = t.shared ? static_cast<int64_t>(t.group) * 2 * width : 0;
+          const int feat = t.n_blk * kFeat + q * 32 + cc;
+#pragma unroll 1
+          for (int ch = 0; ch < 2; ++ch) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) stg[j * kStageRow + lane] = __uint_as_float(ch == 0 ? v0[j] : v1[j]);
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int row = rr + 8 * i;
+              if (feat < width && c0 + row < t.m_valid) {
+                const float* src = stg + row * kStageRow + cc;
+                *reinterpret_cast<uint4*>(save + static_cast<int64_t>(t.row0 + c0 + row) * lds + col0 +
+                                          ch * width + feat) =
+                    make_uint4(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
+                               pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
+              }
+            }
+            __syncwarp();
+          }
+        }
 #pragma unroll 1
         for (int ch = 0; ch < n_out; ++ch) {
           // stage: row = token (c0 + j), column = this lane's feature

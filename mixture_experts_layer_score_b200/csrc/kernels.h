@@ -165,6 +165,11 @@ struct RouterBwdArgs {
 };
 cudaError_t launch_router_backward(const RouterBwdArgs& a, int num_sms, cudaStream_t s);
 
+// dx[t] = dh[t] + dXs[t] (if set) + dx_add[t] (if set) + sum_k dXp[slot_of[t,k]] (fp32 out;
+// slots of -1 are skipped).
+cudaError_t launch_dx_combine(const bf16* dh, const float* dXs, const float* dx_add, const bf16* dXp,
+                              const int32_t* slot_of, int T, int K, int d, float* dx, int num_sms, cudaStream_t s);
+
 // C[M, N] = A(M x K, fp32, element (m, k) at A[m a_sm + k a_sk]) * B (bf16 [K, ldb]), fp32 out.
 struct GemmF32Args {
   const float* A;
@@ -208,8 +213,32 @@ struct GemmArgs {
   int32_t shared_col_stride;      // shared group g writes at column g * shared_col_stride
   uint32_t* status;
   uint64_t wait_limit_ns;
+  // gate/up only, for the backward pass: when set, the pre-activations a = X W_gate^T and
+  // b = X W_up^T are also stored (bf16), a | b side by side: routed [rows, 2F]; shared
+  // [T, K_s 2 F_s] with shared expert g at columns 2 g F_s
+  bf16* save_ab_routed;
+  bf16* save_ab_shared;
 };
 cudaError_t launch_grouped_gemm(bool swiglu, const GemmArgs& a, int grid, cudaStream_t s);
+
+// The experts' backward GEMMs (gemm_bwd_sm100.cu). kBwdDM: da | db from dy and W_down;
+// kBwdDX: dx rows from da | db and W_gate, W_up. The weight maps b0 / b1 of `g` are 4-D
+// views (64 M, K, M / 64, experts) of the weights with box (64, 64, 4, 1), M contiguous.
+enum { kBwdDM = 0, kBwdDX = 1 };
+struct GemmBwdArgs {
+  GemmArgs g;                              // schedule, token-row maps, weight views, status
+  int32_t kb_half_routed, kb_half_shared;  // kBwdDX: F / 64 and F_s / 64 (K blocks per half)
+  const bf16* ab_routed;                   // kBwdDM: the forward's saved a | b
+  const bf16* ab_shared;
+  bf16* dab_routed;                        // kBwdDM out: da | db, same layout
+  bf16* dab_shared;
+  int64_t ld_ab_routed, ld_ab_shared;
+  int32_t width_routed, width_shared;      // F and F_s
+  bf16* dx_routed;                         // kBwdDX out: [rows, d] bf16 per slot
+  float* dx_shared;                        // kBwdDX out: [T, d] fp32, summed over shared experts
+  int64_t ld_dx;
+};
+cudaError_t launch_grouped_gemm_bwd(int mode, const GemmBwdArgs& a, int grid, cudaStream_t s);
 
 // The same grouped GEMM on CTA pairs (clusters of two, tcgen05 cta_group::2): a pair
 // computes 128 features (gate/up) or 256 output rows (down) by up to

@@ -104,3 +104,85 @@ def test_backward_argument_errors():
         assert ei.value.status == M.DSMOE_ERR_INVALID_ARG
     finally:
         layer.close()
+
+
+EXP_CASES = [("tiny", 300), ("gshard_c", 500), ("ds2b", 700), ("v3_slice", 256)]
+
+
+@pytest.mark.parametrize("name,T", EXP_CASES, ids=[f"{c[0]}-T{c[1]}" for c in EXP_CASES])
+def test_expert_backward_input_gradient(name, T):
+    """dL/du through the experts (dsmoe_backward_experts: W_down^T dy -> SiLU backward with
+    the saved pre-activations -> W_gate^T da + W_up^T db on the tensor cores, weights read
+    MN-major) plus the router's part, against the oracle's layer_backward dx (float64):
+    max |err| / RMS <= 3e-2 (bf16 operands: g dh, the saved a and b, da | db and the
+    per-slot rows, each rounded once; fp32 accumulation). The shared experts' fp32 sum dXs
+    is checked on its own against the oracle's SwiGLU backward within 2e-2."""
+    cfg = W.get_config(name)
+    gpu, cpu = make_case(cfg, T)
+    dh = W.normal_bf16((T, cfg.d_model), 1.0, 0, "dh", 0, "cuda")
+    alpha = 0.01
+    layer = M.DSMoE(M.cfg_from(cfg, T), gpu)
+    try:
+        M.dsmoe_set_training(layer.handle, True)
+        out = layer.forward(gpu["x"], with_scores=True)
+        K, N, d = cfg.top_k, cfg.n_routed, cfg.d_model
+        dg = torch.empty((T, K), dtype=torch.float32, device="cuda")
+        dY = torch.empty((T * K, d), dtype=torch.bfloat16, device="cuda")
+        M.dsmoe_backward_gates(layer.handle, T, dh, out["gates"], dg, dY)
+        dl = torch.empty((T, N), dtype=torch.float32, device="cuda")
+        dx_r = torch.empty((T, d), dtype=torch.float32, device="cuda")
+        dWr = torch.empty((N, d), dtype=torch.float32, device="cuda")
+        M.dsmoe_backward_router(layer.handle, T, gpu["x"], gpu["W_router"], out["topk_idx"], out["gates"],
+                                out["scores"], dg, out["f"], alpha, dl, dx_r, dWr)
+        dx = torch.empty((T, d), dtype=torch.float32, device="cuda")
+        M.dsmoe_backward_experts(layer.handle, T, dh, dY, gpu["W_gate"], gpu["W_up"], gpu["W_down"],
+                                 gpu.get("Ws_gate"), gpu.get("Ws_up"), gpu.get("Ws_down"), dx_r, dx)
+        torch.cuda.synchronize()
+        assert M.dsmoe_get_status(layer.handle) == M.DSMOE_OK, M.dsmoe_last_error()
+        dxs = M.workspace_view(layer.handle, "dXs")[:T].clone() if cfg.n_shared else None
+        M.dsmoe_set_training(layer.handle, False)
+    finally:
+        layer.close()
+    ref = PAR.reference_selection(cfg, cpu, out["topk_idx"], out["scores"])
+    PAR.check_routing(cfg, ref, out, T)
+    dh64 = dh.float().cpu().numpy().astype(np.float64)
+    bw = DB.layer_backward(cfg, cpu, dh64, routing=ref, alpha_bal=alpha)
+    e_dx = _rel(dx.cpu().numpy(), bw["dx"])
+    e_s = 0.0
+    if cfg.n_shared:
+        X = cpu["x"].float().numpy().astype(np.float64)
+        ref_s = np.zeros_like(X)
+        for i in range(cfg.n_shared):
+            ref_s += DB.swiglu_backward(X, cpu["Ws_gate"][i], cpu["Ws_up"][i], cpu["Ws_down"][i], dh64)[0]
+        e_s = _rel(dxs.cpu().numpy(), ref_s)
+    for k_ in ("W_gate", "W_up", "W_down"):
+        if hasattr(cpu[k_], "cache"):
+            cpu[k_].cache.clear()
+    print(name, T, "dx err/RMS", e_dx, "shared du err/RMS", e_s)
+    assert e_dx <= 3e-2 and e_s <= 2e-2
+
+
+def test_expert_backward_needs_a_training_forward():
+    cfg = W.get_config("tiny")
+    gpu, _ = make_case(cfg, 64)
+    layer = M.DSMoE(M.cfg_from(cfg, 64), gpu)
+    try:
+        dh = torch.zeros((64, cfg.d_model), dtype=torch.bfloat16, device="cuda")
+        dY = torch.zeros((64 * cfg.top_k, cfg.d_model), dtype=torch.bfloat16, device="cuda")
+        dx = torch.empty((64, cfg.d_model), dtype=torch.float32, device="cuda")
+        args = (dh, dY, gpu["W_gate"], gpu["W_up"], gpu["W_down"], gpu["Ws_gate"], gpu["Ws_up"], gpu["Ws_down"], None,
+                dx)
+        with pytest.raises(M.DsmoeError):  # training buffers not enabled
+            M.dsmoe_backward_experts(layer.handle, 64, *args)
+        M.dsmoe_set_training(layer.handle, True)
+        with pytest.raises(M.DsmoeError):  # no training forward yet
+            M.dsmoe_backward_experts(layer.handle, 64, *args)
+        layer.forward(gpu["x"])
+        with pytest.raises(M.DsmoeError):  # a different T than the forward's
+            M.dsmoe_backward_experts(layer.handle, 32, *args)
+        M.dsmoe_backward_experts(layer.handle, 64, *args)
+        torch.cuda.synchronize()
+        assert M.dsmoe_get_status(layer.handle) == M.DSMOE_OK
+        assert torch.equal(dx, dh.float())  # dh = 0: every part of the gradient is 0 but the residual's
+    finally:
+        layer.close()
