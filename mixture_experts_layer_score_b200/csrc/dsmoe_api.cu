@@ -215,7 +215,8 @@ struct dsmoe_handle {
   } stage[2];
   // the pipelined host entry point: its copy stream and, per staging slot, the events
   // that order input copy -> forward -> output copy -> reuse of the slot
-  cudaStream_t copy_stream = nullptr;
+  cudaStream_t copy_stream = nullptr;    // input copies
+  cudaStream_t copy_stream_out = nullptr;  // output copies (both directions run at once)
   cudaEvent_t ev_in[2] = {}, ev_out[2] = {}, ev_d2h[2] = {};
   int64_t async_calls = 0;
   CUtensorMap tm_xp, tm_a1, tm_a1s;
@@ -311,6 +312,7 @@ static void release(dsmoe_handle* h) {
     for (cudaEvent_t e : {h->ev_in[i], h->ev_out[i], h->ev_d2h[i]})
       if (e) cudaEventDestroy(e);
   if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
+  if (h->copy_stream_out) cudaStreamDestroy(h->copy_stream_out);
   if (h->tr) cudaFree(h->tr);
   if (h->ws) cudaFree(h->ws);
   delete h;
@@ -341,7 +343,7 @@ DSMOE_EXPORT dsmoe_status dsmoe_create(const dsmoe_cfg* cfg, int32_t device, dsm
   h->e_end = h->cfg.n_routed;
   h->num_sms = prop.multiProcessorCount;
   h->pair_clusters[0] = dsmoe::grouped_gemm_pair_max_clusters(false);
-  h->pair_clusters[1] = dsmoe::grouped_gemm_pair_max_clusters(true);
+  h->pair_clusters[1] = dsmoe::gateup_pair_max_clusters();
   dsmoe::router_tc_shape(cfg->n_routed, &h->rt_chunks, &h->rt_nc, &h->rt_cols);
   h->L = plan(h->cfg);
   cudaError_t e = cudaMalloc(&h->ws, h->L.total);
@@ -404,6 +406,7 @@ DSMOE_EXPORT dsmoe_status dsmoe_create(const dsmoe_cfg* cfg, int32_t device, dsm
     for (cudaEvent_t* ev : {&h->ev_in[i], &h->ev_out[i], &h->ev_d2h[i]})
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->copy_stream_out, cudaStreamNonBlocking);
   if (e != cudaSuccess) {
     release(h);
     return fail(DSMOE_ERR_CUDA, "event or stream creation failed: %s", cudaGetErrorString(e));
@@ -656,8 +659,9 @@ dsmoe_status gemm_stage(dsmoe_handle* h, const GemmPlan& p, cudaStream_t s,
     g.expert_mod = p.expert_mod;
     g.n_shared_groups = Ks;
     g.m_shared = T;
-    g.n_tiles_routed = p.n_groups ? cdiv(F, 128) : 0;
-    g.n_tiles_shared = Ks ? cdiv(Fs, 128) : 0;
+    const int ftile = pair ? 256 : 128;  // features per gate/up tile
+    g.n_tiles_routed = p.n_groups ? cdiv(F, ftile) : 0;
+    g.n_tiles_shared = Ks ? cdiv(Fs, ftile) : 0;
     g.kb_routed = d / 64;
     g.kb_shared = d / 64;
     g.kb_per_b_expert_shared = d / 64;
@@ -678,7 +682,7 @@ dsmoe_status gemm_stage(dsmoe_handle* h, const GemmPlan& p, cudaStream_t s,
     if (bound > 0) {
       if (pair) {
         const int clusters = static_cast<int>(bound < h->pair_clusters[1] ? bound : h->pair_clusters[1]);
-        CUDA_TRY(dsmoe::launch_grouped_gemm_pair(true, g, clusters, s));
+        CUDA_TRY(dsmoe::launch_gateup_pair(g, clusters, s));
       } else {
         const int grid = static_cast<int>(bound < h->num_sms ? bound : h->num_sms);
         CUDA_TRY(dsmoe::launch_grouped_gemm(true, g, grid, s));
@@ -786,14 +790,14 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
 
   // tensor maps that depend on the call's pointers
   bool ok = true;
-  const int wm = h->gemm_kernel == DSMOE_GEMM_PAIR ? 7 : 0;  // first weight map of the chosen GEMM kernel
+  const bool pair = h->gemm_kernel == DSMOE_GEMM_PAIR;  // the down projection's weight box differs
   GemmPlan p;
-  p.wg = weight_map(h, wm + 0, a.W_gate, &ok);
-  p.wu = weight_map(h, wm + 1, a.W_up, &ok);
-  p.wd = weight_map(h, wm + 2, a.W_down, &ok);
-  p.swg = Ks ? weight_map(h, wm + 3, a.Ws_gate, &ok) : p.wg;
-  p.swu = Ks ? weight_map(h, wm + 4, a.Ws_up, &ok) : p.wu;
-  p.swd = Ks ? weight_map(h, wm + 5, a.Ws_down, &ok) : p.wd;
+  p.wg = weight_map(h, 0, a.W_gate, &ok);
+  p.wu = weight_map(h, 1, a.W_up, &ok);
+  p.wd = weight_map(h, pair ? 9 : 2, a.W_down, &ok);
+  p.swg = Ks ? weight_map(h, 3, a.Ws_gate, &ok) : p.wg;
+  p.swu = Ks ? weight_map(h, 4, a.Ws_up, &ok) : p.wu;
+  p.swd = Ks ? weight_map(h, pair ? 12 : 5, a.Ws_down, &ok) : p.wd;
   CUtensorMap m_x;  // token rows of x in GEMM tiles (shared groups)
   ok = ok && map_2d(&m_x, a.x, d, T, dsmoe::kGemmGateUpTokenTile);
   if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map of this call");
@@ -877,6 +881,8 @@ dsmoe_status host_forward(dsmoe_handle* h, const HostArgs& a, int slot, cudaStre
   dsmoe_handle::Stage& st = h->stage[slot];
   const size_t xb = static_cast<size_t>(T) * c.d_model * 2, sb = static_cast<size_t>(T) * h->k_active * 4,
                nb = static_cast<size_t>(c.n_routed) * 4;
+  // the slot's input buffer is free once the forward that last read it has finished
+  if (pipelined) CUDA_TRY(cudaStreamWaitEvent(cin, h->ev_out[slot], 0));
   if (T > 0) {
     CUDA_TRY(cudaMemcpyAsync(st.x, a.x_host, xb, cudaMemcpyHostToDevice, cin));
     if (hash) CUDA_TRY(cudaMemcpyAsync(st.ids, a.token_ids_host, static_cast<size_t>(T) * 4, cudaMemcpyHostToDevice, cin));
@@ -923,6 +929,7 @@ DSMOE_EXPORT dsmoe_status dsmoe_forward_host(dsmoe_handle* h, int32_t T, const v
   if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   CUDA_TRY(cudaStreamSynchronize(h->copy_stream));  // no pipelined call still uses the staging
+  CUDA_TRY(cudaStreamSynchronize(h->copy_stream_out));
   STAGE_TRY(host_forward(h, a, 0, s, s, s, false));
   CUDA_TRY(cudaStreamSynchronize(s));
   return DSMOE_OK;
@@ -942,7 +949,7 @@ DSMOE_EXPORT dsmoe_status dsmoe_forward_host_async(dsmoe_handle* h, int32_t T, c
   DeviceGuard g(h->device);
   if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
   const int slot = static_cast<int>(h->async_calls & 1);
-  STAGE_TRY(host_forward(h, a, slot, h->copy_stream, static_cast<cudaStream_t>(stream), h->copy_stream, true));
+  STAGE_TRY(host_forward(h, a, slot, h->copy_stream, static_cast<cudaStream_t>(stream), h->copy_stream_out, true));
   h->async_calls += 1;
   return DSMOE_OK;
 }
@@ -961,6 +968,7 @@ DSMOE_EXPORT dsmoe_status dsmoe_host_sync(dsmoe_handle* h) {
   DeviceGuard g(h->device);
   if (!g.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
   CUDA_TRY(cudaStreamSynchronize(h->copy_stream));
+  CUDA_TRY(cudaStreamSynchronize(h->copy_stream_out));
   return DSMOE_OK;
 }
 
@@ -1027,11 +1035,11 @@ DSMOE_EXPORT dsmoe_status dsmoe_ep_experts(dsmoe_handle* h, int32_t n_src, int32
   CUDA_TRY(dsmoe::launch_group_offsets(recv_counts, groups, h->offsets, h->status, s));
   h->launches += 1;
   bool ok = true;
-  const int wm = h->gemm_kernel == DSMOE_GEMM_PAIR ? 7 : 0;
+  const bool pair = h->gemm_kernel == DSMOE_GEMM_PAIR;
   GemmPlan p;
-  p.wg = weight_map(h, wm + 0, W_gate, &ok, n_local);
-  p.wu = weight_map(h, wm + 1, W_up, &ok, n_local);
-  p.wd = weight_map(h, wm + 2, W_down, &ok, n_local);
+  p.wg = weight_map(h, 0, W_gate, &ok, n_local);
+  p.wu = weight_map(h, 1, W_up, &ok, n_local);
+  p.wd = weight_map(h, pair ? 9 : 2, W_down, &ok, n_local);
   p.swg = p.wg;
   p.swu = p.wu;
   p.swd = p.wd;
@@ -1073,11 +1081,11 @@ DSMOE_EXPORT dsmoe_status dsmoe_ep_combine(dsmoe_handle* h, int32_t T, const voi
   const std::function<cudaError_t(int)> mark = [](int) { return cudaSuccess; };
   if (Ks > 0) {
     bool ok = true;
-    const int wm = h->gemm_kernel == DSMOE_GEMM_PAIR ? 7 : 0;
+    const bool pair = h->gemm_kernel == DSMOE_GEMM_PAIR;
     GemmPlan p;
-    p.swg = weight_map(h, wm + 3, Ws_gate, &ok);
-    p.swu = weight_map(h, wm + 4, Ws_up, &ok);
-    p.swd = weight_map(h, wm + 5, Ws_down, &ok);
+    p.swg = weight_map(h, 3, Ws_gate, &ok);
+    p.swu = weight_map(h, 4, Ws_up, &ok);
+    p.swd = weight_map(h, pair ? 12 : 5, Ws_down, &ok);
     p.wg = p.swg;
     p.wu = p.swu;
     p.wd = p.swd;

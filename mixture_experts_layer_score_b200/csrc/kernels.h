@@ -251,6 +251,12 @@ constexpr int kGemmPairGateUpRows = 64;
 int grouped_gemm_pair_max_clusters(bool swiglu);
 cudaError_t launch_grouped_gemm_pair(bool swiglu, const GemmArgs& a, int clusters, cudaStream_t s);
 
+// The gate/up projection on CTA pairs with two M=256 chains (gemm_gateup_pair_sm100.cu):
+// tiles of 256 features by up to kGemmPairTokenTile tokens; weight maps box (64, 128)
+// (the one-CTA kernel's), token maps box (64, 128); n_tiles_* count 256-feature tiles.
+int gateup_pair_max_clusters();
+cudaError_t launch_gateup_pair(const GemmArgs& a, int clusters, cudaStream_t s);
+
 // ---------------------------------------------------------------- errors (dsmoe_api.cu)
 // Record the calling thread's last-error message (read back by dsmoe_last_error).
 void note_error(const char* fmt, ...);

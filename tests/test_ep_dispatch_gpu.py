@@ -25,7 +25,7 @@ pytestmark = pytest.mark.gpu
 if not torch.cuda.is_available():
     pytest.skip("no GPU", allow_module_level=True)
 
-CASES = [("tiny", 301, 2), ("gshard_c", 700, 3), ("v4_decode_t64", 64, 4), ("v4_hash_t64", 64, 2)]
+CASES = [("tiny", 301, 2), ("gshard_c", 700, 3), ("v4_decode_t16", 16, 4), ("v4_hash_t16", 16, 2)]
 
 
 @pytest.mark.parametrize("name,T,R", CASES, ids=[f"{c[0]}-R{c[2]}" for c in CASES])

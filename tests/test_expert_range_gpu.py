@@ -5,9 +5,11 @@ on engineering trade-offs, item 5: shared experts replicated, routed experts sha
 
 The "ranks" of an R-way split run one after another on the same GPU (each is an
 independent forward; none waits on another). Each partial is compared with the oracle's
-partial (oracle/dsmoe_ep.py gather_partial) element-wise, max |err| / RMS <= 2e-2; the sum
-over ranks, rounded to bf16 by the library, must meet the layer bound against the
-oracle's h; every rank's routing must equal the oracle's and each other's."""
+partial (oracle/dsmoe_ep.py gather_partial) element-wise, max |err| <= 2e-2 RMS(h) with h
+the whole layer's output that the partials add up to (a partial without the residual is
+smaller than h, while its error, one bf16 rounding of each expert row it sums, is the same
+as in h); the sum over ranks, rounded to bf16 by the library, must meet the layer bound
+against the oracle's h; every rank's routing must equal the oracle's and each other's."""
 import numpy as np
 import pytest
 import torch
@@ -23,7 +25,7 @@ pytestmark = pytest.mark.gpu
 if not torch.cuda.is_available():
     pytest.skip("no GPU", allow_module_level=True)
 
-CASES = [("v4_decode_t64", 64, 4), ("v4_decode_t64", 64, 3), ("tiny", 300, 2), ("v4_hash_t64", 64, 2)]
+CASES = [("v4_decode_t16", 16, 4), ("gshard_c", 700, 3), ("tiny", 300, 2), ("v4_hash_t16", 16, 2)]
 WEIGHTS = ("W_gate", "W_up", "W_down")
 
 
@@ -64,13 +66,16 @@ def test_expert_range_partials_sum_to_the_layer(name, T, R):
     ref = PAR.reference_selection(cfg, cpu, routes[0]["topk_idx"], routes[0]["scores"])
     PAR.check_routing(cfg, ref, routes[0], T)
     shared = [(cpu["Ws_gate"][i], cpu["Ws_up"][i], cpu["Ws_down"][i]) for i in range(cfg.n_shared)]
+    all_experts = {e: (cpu["W_gate"][e], cpu["W_up"][e], cpu["W_down"][e]) for e in np.unique(ref["idx"])}
+    h_ref = EP.gather_partial(cpu["x"], ref["idx"], ref["gates"], all_experts, range(N), shared)
+    rms_h = np.sqrt(np.mean(h_ref ** 2))
     worst = 0.0
     for r, (e0, e1, h32) in enumerate(parts):
         local = {e: (cpu["W_gate"][e], cpu["W_up"][e], cpu["W_down"][e]) for e in range(e0, e1)
                  if (ref["idx"] == e).any()}
         p_ref = EP.gather_partial(cpu["x"], ref["idx"], ref["gates"], local, range(e0, e1),
                                   shared if r == 0 else None)
-        err = np.abs(h32.cpu().numpy().astype(np.float64) - p_ref).max() / np.sqrt(np.mean(p_ref ** 2))
+        err = np.abs(h32.cpu().numpy().astype(np.float64) - p_ref).max() / rms_h
         worst = max(worst, float(err))
     total = parts[0][2].clone()
     for _, _, h32 in parts[1:]:
@@ -82,7 +87,7 @@ def test_expert_range_partials_sum_to_the_layer(name, T, R):
     probe.close()
     assert torch.equal(h, total.to(torch.bfloat16))  # round to nearest even, as torch does
     hh = PAR.check_h(cfg, cpu, ref, dict(h=h), np.arange(T))
-    print(name, R, "worst partial err/RMS", worst, hh)
+    print(name, R, "worst partial err / RMS(h)", worst, hh)
     assert worst <= PAR.H_TOL
 
 

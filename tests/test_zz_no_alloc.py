@@ -80,14 +80,15 @@ def test_noalloc_routing_matches_oracle(name, T):
         print(name, "call", call, "near-tie tokens", n_near, "gate err", gerr, "P err", perr)
     # the forward's routing (its own workspace and kernels) picks the same experts where
     # the oracle's keys leave the margin
-    fw_cpu = W.make_inputs(cfg, seed=0, device="cuda", T=T)
-    layer = M.DSMoE(M.cfg_from(cfg, T), fw_cpu)
-    ref = layer.forward(fw_cpu["x"])
+    fw = W.make_inputs(cfg, seed=0, device="cuda", T=T)  # expert weights (routing does not read them)
+    fw.update({k: gpu[k] for k in ("x", "W_router", "b")})
+    layer = M.DSMoE(M.cfg_from(cfg, T), fw)
+    ref = layer.forward(fw["x"])
     torch.cuda.synchronize()
     layer.close()
     cl = torch.as_tensor(clean, device="cuda")
     assert torch.equal(topk[cl], ref["topk_idx"][cl])
-    del fw_cpu
+    del fw
 
 
 def test_noalloc_rejects_sizes_beyond_its_limits():
