@@ -254,8 +254,9 @@ dsmoe_status dsmoe_set_wait_limit(dsmoe_handle* h, uint64_t ns);
  * shared-expert layer equation). Both accumulate each output in fp32 over K in
  * 16-element MMA steps, in the same order, and share the epilogue arithmetic.
  *   DSMOE_GEMM_SINGLE (default) one CTA per tile, M=128 MMAs, tiles of up to 128 tokens.
- *   DSMOE_GEMM_PAIR   CTA pairs on neighbouring SMs share one M=256 MMA per K step,
- *                     tiles of up to 256 tokens.
+ *   DSMOE_GEMM_PAIR   CTA pairs on neighbouring SMs with M=256 MMAs (tcgen05 cta_group::2)
+ *                     and tiles of up to 256 tokens: gate/up as two chains (gate, up) of
+ *                     256 features sharing the token operand, down as 256 output rows.
  * dsmoe_set_gemm_kernel returns DSMOE_ERR_UNSUPPORTED when the pair kernel cannot be
  * launched on the device (the handle keeps its kind), and DSMOE_ERR_INVALID_ARG for
  * another kind. dsmoe_get_gemm_kernel returns the kind in use (-1 for a NULL handle). */

@@ -221,8 +221,8 @@ struct dsmoe_handle {
   int64_t async_calls = 0;
   CUtensorMap tm_xp, tm_a1, tm_a1s;
   // weight maps, cached per pointer: W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, W_router
-  // for the one-CTA GEMM and the router, then the six expert weights for the pair GEMM
-  static constexpr int kMaps = 13;
+  // (the gate/up maps serve both GEMM kernels), then W_down and Ws_down for the pair down GEMM
+  static constexpr int kMaps = 9;
   const void* wkey[kMaps] = {};
   int wkey_n[kMaps] = {};  // experts each cached routed map spans
   CUtensorMap tm_w[kMaps];
@@ -342,7 +342,7 @@ DSMOE_EXPORT dsmoe_status dsmoe_create(const dsmoe_cfg* cfg, int32_t device, dsm
   h->k_active = h->cfg.top_k;
   h->e_end = h->cfg.n_routed;
   h->num_sms = prop.multiProcessorCount;
-  h->pair_clusters[0] = dsmoe::grouped_gemm_pair_max_clusters(false);
+  h->pair_clusters[0] = dsmoe::down_pair_max_clusters();
   h->pair_clusters[1] = dsmoe::gateup_pair_max_clusters();
   dsmoe::router_tc_shape(cfg->n_routed, &h->rt_chunks, &h->rt_nc, &h->rt_cols);
   h->L = plan(h->cfg);
@@ -494,14 +494,8 @@ const CUtensorMap* weight_map(dsmoe_handle* h, int which, const void* ptr, bool*
       case 4: r = map_3d(&h->tm_w[which], ptr, c.d_model, c.d_ff_shared, c.n_shared, 128); break;
       case 5: r = map_3d(&h->tm_w[which], ptr, c.d_ff_shared, c.d_model, c.n_shared, 256); break;
       case 6: r = map_2d(&h->tm_w[which], ptr, c.d_model, c.n_routed, static_cast<uint32_t>(h->rt_nc)); break;
-      case 7:
-      case 8: r = map_3d(&h->tm_w[which], ptr, c.d_model, c.d_ff, n_local, dsmoe::kGemmPairGateUpRows); break;
-      case 9: r = map_3d(&h->tm_w[which], ptr, c.d_ff, c.d_model, n_local, 128); break;
-      case 10:
-      case 11:
-        r = map_3d(&h->tm_w[which], ptr, c.d_model, c.d_ff_shared, c.n_shared, dsmoe::kGemmPairGateUpRows);
-        break;
-      case 12: r = map_3d(&h->tm_w[which], ptr, c.d_ff_shared, c.d_model, c.n_shared, 128); break;
+      case 7: r = map_3d(&h->tm_w[which], ptr, c.d_ff, c.d_model, n_local, 128); break;
+      case 8: r = map_3d(&h->tm_w[which], ptr, c.d_ff_shared, c.d_model, c.n_shared, 128); break;
     }
     if (!r) {
       h->wkey[which] = nullptr;
@@ -728,7 +722,7 @@ dsmoe_status gemm_stage(dsmoe_handle* h, const GemmPlan& p, cudaStream_t s,
     if (bound > 0) {
       if (pair) {
         const int clusters = static_cast<int>(bound < h->pair_clusters[0] ? bound : h->pair_clusters[0]);
-        CUDA_TRY(dsmoe::launch_grouped_gemm_pair(false, g, clusters, s));
+        CUDA_TRY(dsmoe::launch_down_pair(g, clusters, s));
       } else {
         const int grid = static_cast<int>(bound < h->num_sms ? bound : h->num_sms);
         CUDA_TRY(dsmoe::launch_grouped_gemm(false, g, grid, s));
@@ -794,10 +788,10 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
   GemmPlan p;
   p.wg = weight_map(h, 0, a.W_gate, &ok);
   p.wu = weight_map(h, 1, a.W_up, &ok);
-  p.wd = weight_map(h, pair ? 9 : 2, a.W_down, &ok);
+  p.wd = weight_map(h, pair ? 7 : 2, a.W_down, &ok);
   p.swg = Ks ? weight_map(h, 3, a.Ws_gate, &ok) : p.wg;
   p.swu = Ks ? weight_map(h, 4, a.Ws_up, &ok) : p.wu;
-  p.swd = Ks ? weight_map(h, pair ? 12 : 5, a.Ws_down, &ok) : p.wd;
+  p.swd = Ks ? weight_map(h, pair ? 8 : 5, a.Ws_down, &ok) : p.wd;
   CUtensorMap m_x;  // token rows of x in GEMM tiles (shared groups)
   ok = ok && map_2d(&m_x, a.x, d, T, dsmoe::kGemmGateUpTokenTile);
   if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map of this call");
@@ -1039,7 +1033,7 @@ DSMOE_EXPORT dsmoe_status dsmoe_ep_experts(dsmoe_handle* h, int32_t n_src, int32
   GemmPlan p;
   p.wg = weight_map(h, 0, W_gate, &ok, n_local);
   p.wu = weight_map(h, 1, W_up, &ok, n_local);
-  p.wd = weight_map(h, pair ? 9 : 2, W_down, &ok, n_local);
+  p.wd = weight_map(h, pair ? 7 : 2, W_down, &ok, n_local);
   p.swg = p.wg;
   p.swu = p.wu;
   p.swd = p.wd;
@@ -1085,7 +1079,7 @@ DSMOE_EXPORT dsmoe_status dsmoe_ep_combine(dsmoe_handle* h, int32_t T, const voi
     GemmPlan p;
     p.swg = weight_map(h, 3, Ws_gate, &ok);
     p.swu = weight_map(h, 4, Ws_up, &ok);
-    p.swd = weight_map(h, pair ? 12 : 5, Ws_down, &ok);
+    p.swd = weight_map(h, pair ? 8 : 5, Ws_down, &ok);
     p.wg = p.swg;
     p.wu = p.swu;
     p.wd = p.swd;

@@ -1,27 +1,17 @@
-// gemm_pair_sm100.cu -- the grouped expert GEMMs on CTA pairs (tcgen05 cta_group::2).
+// gemm_pair_sm100.cu -- the down projection of the grouped expert GEMMs on CTA pairs
+// (tcgen05 cta_group::2); the gate/up projection's pair kernel is gemm_gateup_pair_sm100.cu.
 //
-// Same contractions, groups and tile order as gemm_sm100.cu (DeepSeekMoE summary,
-// shared-expert layer equation; SwiGLU form noted on the "MoE: sparse activation" page):
-//   gate/up:  A1[r, n] = SiLU(sum_k X[r,k] W_gate[e,n,k]) * (sum_k X[r,k] W_up[e,n,k])
-//   down:     Y[r, n]  = sum_k A1[r,k] W_down[e,n,k]
+// Same contraction, groups and tile order as gemm_sm100.cu (DeepSeekMoE summary,
+// shared-expert layer equation):   Y[r, n] = sum_k A1[r,k] W_down[e,n,k]
 // but each tile is computed by a cluster of two CTAs on neighbouring SMs with one M=256
 // MMA per K step (weights on M, tokens on N, N = the tile's token count rounded up to
 // 16, at most 256). Each SM stages only its own 128 weight rows and half of the token
-// rows, so per MAC it reads half the shared-memory operand bytes of a one-CTA M=128,
-// N=128 MMA. Its outputs are bit-identical to the one-CTA kernel's. On B200 it halves
-// the tensor core's shared-memory read traffic but is not faster than the one-CTA
-// kernel, which therefore stays the default: both are bound by the latency of their
-// operand loads, not by that port.
+// rows, so per MAC it stages and reads half the operand bytes of a one-CTA M=128, N=128
+// MMA. Its outputs are bit-identical to the one-CTA kernel's.
 //
-// Tile of a pair (even CTA = rank 0, odd = rank 1):
-//   gate/up: 128 output features f0..f0+127; rank r holds the 64 gate rows and then
-//            the 64 up rows of features f0+64r..f0+64r+63 (two TMA boxes), so TMEM lanes
-//            0-63 hold gate and 64-127 up values: the epilogue warps reading lanes
-//            [32p, 32p+32) and [64+32p, 96+32p) hold the gate and up halves of the same
-//            32 features and trade half of their tokens through shared memory.
-//   down:    256 output rows; rank r holds rows 128r..128r+127 of the tile.
-//   tokens:  rank 0 stages token rows row0.., rank 1 rows row0+N/2.. (the MMA's B
-//            columns N/2..N-1 come from the odd CTA).
+// Tile of a pair (even CTA = rank 0, odd = rank 1): 256 output rows, rank r holds rows
+// 128r..128r+127; token rows: rank 0 stages row0.., rank 1 row0+N/2.. (the MMA's B
+// columns N/2..N-1 come from the odd CTA).
 //
 // Roles (192 threads per CTA):
 //   warp 0     TMA producer of this CTA's half of every stage (6 stages of 32 KB); all
@@ -33,8 +23,8 @@
 //   warps 2-5  epilogue of this CTA's 128 accumulator rows; one lane per warp releases
 //              the accumulator on the even CTA's `acc_empty` barrier.
 // Every wait is bounded; a role that gives up raises the abort flag of both CTAs and a
-// status bit. At the end the even CTA waits (bounded) for every copy either CTA issued
-// and for its MMAs, and only then may either CTA release TMEM and exit.
+// status bit. At the end the even CTA waits (at least one second) for every copy either
+// CTA issued and for its MMAs, and only then may either CTA release TMEM and exit.
 #include "grouped_tiles.cuh"
 #include "sm100_pair_ptx.cuh"
 
@@ -54,30 +44,21 @@ constexpr int kStages = 6;
 constexpr int kBufs = 2;
 constexpr uint32_t kAccCols = kTok;
 constexpr uint32_t kStageRow = 33;
-constexpr int kGU = kGemmPairGateUpRows;  // rows per gate or up box
 
 constexpr uint32_t kOffA = 0;
 constexpr uint32_t kOffB = kOffA + kStages * kABytes;
 constexpr uint32_t kOffBars = kOffB + kStages * kBBytes;
-// landed, empty, acc_full, acc_empty, drain, and the gate/up exchange [2 slots][2 pairs]
-constexpr uint32_t kNumBars = 2 * kStages + 2 * kBufs + 1 + 4;
+// landed, empty, acc_full, acc_empty, drain
+constexpr uint32_t kNumBars = 2 * kStages + 2 * kBufs + 1;
 constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;      // tmem slot, abort, never, pad, issued[kStages]
 constexpr uint32_t kOffTiles = (kOffMisc + 16 + kStages * 4 + 15) & ~15u;
 constexpr uint32_t kOffEpi = (kOffTiles + (kGemmMaxGroups + 1) * 4 + 15) & ~15u;
-// epilogue scratch. down: per warp a 32 x 33 fp32 transpose tile. gate/up: the gate/up
-// exchange, [2 chunk buffers][2 warp pairs][2 directions][16 tokens][32 lanes] fp32,
-// then per warp a 16 x 33 transpose tile.
-constexpr uint32_t kXchgBytes = 2 * 2 * 2 * 16 * 32 * 4;
-constexpr uint32_t kEpiDown = 4 * 32 * kStageRow * 4;
-constexpr uint32_t kEpiGateUp = kXchgBytes + 4 * 16 * kStageRow * 4;
-constexpr uint32_t kSmemUsed = kOffEpi + (kEpiDown > kEpiGateUp ? kEpiDown : kEpiGateUp);
+constexpr uint32_t kSmemUsed = kOffEpi + 4 * 32 * kStageRow * 4;  // per warp a 32 x 33 fp32 transpose tile
 constexpr size_t kSmemBytes = kSmemUsed + 1024;  // slack to align the ring to 1024 bytes
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kBufs * kAccCols <= kTmemCols, "TMEM budget");
-static_assert(2 * kGU == kRowsPerCta, "gate/up rows per CTA");
 
-template <bool kSwiGLU>
-__global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair_kernel(const __grid_constant__ GemmArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) down_pair_kernel(const __grid_constant__ GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_addr(smem_raw) & 1023u)) & 1023u;
   uint8_t* base = smem_raw + pad;
@@ -89,7 +70,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair_kernel(const __
   uint64_t* acc_full = bars + 2 * kStages;
   uint64_t* acc_empty = acc_full + kBufs;
   uint64_t* drain = acc_empty + kBufs;
-  uint64_t* xbar = drain + 1;  // [slot][pair]: one lane of each warp of the pair arrives
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + kOffMisc + 4);
   volatile int* never_flag = reinterpret_cast<volatile int*>(base + kOffMisc + 8);
@@ -116,7 +96,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair_kernel(const __
       mbar_init(&acc_empty[i], 2 * 4);  // one lane of each epilogue warp of both CTAs
     }
     mbar_init(drain, 1);
-    for (int i = 0; i < 4; ++i) mbar_init(&xbar[i], 2);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -138,7 +117,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair_kernel(const __
       // ------------------------------------------------------------------ TMA producer
       tma_prefetch_desc(&a.a_routed);
       tma_prefetch_desc(&a.b0_routed);
-      if (kSwiGLU) tma_prefetch_desc(&a.b1_routed);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -148,7 +126,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair_kernel(const __
         const int brow = t.row0 + (even ? 0 : n_mma / 2);
         const CUtensorMap* tx = t.shared ? &a.a_shared : &a.a_routed;
         const CUtensorMap* tw0 = t.shared ? &a.b0_shared : &a.b0_routed;
-        const CUtensorMap* tw1 = t.shared ? &a.b1_shared : &a.b1_routed;
         const int kb_per = t.shared ? a.kb_per_b_expert_shared : t.kb_n;
         for (int kb = 0; kb < t.kb_n; ++kb) {
           if (!pair::mbar_wait_bounded_cl(&empty[stage], phase ^ 1u, a.wait_limit_ns, abort_flag)) {
@@ -159,15 +136,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair_kernel(const __
           if (even) mbar_arrive_expect_tx(&landed[stage], 2 * kStageBytes);
           const int be = t.expert + kb / kb_per;
           const int bk = (kb % kb_per) * kBK;
-          uint8_t* sa = sA + stage * kABytes;
-          if (kSwiGLU) {  // [64 gate rows | 64 up rows] of features f0 .. f0+63
-            const int f0 = t.n_blk * 2 * kGU + static_cast<int>(rank) * kGU;
-            pair::tma_load_3d_pair(sa, tw0, bar, bk, f0, be);
-            pair::tma_load_3d_pair(sa + kGU * 128, tw1, bar, bk, f0, be);
-          } else {  // 128 consecutive output rows
-            pair::tma_load_3d_pair(sa, tw0, bar, bk, t.n_blk * 2 * kRowsPerCta + static_cast<int>(rank) * kRowsPerCta,
-                                   be);
-          }
+          uint8_t* sa = sA + stage * kABytes;  // 128 consecutive output rows
+          pair::tma_load_3d_pair(sa, tw0, bar, bk, t.n_blk * 2 * kRowsPerCta + static_cast<int>(rank) * kRowsPerCta, be);
           pair::tma_load_2d_pair(sB + stage * kBBytes, tx, bar, kb * kBK, brow);
           issued_n[stage] += 1;
           if (++stage == kStages) {
@@ -233,7 +203,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair_kernel(const __
     const int q = warp & 3;  // this warp may read TMEM lanes [32q, 32q+32)
     float* stg = reinterpret_cast<float*>(base + kOffEpi) + q * 32 * kStageRow;
     int it = 0;
-    uint32_t n_xchg = 0;  // gate/up exchanges done by this warp (slot = n & 1, parity = (n >> 1) & 1)
     bool ok = true;
     for (int tile = pair_id; ok && tile < total; tile += n_pairs, ++it) {
       const Tile t = decode_tile<kTok>(a, tile_start, G, tile);
@@ -246,66 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair_kernel(const __
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
       const int n_valid = t.shared ? a.n_valid_shared : a.n_valid_routed;
       const int64_t ld = t.shared ? a.ld_shared : a.ld_routed;
-      if (kSwiGLU) {
-        // Warp pair p (TMEM lanes 32p.. gate, 64+32p.. up) owns features feat0 + lane.
-        // Per 32 tokens the gate warp produces tokens 0-15 and the up warp tokens 16-31:
-        // each hands the other half of its values over through shared memory (an
-        // mbarrier per exchange slot, bounded waits; slots alternate, so a slot is
-        // rewritten only after the partner's arrival on the other slot, which follows
-        // its read of this one), then each warp transposes its 16 tokens x 32 features
-        // and lane L stores 8 features (16 bytes) of token L/4 and of token 8 + L/4.
-        const int p = q & 1;
-        const bool is_gate = q < 2;
-        const int feat0 = t.n_blk * 2 * kGU + static_cast<int>(rank) * kGU + p * 32;
-        float* xchg = reinterpret_cast<float*>(base + kOffEpi);
-        float* stg16 = xchg + kXchgBytes / 4 + q * 16 * kStageRow;
-        bf16* obase = t.shared ? a.out_shared + static_cast<int64_t>(t.group) * a.shared_col_stride : a.out_routed;
-        const int rr = lane >> 2, cc = (lane & 3) * 8;
-        const bool ok_f = feat0 + cc < n_valid;  // n_valid is a multiple of 64, feat0 + cc of 8
-        const int tok_off = is_gate ? 0 : 16;
-#pragma unroll 1
-        for (int c0 = 0; c0 < t.m_valid; c0 += 32, ++n_xchg) {
-          uint32_t v[32];
-          tmem_ld16(tb + c0, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
-          tmem_ld16(tb + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
-          tmem_wait_ld();
-          // [slot][pair][direction: 0 = gate values sent, 1 = up values sent][16][32]
-          const int sl = static_cast<int>(n_xchg & 1u);
-          float* slot = xchg + (sl * 4 + p * 2) * 16 * 32;
-          float* mine = slot + (is_gate ? 0 : 16 * 32);
-          const float* theirs = slot + (is_gate ? 16 * 32 : 0);
-#pragma unroll
-          for (int j = 0; j < 16; ++j)  // gate sends tokens 16-31, up sends tokens 0-15
-            mine[j * 32 + lane] = __uint_as_float(is_gate ? v[16 + j] : v[j]);
-          __syncwarp();  // the warp's writes are ordered before its one arrival
-          if (lane == 0) mbar_arrive(&xbar[sl * 2 + p]);
-          if (!mbar_wait_warp(&xbar[sl * 2 + p], (n_xchg >> 1) & 1u, a.wait_limit_ns, abort_flag)) {
-            ok = false;
-            break;
-          }
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float other = theirs[j * 32 + lane];
-            const float g = is_gate ? __uint_as_float(v[j]) : other;
-            const float u = is_gate ? other : __uint_as_float(v[16 + j]);
-            stg16[j * kStageRow + lane] = __fdividef(g, 1.0f + __expf(-g)) * u;  // SiLU(g) * u
-          }
-          __syncwarp();
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int tt = rr + 8 * i;  // token of this warp's half
-            const int tok = c0 + tok_off + tt;
-            if (ok_f && tok < t.m_valid) {
-              const float* src = stg16 + tt * kStageRow + cc;
-              *reinterpret_cast<uint4*>(obase + static_cast<int64_t>(t.row0 + tok) * ld + feat0 + cc) =
-                  make_uint4(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
-                             pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
-            }
-          }
-          __syncwarp();
-        }
-        if (!ok) break;
-      } else {
+      {
         // thread of TMEM lane l holds output row feat_base + l; per 32 tokens the warp
         // transposes its 32 rows x 32 tokens and lane L stores 8 consecutive outputs of
         // token L/4 + 8i (16 B of bf16, or 32 B of fp32 with the residual added)
@@ -395,7 +305,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair_kernel(const __
   }
 }
 
-template <bool kSwiGLU>
 cudaLaunchConfig_t pair_config(int clusters, cudaStream_t s, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters, 1, 1);
@@ -410,39 +319,31 @@ cudaLaunchConfig_t pair_config(int clusters, cudaStream_t s, cudaLaunchAttribute
   cfg.numAttrs = 1;
   return cfg;
 }
+}  // namespace
 
-template <bool kSwiGLU>
-int max_clusters() {
-  if (cudaFuncSetAttribute(grouped_gemm_pair_kernel<kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+int down_pair_max_clusters() {
+  if (cudaFuncSetAttribute(down_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(kSmemBytes)) != cudaSuccess)
     return 0;
   cudaLaunchAttribute attr;
-  cudaLaunchConfig_t cfg = pair_config<kSwiGLU>(1, nullptr, &attr);
+  cudaLaunchConfig_t cfg = pair_config(1, nullptr, &attr);
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_pair_kernel<kSwiGLU>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, down_pair_kernel, &cfg) != cudaSuccess) {
     (void)cudaGetLastError();
     return 0;
   }
   return n;
 }
 
-template <bool kSwiGLU>
-cudaError_t launch(const GemmArgs& a, int clusters, cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+cudaError_t launch_down_pair(const GemmArgs& a, int clusters, cudaStream_t s) {
+  if (a.n_shared_groups + a.n_routed > kGemmMaxGroups) return cudaErrorInvalidValue;
+  if (clusters < 1) clusters = 1;
+  cudaError_t e = cudaFuncSetAttribute(down_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr;
-  cudaLaunchConfig_t cfg = pair_config<kSwiGLU>(clusters, s, &attr);
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<kSwiGLU>, a);
-}
-}  // namespace
-
-int grouped_gemm_pair_max_clusters(bool swiglu) { return swiglu ? max_clusters<true>() : max_clusters<false>(); }
-
-cudaError_t launch_grouped_gemm_pair(bool swiglu, const GemmArgs& a, int clusters, cudaStream_t s) {
-  if (a.n_shared_groups + a.n_routed > kGemmMaxGroups) return cudaErrorInvalidValue;
-  if (clusters < 1) clusters = 1;
-  return swiglu ? launch<true>(a, clusters, s) : launch<false>(a, clusters, s);
+  cudaLaunchConfig_t cfg = pair_config(clusters, s, &attr);
+  return cudaLaunchKernelEx(&cfg, down_pair_kernel, a);
 }
 
 }  // namespace dsmoe

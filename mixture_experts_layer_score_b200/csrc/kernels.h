@@ -240,16 +240,14 @@ struct GemmBwdArgs {
 };
 cudaError_t launch_grouped_gemm_bwd(int mode, const GemmBwdArgs& a, int grid, cudaStream_t s);
 
-// The same grouped GEMM on CTA pairs (clusters of two, tcgen05 cta_group::2): a pair
-// computes 128 features (gate/up) or 256 output rows (down) by up to
-// kGemmPairTokenTile tokens; each CTA stages 128 weight rows and half of the tile's
-// token rows. Weight maps: box (64, kGemmPairGateUpRows) for gate/up, (64, 128) for
-// down; token maps: box (64, 128).
+// The down projection on CTA pairs (gemm_pair_sm100.cu; clusters of two, tcgen05
+// cta_group::2): a pair computes 256 output rows by up to kGemmPairTokenTile tokens; each
+// CTA stages 128 weight rows and half of the tile's token rows. Weight maps: box
+// (64, 128); token maps: box (64, 128).
 constexpr int kGemmPairTokenTile = 256;
-constexpr int kGemmPairGateUpRows = 64;
 // Largest number of co-resident pairs (0 when the pair kernel cannot be launched).
-int grouped_gemm_pair_max_clusters(bool swiglu);
-cudaError_t launch_grouped_gemm_pair(bool swiglu, const GemmArgs& a, int clusters, cudaStream_t s);
+int down_pair_max_clusters();
+cudaError_t launch_down_pair(const GemmArgs& a, int clusters, cudaStream_t s);
 
 // The gate/up projection on CTA pairs with two M=256 chains (gemm_gateup_pair_sm100.cu):
 // tiles of 256 features by up to kGemmPairTokenTile tokens; weight maps box (64, 128)

@@ -22,6 +22,8 @@ Shapes follow the configurations the DeepSeekMoE pages describe:
   scores (V4 book ch. 2, section 2 equation) with a selection-only bias.
 * ``v4_hash_t{16,64,256}``: hash-routed layer (V4 book ch. 2, section 5),
   expert = token_id * 2654435761 mod 384.
+* ``v4_decode_slice``: the V4 decode shapes (T=16) with 48 routed experts, a small case
+  for profiler captures of the weight-streaming GEMMs.
 
 Values: x ~ N(0,1); expert weights ~ N(0, 1/fan_in); router weights
 ~ N(0, 1/d) unless the configuration fixes N(0, 0.02^2); bias ~ U(-0.1, 0.1).
@@ -122,6 +124,9 @@ def _cfgs():
         c[f"v4_hash_t{t}"] = MoEConfig(f"v4_hash_t{t}", T=t, d_model=7168, n_routed=384,
                                        top_k=1, d_ff=2048, n_shared=1, d_ff_shared=2048,
                                        score=ROUTE_HASH)
+    # the V4 decode layer's matrix shapes with 48 of its routed experts (4.3 GB of weights):
+    # a small case for profiler captures of the weight-streaming GEMMs
+    c["v4_decode_slice"] = c["v4_decode_t16"].replace(name="v4_decode_slice", n_routed=48)
     return c
 
 
