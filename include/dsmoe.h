@@ -410,9 +410,28 @@ dsmoe_status dsmoe_backward_gates(dsmoe_handle* h, int32_t T, const void* dh, co
  *                                    residual, shared-expert and routed-expert parts of dL/du
  *   Two grouped GEMMs on the tensor cores (the weights read MN-major, in the forward's
  *   layout) and one combine; fp32 accumulation, da | db and the per-slot du rows stored
- *   as bf16, the shared experts' du summed in fp32. The weight gradients are not computed
- *   here.
+ *   as bf16, the shared experts' du summed in fp32. The weight gradients are computed by
+ *   dsmoe_backward_weights.
  */
+/*
+ * dsmoe_backward_weights -- the experts' weight gradients, after dsmoe_backward_experts
+ * for the last training forward (same T, else DSMOE_ERR_INVALID_ARG):
+ *   dW_down = sum_r dy_r m_r^T, dW_gate = sum_r da_r u_r^T, dW_up = sum_r db_r u_r^T
+ * summed over the rows r each expert applied to (routed: its picks' slots, with
+ * dy = g dh; shared: every token, dy = dh), from the forward's saved m (A1) and gathered
+ * rows u, and the da | db of dsmoe_backward_experts:
+ *     dh, dY, x          bf16, as given to the forward and dsmoe_backward_experts
+ *     dW_gate, dW_up     fp32 [N_local, F, d] out   (N_local = the handle's expert range)
+ *     dW_down            fp32 [N_local, d, F] out
+ *     dWs_gate, dWs_up   fp32 [K_s, F_s, d] out, dWs_down fp32 [K_s, d, F_s] out
+ *                        (all three NULL iff the handle adds no shared experts)
+ *   Grouped GEMMs on the tensor cores reducing over token rows (both operands MN-major,
+ *   each routed expert's rows a ragged K range), fp32 accumulation of bf16 products.
+ *   An expert no token picked gets a zero gradient.
+ */
+dsmoe_status dsmoe_backward_weights(dsmoe_handle* h, int32_t T, const void* dh, const void* dY, const void* x,
+                                    float* dW_gate, float* dW_up, float* dW_down, float* dWs_gate, float* dWs_up,
+                                    float* dWs_down, void* stream);
 dsmoe_status dsmoe_set_training(dsmoe_handle* h, int32_t enable);
 dsmoe_status dsmoe_backward_experts(dsmoe_handle* h, int32_t T, const void* dh, const void* dY, const void* W_gate,
                                     const void* W_up, const void* W_down, const void* Ws_gate, const void* Ws_up,

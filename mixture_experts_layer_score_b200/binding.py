@@ -32,7 +32,7 @@ ABI_FUNCTIONS = (
     "dsmoe_set_selection", "dsmoe_get_selection", "dsmoe_set_expert_range", "dsmoe_get_expert_range",
     "dsmoe_round_bf16", "dsmoe_backward_gates", "dsmoe_backward_router", "dsmoe_ep_route", "dsmoe_ep_experts",
     "dsmoe_ep_combine", "dsmoe_forward_host_async", "dsmoe_host_join", "dsmoe_host_sync", "dsmoe_set_training",
-    "dsmoe_backward_experts",
+    "dsmoe_backward_experts", "dsmoe_backward_weights",
 )
 
 
@@ -72,6 +72,7 @@ def _load():
         "dsmoe_host_sync": (ctypes.c_int, [vp]),
         "dsmoe_set_training": (ctypes.c_int, [vp, i32]),
         "dsmoe_backward_experts": (ctypes.c_int, [vp, i32] + [vp] * 10 + [vp]),
+        "dsmoe_backward_weights": (ctypes.c_int, [vp, i32] + [vp] * 9 + [vp]),
         "dsmoe_balance_stats": (ctypes.c_int, [vp, i64, vp, vp, vp, vp, vp]),
         "dsmoe_get_status": (ctypes.c_int, [vp]),
         "dsmoe_set_wait_limit": (ctypes.c_int, [vp, u64]),
@@ -290,6 +291,13 @@ def dsmoe_backward_experts(handle, T, dh, dY, W_gate, W_up, W_down, Ws_gate, Ws_
     _check(_lib.dsmoe_backward_experts(handle, int(T), *[_ptr(t) for t in (
         dh, dY, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, dx_add, dx)], _stream(stream)),
         "dsmoe_backward_experts")
+
+
+def dsmoe_backward_weights(handle, T, dh, dY, x, dW_gate, dW_up, dW_down, dWs_gate, dWs_up, dWs_down,
+                           stream=None) -> None:
+    _check(_lib.dsmoe_backward_weights(handle, int(T), *[_ptr(t) for t in (
+        dh, dY, x, dW_gate, dW_up, dW_down, dWs_gate, dWs_up, dWs_down)], _stream(stream)),
+        "dsmoe_backward_weights")
 
 
 def dsmoe_backward_gates(handle, T, dh, gates, dg, dY, stream=None) -> None:

@@ -107,6 +107,21 @@ bool map_4d_mn(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, ui
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3D bf16 view (64, rows, cols / 64) of a [rows, cols] buffer (cols contiguous), 128-byte
+// swizzle, box (64, 64, atoms): one copy lands 64 rows x 64*atoms columns as MN-major
+// atoms (the weight-gradient GEMMs' operands, reduced over rows).
+bool map_view_mn(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t atoms) {
+  auto enc = tensor_map_encoder();
+  if (!enc || cols % 64 || rows == 0) return false;
+  cuuint64_t dims[3] = {64, rows, cols / 64};
+  cuuint64_t strides[2] = {cols * 2, 128};
+  cuuint32_t box[3] = {64, 64, atoms};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct DeviceGuard {
   int prev = -1, want;
   bool ok = false;
@@ -239,6 +254,7 @@ struct dsmoe_handle {
   bf16 *AB = nullptr, *ABs = nullptr, *dAB = nullptr, *dABs = nullptr, *dXp = nullptr;
   float* dXs = nullptr;
   int32_t saved_T = -1;  // tokens of the last forward that saved a | b
+  bool dab_ready = false;  // da | db of that forward computed (dsmoe_backward_experts)
 };
 
 // ========================================================================================
@@ -814,7 +830,10 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
   p.Y_out = h->Y;
   p.save_ab = h->tr != nullptr;
   STAGE_TRY(gemm_stage(h, p, s, mark));
-  if (h->tr) h->saved_T = T;
+  if (h->tr) {
+    h->saved_T = T;
+    h->dab_ready = false;
+  }
   STAGE_TRY(combine_stage(h, a, h->Y, Ks, h->add_shared, h->partial, s));
   CUDA_TRY(mark(7));
   if (timing) h->timed_forwards += 1;
@@ -1442,6 +1461,84 @@ DSMOE_EXPORT dsmoe_status dsmoe_backward_experts(dsmoe_handle* h, int32_t T, con
   }
   CUDA_TRY(dsmoe::launch_dx_combine(static_cast<const bf16*>(dh), Ks ? h->dXs : nullptr, dx_add, h->dXp, h->slot_of,
                                     T, K, d, dx, h->num_sms, s));
+  h->launches += 3;
+  h->dab_ready = true;
+  return DSMOE_OK;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_backward_weights(dsmoe_handle* h, int32_t T, const void* dh, const void* dY,
+                                                 const void* x, float* dW_gate, float* dW_up, float* dW_down,
+                                                 float* dWs_gate, float* dWs_up, float* dWs_down, void* stream) {
+  if (!h) return fail(DSMOE_ERR_INVALID_ARG, "handle is NULL");
+  const dsmoe_cfg& c = h->cfg;
+  if (!h->tr) return fail(DSMOE_ERR_INVALID_ARG, "training buffers are not enabled (dsmoe_set_training)");
+  if (T != h->saved_T || T <= 0 || !h->dab_ready)
+    return fail(DSMOE_ERR_INVALID_ARG,
+                "call after dsmoe_backward_experts for the last training forward (T = %d, forward T = %d)", T,
+                h->saved_T);
+  const int Ks = h->add_shared ? c.n_shared : 0;
+  if (!dh || !dY || !x || !dW_gate || !dW_up || !dW_down || (Ks && (!dWs_gate || !dWs_up || !dWs_down)))
+    return fail(DSMOE_ERR_INVALID_ARG, "NULL argument");
+  const void* must_align[] = {dh, dY, x, dW_gate, dW_up, dW_down, dWs_gate, dWs_up, dWs_down};
+  for (const void* q : must_align)
+    if (q && !aligned16(q)) return fail(DSMOE_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", q);
+  DeviceGuard gd(h->device);
+  if (!gd.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int d = c.d_model, F = c.d_ff, Fs = c.d_ff_shared;
+  const int NL = h->e_end - h->e_begin;
+  // operand views: routed rows in slot order (the T K' rows this forward wrote; the
+  // copies read zeros past them), shared rows = the T tokens
+  const uint64_t S = static_cast<uint64_t>(T) * h->k_active, KsFs = static_cast<uint64_t>(Ks) * Fs;
+  CUtensorMap v_dY, v_A1, v_dAB, v_Xp, v_dh, v_A1s, v_dABs, v_x;
+  bool ok = map_view_mn(&v_dY, dY, S, d, 4) && map_view_mn(&v_A1, h->A1, S, F, 2) &&
+            map_view_mn(&v_dAB, h->dAB, S, 2 * static_cast<uint64_t>(F), 4) && map_view_mn(&v_Xp, h->Xp, S, d, 2);
+  if (Ks)
+    ok = ok && map_view_mn(&v_dh, dh, T, d, 4) && map_view_mn(&v_A1s, h->A1s, T, KsFs, 2) &&
+         map_view_mn(&v_dABs, h->dABs, T, 2 * KsFs, 4) && map_view_mn(&v_x, x, T, d, 2);
+  if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map of the weight gradients");
+  auto plan = [&](dsmoe::GemmDwArgs& g, int M, int N, int Ms, int Ns) {
+    memset(&g, 0, sizeof(g));
+    g.offsets = h->offsets + h->e_begin;
+    g.n_routed = NL;
+    g.n_shared = Ks;
+    g.T = T;
+    g.m_routed = M;
+    g.n_routed_cols = N;
+    g.m_shared = Ms;
+    g.n_shared_cols = Ns;
+    g.m_tiles_routed = cdiv(M, 256);
+    g.n_tiles_routed = cdiv(N, 128);
+    g.m_tiles_shared = Ks ? cdiv(Ms, 256) : 0;
+    g.n_tiles_shared = Ks ? cdiv(Ns, 128) : 0;
+    g.status = h->status;
+    g.wait_limit_ns = h->wait_ns;
+  };
+  // dW_down[e] = sum_r dy_r m_r^T: A = dY (d columns), B = A1 (F columns)
+  dsmoe::GemmDwArgs g;
+  plan(g, d, F, d, Fs);
+  g.a_routed = v_dY;
+  g.b_routed = v_A1;
+  g.a_shared = Ks ? v_dh : v_dY;
+  g.b_shared = Ks ? v_A1s : v_A1;
+  g.b_atom_step_shared = Fs / 64;
+  g.out_routed = dW_down;
+  g.out_shared = dWs_down;
+  CUDA_TRY(dsmoe::launch_grouped_dw(g, h->num_sms, s));
+  // dW_gate[e] = sum_r da_r u_r^T and dW_up[e] = sum_r db_r u_r^T: A = da | db, B = Xp (x)
+  for (int up = 0; up < 2; ++up) {
+    plan(g, F, d, Fs, d);
+    g.a_routed = v_dAB;
+    g.b_routed = v_Xp;
+    g.a_shared = Ks ? v_dABs : v_dAB;
+    g.b_shared = Ks ? v_x : v_Xp;
+    g.a_atom0_routed = up ? F / 64 : 0;
+    g.a_atom0_shared = up ? Fs / 64 : 0;
+    g.a_atom_step_shared = 2 * Fs / 64;
+    g.out_routed = up ? dW_up : dW_gate;
+    g.out_shared = up ? dWs_up : dWs_gate;
+    CUDA_TRY(dsmoe::launch_grouped_dw(g, h->num_sms, s));
+  }
   h->launches += 3;
   return DSMOE_OK;
 }

@@ -1,0 +1,334 @@
+// gemm_dw_sm100.cu -- the experts' weight gradients on the 5th-generation tensor cores.
+//
+// For an expert FFN y = W_down m, m = SiLU(a) * b, a = W_gate u, b = W_up u (DeepSeekMoE
+// summary, shared-expert layer equation; SwiGLU form noted on the "MoE: sparse
+// activation" page), summed over the rows r the expert applies to:
+//   dW_down = sum_r dy_r m_r^T,   dW_gate = sum_r da_r u_r^T,   dW_up = sum_r db_r u_r^T
+// i.e. D[i, j] = sum_r A[r, i] B[r, j] with the reduction over token rows, which are
+// contiguous in both operands' [rows, cols] layouts: both MMA operands are MN-major, and
+// each routed expert's K range is its segment of the slot order (ragged), each shared
+// expert's all T tokens.
+//
+// One CTA per SM, 192 threads: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
+// warps 2-5 epilogue. A tile is 256 output rows (two M=128 chains) by 128 output columns;
+// per 64-row K block the producer stages A (256 columns of the A buffer) and B (128
+// columns of the B buffer) through 3-D views (64, rows, cols / 64) that land as 64-element
+// MN-major swizzle-128B atoms 8 KB apart. A K block that runs past the group's last row
+// holds rows of the next group (or the buffer's zero fill): the MMA warp zeroes those rows
+// in shared memory (and makes the stores visible to the tensor core) before the MMAs. A
+// group with no rows gets a zero tile. Output fp32, D row-major per group.
+// Every wait is bounded; a role that gives up raises the abort flag and a status bit, the
+// CTA waits (at least one second) for its copies and MMAs in flight, frees TMEM, returns.
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace dsmoe {
+
+namespace {
+constexpr int kBK = 64;
+constexpr int kFeat = 128;
+constexpr int kMmaK = 16;
+constexpr int kThreads = 192;
+constexpr int kEpiThreads = 128;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kN = 128;                             // output columns per tile (the MMA's N)
+constexpr int kStages = 4;
+constexpr uint32_t kABytes = 2 * kFeat * kBK * 2;  // 32 KB: 256 output rows x 64 K rows
+constexpr uint32_t kBBytes = kN * kBK * 2;         // 16 KB: 128 output columns x 64 K rows
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr uint32_t kAccCols = 2 * kN;
+constexpr int kBufs = 2;
+constexpr uint32_t kStageRow = 33;
+constexpr uint32_t kAtom = kBK * 128;              // one 64-element atom column of a stage: 8 KB
+constexpr uint32_t kOffA = 0;
+constexpr uint32_t kOffB = kOffA + kStages * kABytes;
+constexpr uint32_t kOffBars = kOffB + kStages * kBBytes;
+constexpr uint32_t kNumBars = 2 * kStages + 2 * kBufs + 1;
+constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
+constexpr uint32_t kOffEpi = (kOffMisc + 16 + 15) & ~15u;
+constexpr uint32_t kSmemUsed = kOffEpi + 4 * 32 * kStageRow * 4;
+constexpr size_t kSmemBytes = kSmemUsed + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(kAtom >> 4) << 16;  // leading byte offset: next 64 MN elements
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;   // stride byte offset: next 8 K rows
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
+__device__ __forceinline__ void tma_load_3d_view(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t row,
+                                                 int32_t atom) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
+          smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(0), "r"(row), "r"(atom)
+      : "memory");
+}
+
+struct DwTile {
+  int group, shared, row0, rows, m_blk, n_blk;
+};
+
+__device__ __forceinline__ DwTile dw_decode(const GemmDwArgs& a, int tile) {
+  DwTile t;
+  const int tiles_s = a.m_tiles_shared * a.n_tiles_shared, tiles_r = a.m_tiles_routed * a.n_tiles_routed;
+  int local, n_tiles;
+  if (tile < a.n_shared * tiles_s) {
+    t.shared = 1;
+    t.group = tile / tiles_s;
+    local = tile - t.group * tiles_s;
+    n_tiles = a.n_tiles_shared;
+    t.row0 = 0;
+    t.rows = a.T;
+  } else {
+    t.shared = 0;
+    const int r = tile - a.n_shared * tiles_s;
+    t.group = r / tiles_r;
+    local = r - t.group * tiles_r;
+    n_tiles = a.n_tiles_routed;
+    t.row0 = a.offsets[t.group];
+    t.rows = max(a.offsets[t.group + 1] - t.row0, 0);
+  }
+  t.m_blk = local / n_tiles;
+  t.n_blk = local % n_tiles;
+  return t;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_constant__ GemmDwArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_addr(smem_raw) & 1023u)) & 1023u;
+  uint8_t* base = smem_raw + pad;
+  uint8_t* sA = base + kOffA;
+  uint8_t* sB = base + kOffB;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + kOffBars);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kStages;
+  uint64_t* acc_full = bars + 2 * kStages;
+  uint64_t* acc_empty = acc_full + kBufs;
+  uint64_t* drain = acc_empty + kBufs;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + kOffMisc + 4);
+  volatile int* never_flag = reinterpret_cast<volatile int*>(base + kOffMisc + 8);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int total = a.n_shared * a.m_tiles_shared * a.n_tiles_shared +
+                    a.n_routed * a.m_tiles_routed * a.n_tiles_routed;
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    *never_flag = 0;
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < kBufs; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], kEpiThreads);
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  uint32_t issued_mask = 0, issued_parity = 0;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------------ TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        const DwTile t = dw_decode(a, tile);
+        const CUtensorMap* ta = t.shared ? &a.a_shared : &a.a_routed;
+        const CUtensorMap* tb = t.shared ? &a.b_shared : &a.b_routed;
+        const int a_atom = (t.shared ? a.a_atom0_shared + t.group * a.a_atom_step_shared : a.a_atom0_routed) +
+                           t.m_blk * (2 * kFeat / 64);
+        const int b_atom = (t.shared ? a.b_atom0_shared + t.group * a.b_atom_step_shared : a.b_atom0_routed) +
+                           t.n_blk * (kN / 64);
+        const int kb_n = (t.rows + kBK - 1) / kBK;
+        for (int kb = 0; kb < kb_n; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, a.wait_limit_ns, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], kStageBytes);
+          tma_load_3d_view(sA + stage * kABytes, ta, &full[stage], t.row0 + kb * kBK, a_atom);
+          tma_load_3d_view(sB + stage * kBBytes, tb, &full[stage], t.row0 + kb * kBK, b_atom);
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(a.status, kStatusTimeoutProducer);
+      }
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------------------- MMA issuer
+    // The whole warp follows the loop: on a K block that runs past the group's rows it
+    // zeroes those rows of both operands first; lane 0 issues the MMAs.
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    int it = 0;
+    const uint32_t idesc = idesc_bf16_f32(kFeat, kN) | (1u << 15) | (1u << 16);  // A and B MN-major
+    for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++it) {
+      const DwTile t = dw_decode(a, tile);
+      const int kb_n = (t.rows + kBK - 1) / kBK;
+      const int acc = it % kBufs;
+      if (!mbar_wait_warp(&acc_empty[acc], ((it / kBufs) & 1) ^ 1u, a.wait_limit_ns, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d0 = tmem_base + acc * kAccCols;
+      for (int kb = 0; kb < kb_n; ++kb) {
+        if (!mbar_wait_warp(&full[stage], phase, a.wait_limit_ns, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int valid = t.rows - kb * kBK;  // rows of this K block inside the group
+        if (valid < kBK) {
+          // 6 atom columns (4 of A, 2 of B) x (64 - valid) rows of 128 B, 16 B per lane
+          const int bad = kBK - valid;
+          for (int i = lane; i < 6 * bad * 8; i += 32) {
+            const int col = i / (bad * 8), rem = i - col * bad * 8;
+            const int r = valid + rem / 8, q = rem % 8;
+            uint8_t* atom = col < 4 ? sA + stage * kABytes + col * kAtom : sB + stage * kBBytes + (col - 4) * kAtom;
+            *reinterpret_cast<uint4*>(atom + r * 128 + q * 16) = make_uint4(0u, 0u, 0u, 0u);  // row r: 128 B
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+        }
+        if (lane == 0) {
+          const uint32_t abase = smem_addr(sA + stage * kABytes), bbase = smem_addr(sB + stage * kBBytes);
+#pragma unroll
+          for (int k = 0; k < kBK / kMmaK; ++k) {
+            const uint32_t accum = (kb | k) ? 1u : 0u;
+            const uint32_t koff = static_cast<uint32_t>(k) * kMmaK * 128;
+            const uint64_t bd = desc_mn_sw128(bbase + koff);
+            mma_bf16_ss(d0, desc_mn_sw128(abase + koff), bd, idesc, accum);
+            mma_bf16_ss(d0 + kN, desc_mn_sw128(abase + 2 * kAtom + koff), bd, idesc, accum);
+          }
+          mma_commit(&empty[stage]);
+        }
+        __syncwarp();
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (lane == 0) mma_commit(&acc_full[acc]);  // with no K block: arrives at once
+      __syncwarp();
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      atomicOr(a.status, kStatusTimeoutMma);
+    }
+  } else {
+    // -------------------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    float* stg = reinterpret_cast<float*>(base + kOffEpi) + q * 32 * kStageRow;
+    const int rr = lane >> 2, cc = (lane & 3) * 8;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+      const DwTile t = dw_decode(a, tile);
+      const int acc = it % kBufs;
+      if (!mbar_wait_warp_sleepy(&acc_full[acc], (it / kBufs) & 1, a.wait_limit_ns, abort_flag)) {
+        if (lane == 0) {
+          *abort_flag = 1;
+          atomicOr(a.status, kStatusTimeoutEpilogue);
+        }
+        break;
+      }
+      tc_fence_after();
+      const bool empty_group = t.rows == 0;
+      const int M = t.shared ? a.m_shared : a.m_routed, N = t.shared ? a.n_shared_cols : a.n_routed_cols;
+      float* out = (t.shared ? a.out_shared : a.out_routed) + static_cast<int64_t>(t.group) * M * N;
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
+#pragma unroll 1
+      for (int ch = 0; ch < 2; ++ch) {
+#pragma unroll 1
+        for (int c0 = 0; c0 < kN; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld16(tb + ch * kN + c0, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+          tmem_ld16(tb + ch * kN + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) stg[j * kStageRow + lane] = empty_group ? 0.f : __uint_as_float(v[j]);
+          __syncwarp();
+          // lane L writes 8 consecutive columns c0 + cc.. of output row m_base + L/4 + 8i
+          const int m_base = t.m_blk * 2 * kFeat + ch * kFeat + q * 32;
+          const int n = t.n_blk * kN + c0 + cc;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int row = rr + 8 * i;
+            if (m_base + row < M && n < N) {
+              float vals[8];
+#pragma unroll
+              for (int k = 0; k < 8; ++k) vals[k] = stg[(cc + k) * kStageRow + row];
+              float4* dst = reinterpret_cast<float4*>(out + static_cast<int64_t>(m_base + row) * N + n);
+              dst[0] = make_float4(vals[0], vals[1], vals[2], vals[3]);
+              dst[1] = make_float4(vals[4], vals[5], vals[6], vals[7]);
+            }
+          }
+          __syncwarp();
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[acc]);
+    }
+  }
+
+  __syncthreads();
+  if (*abort_flag) {
+    if (warp == 0 && lane == 0) {
+      for (int s = 0; s < kStages; ++s)
+        if ((issued_mask >> s) & 1u)
+          if (!mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, drain_wait_limit(a.wait_limit_ns), never_flag))
+            atomicOr(a.status, kStatusTimeoutDrain);
+    }
+    if (warp == 1 && lane == 0) {
+      mma_commit(drain);
+      if (!mbar_wait_bounded(drain, 0, drain_wait_limit(a.wait_limit_ns), never_flag))
+        atomicOr(a.status, kStatusTimeoutDrain);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+}  // namespace
+
+cudaError_t launch_grouped_dw(const GemmDwArgs& a, int num_sms, cudaStream_t s) {
+  const int64_t total = static_cast<int64_t>(a.n_shared) * a.m_tiles_shared * a.n_tiles_shared +
+                        static_cast<int64_t>(a.n_routed) * a.m_tiles_routed * a.n_tiles_routed;
+  if (total <= 0) return cudaSuccess;
+  const int grid = static_cast<int>(total < num_sms ? total : num_sms);
+  cudaError_t e = cudaFuncSetAttribute(grouped_dw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  grouped_dw_kernel<<<grid, kThreads, kSmemBytes, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace dsmoe

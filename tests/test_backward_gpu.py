@@ -111,12 +111,16 @@ def test_backward_argument_errors():
         layer.close()
 
 
-EXP_CASES = [("tiny", 300), ("gshard_c", 500), ("ds2b", 700), ("v3_slice", 256)]
+EXP_CASES = [("tiny", 300), ("gshard_c", 500), ("ds2b", 700), ("v3_slice", 256), ("tiny", 37)]
 
 
 @pytest.mark.parametrize("name,T", EXP_CASES, ids=[f"{c[0]}-T{c[1]}" for c in EXP_CASES])
 def test_expert_backward_input_gradient(name, T):
-    """dL/du through the experts (dsmoe_backward_experts: W_down^T dy -> SiLU backward with
+    """Weight gradients dW_gate, dW_up, dW_down of every routed and shared expert
+    (dsmoe_backward_weights: ragged token reductions on the tensor cores) against the
+    oracle's layer_backward within 3e-2 of RMS per matrix (the same bf16 operands as
+    below, summed over tokens), an unpicked expert's gradient exactly zero; and
+    dL/du through the experts (dsmoe_backward_experts: W_down^T dy -> SiLU backward with
     the saved pre-activations -> W_gate^T da + W_up^T db on the tensor cores, weights read
     MN-major) plus the router's part, against the oracle's layer_backward dx (float64):
     max |err| / RMS <= 3e-2 (bf16 operands: g dh, the saved a and b, da | db and the
@@ -142,6 +146,13 @@ def test_expert_backward_input_gradient(name, T):
         dx = torch.empty((T, d), dtype=torch.float32, device="cuda")
         M.dsmoe_backward_experts(layer.handle, T, dh, dY, gpu["W_gate"], gpu["W_up"], gpu["W_down"],
                                  gpu.get("Ws_gate"), gpu.get("Ws_up"), gpu.get("Ws_down"), dx_r, dx)
+        F, Ks, Fs = cfg.d_ff, cfg.n_shared, cfg.d_ff_shared
+        dW = {k: torch.full(shp, float("nan"), device="cuda") for k, shp in (
+            ("dW_gate", (N, F, d)), ("dW_up", (N, F, d)), ("dW_down", (N, d, F)))}
+        dWs = {k: (torch.full(shp, float("nan"), device="cuda") if Ks else None) for k, shp in (
+            ("dWs_gate", (Ks, Fs, d)), ("dWs_up", (Ks, Fs, d)), ("dWs_down", (Ks, d, Fs)))}
+        M.dsmoe_backward_weights(layer.handle, T, dh, dY, gpu["x"], dW["dW_gate"], dW["dW_up"], dW["dW_down"],
+                                 dWs["dWs_gate"], dWs["dWs_up"], dWs["dWs_down"])
         torch.cuda.synchronize()
         assert M.dsmoe_get_status(layer.handle) == M.DSMOE_OK, M.dsmoe_last_error()
         dxs = M.workspace_view(layer.handle, "dXs")[:T].clone() if cfg.n_shared else None
@@ -160,11 +171,25 @@ def test_expert_backward_input_gradient(name, T):
         for i in range(cfg.n_shared):
             ref_s += DB.swiglu_backward(X, cpu["Ws_gate"][i], cpu["Ws_up"][i], cpu["Ws_down"][i], dh64)[0]
         e_s = _rel(dxs.cpu().numpy(), ref_s)
+    # weight gradients: every expert (one no token picked is exactly zero), per matrix
+    used = np.unique(ref["idx"])
+    e_w = {}
+    for k in ("dW_gate", "dW_up", "dW_down"):
+        got = dW[k]
+        unused = torch.ones(N, dtype=torch.bool)
+        unused[torch.as_tensor(used)] = False
+        if bool(unused.any()):
+            assert bool((got[unused.cuda()] == 0).all()), f"{k}: an unused expert's gradient is not zero"
+        e_w[k] = _rel(got[torch.as_tensor(used).cuda()].cpu().numpy(), bw[k][used])
+    if Ks:
+        for k in ("dWs_gate", "dWs_up", "dWs_down"):
+            e_w[k] = _rel(dWs[k].cpu().numpy(), bw[k])
     for k_ in ("W_gate", "W_up", "W_down"):
         if hasattr(cpu[k_], "cache"):
             cpu[k_].cache.clear()
-    print(name, T, "dx err/RMS", e_dx, "shared du err/RMS", e_s)
+    print(name, T, "dx err/RMS", e_dx, "shared du err/RMS", e_s, "dW err/RMS", e_w)
     assert e_dx <= 3e-2 and e_s <= 2e-2
+    assert all(v <= 3e-2 for v in e_w.values()), e_w
 
 
 def test_expert_backward_needs_a_training_forward():
