@@ -39,6 +39,14 @@ def _rel(got, ref):
     return float(np.abs(np.asarray(got, dtype=np.float64) - ref).max() / max(np.sqrt(np.mean(ref ** 2)), 1e-30))
 
 
+def _rel_fro_per_expert(got, ref):
+    """max over the leading (expert) axis of ||got_e - ref_e||_F / ||ref_e||_F."""
+    err = np.asarray(got, dtype=np.float64) - ref
+    num = np.sqrt((err ** 2).reshape(err.shape[0], -1).sum(axis=1))
+    den = np.sqrt((ref ** 2).reshape(ref.shape[0], -1).sum(axis=1))
+    return float((num / np.maximum(den, 1e-30)).max())
+
+
 @pytest.mark.parametrize("name,T,alpha,mask,k", CASES, ids=[f"{c[0]}-T{c[1]}" + (f"-m{c[3]}k{c[4]}" if c[3] else "")
                                                            for c in CASES])
 def test_gate_and_router_backward(name, T, alpha, mask, k):
@@ -118,8 +126,12 @@ EXP_CASES = [("tiny", 300), ("gshard_c", 500), ("ds2b", 700), ("v3_slice", 256),
 def test_expert_backward_input_gradient(name, T):
     """Weight gradients dW_gate, dW_up, dW_down of every routed and shared expert
     (dsmoe_backward_weights: ragged token reductions on the tensor cores) against the
-    oracle's layer_backward within 3e-2 of RMS per matrix (the same bf16 operands as
-    below, summed over tokens), an unpicked expert's gradient exactly zero; and
+    oracle's layer_backward, expert by expert: ||err||_F / ||ref||_F <= 1e-2 (the bf16
+    operands below, each rounded once, give a few 2^-9 per rank-1 term; a token missing
+    from or added to an expert's K range moves it by about 1/sqrt(rows)), and an unpicked
+    expert's gradient exactly zero. (max |err| / RMS is no bound here: an expert that few
+    tokens picked has a gradient of a few outer products, whose largest element is tens of
+    times its RMS.) And
     dL/du through the experts (dsmoe_backward_experts: W_down^T dy -> SiLU backward with
     the saved pre-activations -> W_gate^T da + W_up^T db on the tensor cores, weights read
     MN-major) plus the router's part, against the oracle's layer_backward dx (float64):
@@ -180,16 +192,16 @@ def test_expert_backward_input_gradient(name, T):
         unused[torch.as_tensor(used)] = False
         if bool(unused.any()):
             assert bool((got[unused.cuda()] == 0).all()), f"{k}: an unused expert's gradient is not zero"
-        e_w[k] = _rel(got[torch.as_tensor(used).cuda()].cpu().numpy(), bw[k][used])
+        e_w[k] = _rel_fro_per_expert(got[torch.as_tensor(used).cuda()].cpu().numpy(), bw[k][used])
     if Ks:
         for k in ("dWs_gate", "dWs_up", "dWs_down"):
-            e_w[k] = _rel(dWs[k].cpu().numpy(), bw[k])
+            e_w[k] = _rel_fro_per_expert(dWs[k].cpu().numpy(), bw[k])
     for k_ in ("W_gate", "W_up", "W_down"):
         if hasattr(cpu[k_], "cache"):
             cpu[k_].cache.clear()
     print(name, T, "dx err/RMS", e_dx, "shared du err/RMS", e_s, "dW err/RMS", e_w)
     assert e_dx <= 3e-2 and e_s <= 2e-2
-    assert all(v <= 3e-2 for v in e_w.values()), e_w
+    assert all(v <= 1e-2 for v in e_w.values()), e_w
 
 
 def test_expert_backward_needs_a_training_forward():
