@@ -89,37 +89,49 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-KERNEL_SOURCES = {"gemm_gate_up": "mixture_experts_layer_score_b200/csrc/gemm_sm100.cu",
-                  "gemm_down": "mixture_experts_layer_score_b200/csrc/gemm_sm100.cu",
-                  "router": "mixture_experts_layer_score_b200/csrc/router_sm100.cu"}
-PAIR_GEMM_SOURCE = "mixture_experts_layer_score_b200/csrc/gemm_pair_sm100.cu"
+CSRC = "mixture_experts_layer_score_b200/csrc/"
+# the sources that decide each stage's memory traffic: the kernel and, for the grouped
+# GEMMs, the tile schedule
+KERNEL_SOURCES = {"gemm_gate_up": ("gemm_sm100.cu", "grouped_tiles.cuh"),
+                  "gemm_down": ("gemm_sm100.cu", "grouped_tiles.cuh"),
+                  "router": ("router_sm100.cu",)}
+PAIR_GEMM_SOURCES = {"gemm_gate_up": ("gemm_gateup_pair_sm100.cu", "grouped_tiles.cuh"),
+                     "gemm_down": ("gemm_pair_sm100.cu", "grouped_tiles.cuh")}
 
 
 def source_digest(stage, gemm="single"):
+    """First 16 hex digits of the sha256 over the stage's kernel sources, in order."""
     import hashlib
-    src = PAIR_GEMM_SOURCE if (gemm == "pair" and stage.startswith("gemm")) else KERNEL_SOURCES[stage]
-    path = os.path.join(ROOT, src)
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    srcs = PAIR_GEMM_SOURCES[stage] if (gemm == "pair" and stage in PAIR_GEMM_SOURCES) else KERNEL_SOURCES[stage]
+    h = hashlib.sha256()
+    for src in srcs:
+        with open(os.path.join(ROOT, CSRC + src), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
-def captured_traffic(stage, weight_bytes, gemm="single"):
+def captured_traffic(stage, weight_bytes, gemm="single", workload=None):
     """DRAM bytes per launch of `stage` from the committed ncu summary
     (profiles/ncu_dram_traffic.txt): the captured launch's DRAM read+write bytes divided by
-    the algorithmic weight bytes it streamed, scaled to this launch's weight bytes (the
-    capture runs a smaller case of the same kernel; its DRAM traffic is dominated by the
-    expert weights and grows with them). None when the kernel source changed since the
-    capture or no capture is recorded."""
+    the algorithmic weight bytes it streamed, scaled to this launch's weight bytes. A
+    capture of the benchmarked workload itself is preferred (the scaling is then the
+    identity); otherwise the first capture of the stage is scaled (its DRAM traffic is
+    dominated by the expert weights and grows with them). None when the kernel sources
+    changed since the capture or no capture is recorded."""
     path = os.path.join(ROOT, "profiles", "ncu_dram_traffic.txt")
     if not os.path.exists(path):
         return None
     digest = source_digest(stage, gemm)
+    found = []
     with open(path) as f:
         for line in f:
             parts = line.split()
-            if len(parts) >= 4 and not line.startswith("#") and parts[0] == stage and parts[1] == digest:
-                return float(parts[2]) / float(parts[3]) * weight_bytes
-    return None
+            if len(parts) >= 5 and not line.startswith("#") and parts[0] == stage and parts[1] == digest:
+                found.append((parts[4] == workload, float(parts[2]) / float(parts[3])))
+    if not found:
+        return None
+    same = [r for m, r in found if m]
+    return (same[0] if same else found[0][1]) * weight_bytes
 
 
 def config_block(cfg, n_gpus):
@@ -380,7 +392,7 @@ def run_native(args, cfg):
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "frac_of_spec": achieved / SPEC_HBM_GBS}
-    traffic = captured_traffic(dom, weight_bytes[dom], args.gemm)
+    traffic = captured_traffic(dom, weight_bytes[dom], args.gemm, cfg.name)
     roof.update({"kernel": dom, "kernel_ms": dom_ms, "traffic": traffic,
                  "peak_source": f"{peak_src} ({tensor_key if roof['bound'] == 'tensor' else 'hbm_gbs'})",
                  "peak_choice": PEAK_CHOICE,

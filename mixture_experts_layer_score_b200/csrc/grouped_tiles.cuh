@@ -3,9 +3,10 @@
 // Groups are the shared experts (dense, m_shared rows each) followed by the routed
 // groups (segments of the expert-contiguous slot order, from the device-side offsets).
 // A routed group is one expert, or, with expert_mod = n > 0, group g applies expert
-// g mod n (rows received from several ranks, grouped by source and then by expert). A group of M rows has ceil(M / kTok) token tiles times n_tiles output tiles;
-// tiles are numbered group by group, token tiles fastest, so that the CTAs working at
-// the same time share each weight tile through L2. The per-group prefix lives in shared
+// g mod n (rows received from several ranks, grouped by source and then by expert). A
+// group of M rows has ceil(M / kTok) token tiles of near-equal size times n_tiles output
+// tiles; tiles are numbered group by group, token tiles fastest, so that the CTAs working
+// at the same time share each weight tile through L2. The per-group prefix lives in shared
 // memory and is built by every CTA from the offsets (no host synchronisation).
 #pragma once
 
@@ -87,8 +88,15 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int32_t* ti
   const int local = tile - tile_start[lo];
   const int m_blk = local % mt;
   t.n_blk = local / mt;
-  t.row0 = base + m_blk * kTok;
-  t.m_valid = min(kTok, M - m_blk * kTok);
+  // The group's rows are split evenly over its mt token tiles in 16-row granules (tile
+  // sizes differ by at most 16), not into full tiles and one ragged remainder: the CTAs
+  // sharing a weight tile then run at the same MMA rate and stay close enough in K for
+  // the second reader to find the weights in L2. The MMA work is the same, since N is
+  // the tile's row count rounded up to 16 either way.
+  const int gr = (M + 15) >> 4, q = gr / mt, rem = gr - q * mt;
+  const int g0 = m_blk * q + min(m_blk, rem);
+  t.row0 = base + g0 * 16;
+  t.m_valid = min((q + (m_blk < rem ? 1 : 0)) * 16, M - g0 * 16);
   return t;
 }
 
