@@ -234,7 +234,7 @@ struct dsmoe_handle {
   cudaStream_t copy_stream_out = nullptr;  // output copies (both directions run at once)
   cudaEvent_t ev_in[2] = {}, ev_out[2] = {}, ev_d2h[2] = {};
   int64_t async_calls = 0;
-  CUtensorMap tm_xp, tm_a1, tm_a1s;
+  CUtensorMap tm_a1, tm_a1s;
   // weight maps, cached per pointer: W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, W_router
   // (the gate/up maps serve both GEMM kernels), then W_down and Ws_down for the pair down GEMM
   static constexpr int kMaps = 9;
@@ -400,8 +400,8 @@ DSMOE_EXPORT dsmoe_status dsmoe_create(const dsmoe_cfg* cfg, int32_t device, dsm
   }
   const dsmoe_cfg& c = h->cfg;
   const uint64_t S = static_cast<uint64_t>(c.max_tokens) * c.top_k;
-  const uint32_t t1 = dsmoe::kGemmGateUpTokenTile, t2 = dsmoe::kGemmDownTokenTile;
-  bool ok = map_2d(&h->tm_xp, h->Xp, c.d_model, S, t1) && map_2d(&h->tm_a1, h->A1, c.d_ff, S, t2);
+  const uint32_t t2 = dsmoe::kGemmTokenTile;  // the down projection's token tile
+  bool ok = map_2d(&h->tm_a1, h->A1, c.d_ff, S, t2);
   if (c.n_shared > 0)
     ok = ok && map_2d(&h->tm_a1s, h->A1s, static_cast<uint64_t>(c.n_shared) * c.d_ff_shared, c.max_tokens, t2);
   else
@@ -637,8 +637,9 @@ dsmoe_status scan_permute_stage(dsmoe_handle* h, const FwdArgs& a, cudaStream_t 
 // the T token rows of `x_map` (gate/up) / h->A1s (down). Gate/up writes A1 (routed) and
 // A1s (shared); down writes Y_out (routed) and Hs = residual + shared outputs (fp32).
 struct GemmPlan {
-  const CUtensorMap* rows_map;      // routed token rows (Xp or received rows), gate/up A operand
-  const CUtensorMap* x_map;         // x rows of the shared groups
+  const void* rows;                 // routed token rows (Xp or received rows), gate/up operand
+  uint64_t rows_extent;             // rows addressable at `rows` ([rows_extent, d])
+  const void* x;                    // [T, d] x rows of the shared groups
   const int32_t* offsets;
   int n_groups, expert_mod;
   int64_t routed_rows;              // rows the routed groups cover (tile bound)
@@ -656,10 +657,17 @@ dsmoe_status gemm_stage(dsmoe_handle* h, const GemmPlan& p, cudaStream_t s,
   const bool pair = h->gemm_kernel == DSMOE_GEMM_PAIR;
   // ---- gate/up GEMM with SiLU(gate) * up
   {
+    // token tile of this launch (the pair kernel stages 128 of its 256 token rows per CTA)
+    const int tok = pair ? dsmoe::kGemmTokenTile : dsmoe::gateup_token_tile(d, p.routed_rows, p.n_groups);
+    CUtensorMap m_rows, m_x;
+    bool ok = true;
+    if (p.n_groups > 0) ok = map_2d(&m_rows, p.rows, d, p.rows_extent, tok);
+    if (Ks > 0) ok = ok && map_2d(&m_x, p.x, d, T, tok);
+    if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a token tensor map of the gate/up GEMM");
     dsmoe::GemmArgs g;
     memset(&g, 0, sizeof(g));
-    g.a_routed = *p.rows_map;
-    g.a_shared = *p.x_map;
+    g.a_routed = p.n_groups > 0 ? m_rows : m_x;  // (a kind with no groups is never read)
+    g.a_shared = Ks > 0 ? m_x : m_rows;
     g.b0_routed = *p.wg;
     g.b1_routed = *p.wu;
     g.b0_shared = *p.swg;
@@ -686,7 +694,7 @@ dsmoe_status gemm_stage(dsmoe_handle* h, const GemmPlan& p, cudaStream_t s,
     g.save_ab_shared = p.save_ab ? h->ABs : nullptr;
     g.status = h->status;
     g.wait_limit_ns = h->wait_ns;
-    const int64_t tt = pair ? dsmoe::kGemmPairTokenTile : dsmoe::kGemmGateUpTokenTile;
+    const int64_t tt = pair ? dsmoe::kGemmPairTokenTile : tok;
     const int64_t bound = (cdiv(p.routed_rows, tt) + p.n_groups) * static_cast<int64_t>(g.n_tiles_routed) +
                           static_cast<int64_t>(Ks) * cdiv(T, tt) * g.n_tiles_shared;
     if (bound > 0) {
@@ -695,7 +703,7 @@ dsmoe_status gemm_stage(dsmoe_handle* h, const GemmPlan& p, cudaStream_t s,
         CUDA_TRY(dsmoe::launch_gateup_pair(g, clusters, s));
       } else {
         const int grid = static_cast<int>(bound < h->num_sms ? bound : h->num_sms);
-        CUDA_TRY(dsmoe::launch_grouped_gemm(true, g, grid, s));
+        CUDA_TRY(dsmoe::launch_grouped_gemm(true, tok, g, grid, s));
       }
       h->launches += 1;
     }
@@ -732,7 +740,7 @@ dsmoe_status gemm_stage(dsmoe_handle* h, const GemmPlan& p, cudaStream_t s,
     g.shared_col_stride = 0;
     g.status = h->status;
     g.wait_limit_ns = h->wait_ns;
-    const int64_t tt = pair ? dsmoe::kGemmPairTokenTile : dsmoe::kGemmDownTokenTile;
+    const int64_t tt = pair ? dsmoe::kGemmPairTokenTile : dsmoe::kGemmTokenTile;
     const int64_t bound = (cdiv(p.routed_rows, tt) + p.n_groups) * static_cast<int64_t>(g.n_tiles_routed) +
                           static_cast<int64_t>(g.n_shared_groups) * cdiv(T, tt) * g.n_tiles_shared;
     if (bound > 0) {
@@ -741,7 +749,7 @@ dsmoe_status gemm_stage(dsmoe_handle* h, const GemmPlan& p, cudaStream_t s,
         CUDA_TRY(dsmoe::launch_down_pair(g, clusters, s));
       } else {
         const int grid = static_cast<int>(bound < h->num_sms ? bound : h->num_sms);
-        CUDA_TRY(dsmoe::launch_grouped_gemm(false, g, grid, s));
+        CUDA_TRY(dsmoe::launch_grouped_gemm(false, dsmoe::kGemmTokenTile, g, grid, s));
       }
       h->launches += 1;
     }
@@ -786,7 +794,7 @@ dsmoe_status zero_stats(const FwdArgs& a, int N, cudaStream_t s) {
 
 dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
   const dsmoe_cfg& c = h->cfg;
-  const int T = a.T, N = c.n_routed, K = h->k_active, d = c.d_model;
+  const int T = a.T, N = c.n_routed, K = h->k_active;
   // shared experts (and the residual) only where this handle adds them
   const int Ks = h->add_shared ? c.n_shared : 0;
   const int e0 = h->e_begin, NL = h->e_end - h->e_begin;  // routed experts applied here
@@ -808,8 +816,6 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
   p.swg = Ks ? weight_map(h, 3, a.Ws_gate, &ok) : p.wg;
   p.swu = Ks ? weight_map(h, 4, a.Ws_up, &ok) : p.wu;
   p.swd = Ks ? weight_map(h, pair ? 8 : 5, a.Ws_down, &ok) : p.wd;
-  CUtensorMap m_x;  // token rows of x in GEMM tiles (shared groups)
-  ok = ok && map_2d(&m_x, a.x, d, T, dsmoe::kGemmGateUpTokenTile);
   if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map of this call");
 
   CUDA_TRY(mark(0));
@@ -818,8 +824,9 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
   CUDA_TRY(mark(2));
   STAGE_TRY(scan_permute_stage(h, a, s, sel_grid, e0, e0 + NL, mark));
   CUDA_TRY(mark(4));
-  p.rows_map = &h->tm_xp;
-  p.x_map = &m_x;
+  p.rows = h->Xp;
+  p.rows_extent = static_cast<uint64_t>(c.max_tokens) * c.top_k;
+  p.x = a.x;
   p.offsets = h->offsets + e0;
   p.n_groups = NL;
   p.expert_mod = 0;
@@ -1056,12 +1063,10 @@ DSMOE_EXPORT dsmoe_status dsmoe_ep_experts(dsmoe_handle* h, int32_t n_src, int32
   p.swg = p.wg;
   p.swu = p.wu;
   p.swd = p.wd;
-  CUtensorMap m_rows;
-  const uint32_t box = h->gemm_kernel == DSMOE_GEMM_PAIR ? 128 : dsmoe::kGemmGateUpTokenTile;
-  ok = ok && map_2d(&m_rows, rows, c.d_model, static_cast<uint64_t>(n_rows), box);
   if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map of this call");
-  p.rows_map = &m_rows;
-  p.x_map = &m_rows;
+  p.rows = rows;
+  p.rows_extent = static_cast<uint64_t>(n_rows);
+  p.x = rows;
   p.offsets = h->offsets;
   p.n_groups = groups;
   p.expert_mod = n_local;
@@ -1102,11 +1107,10 @@ DSMOE_EXPORT dsmoe_status dsmoe_ep_combine(dsmoe_handle* h, int32_t T, const voi
     p.wg = p.swg;
     p.wu = p.swu;
     p.wd = p.swd;
-    CUtensorMap m_x;
-    ok = ok && map_2d(&m_x, x, c.d_model, T, dsmoe::kGemmGateUpTokenTile);
     if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map of this call");
-    p.rows_map = &m_x;
-    p.x_map = &m_x;
+    p.rows = x;
+    p.rows_extent = static_cast<uint64_t>(T);
+    p.x = x;
     p.offsets = h->offsets;
     p.n_groups = 0;
     p.expert_mod = 0;

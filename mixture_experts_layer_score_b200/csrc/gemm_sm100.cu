@@ -13,25 +13,32 @@
 // Orientation: the MMA's M dimension is the weights' output features and its N
 // dimension is the group's tokens, D^T[feature, token] = W[feature, :] . X[token, :]^T.
 // A tile is 128 (gate/up: 128 gate + the same 128 up features; down: 2 x 128 output
-// features) by at most 128 tokens, and N is the tile's token count rounded up to 16,
+// features) by at most kTok tokens, and N is the tile's token count rounded up to 16,
 // so an expert's ragged last tile wastes at most 15 token columns of tensor work and
-// an expert with a handful of decode tokens costs N=16, not a 128-row tile.
+// an expert with a handful of decode tokens costs N=16, not a full tile.
 //
-// One CTA per SM, 192 threads in three roles:
+// Token tile kTok = 128 or 256 (a template parameter chosen per launch). A 256-token
+// tile stages the same weight bytes for twice the MMA work and runs the MMAs at N=256,
+// where the tensor core reads fewer shared-memory bytes per MAC than at N=128; its two
+// chains then fill all 512 TMEM columns, so the next tile's MMAs wait for this tile's
+// epilogue. It pays where the K loop is long (d >= 4096) and experts hold a few hundred
+// rows; elsewhere the 128-token tile with two accumulators is faster.
+//
+// One CTA per SM, 320 threads in three roles:
 //   warp 0     TMA producer: per 64-wide K block a 256x64 weight tile (two 128-row
-//              halves) and a 128x64 token tile through a 4-stage shared-memory ring of
-//              48 KB stages (mbarrier full/empty pairs).
-//   warp 1     allocates 512 TMEM columns (two accumulators, each two chains of 128
-//              columns) and issues tcgen05.mma (M=128, N=16..128, K=16) from one
-//              thread, two chains (one per weight half) sharing the token tile; commits
-//              free ring stages and publish finished accumulators.
-//   warps 2-5  epilogue: thread f of TMEM lane f owns output feature f of both chains;
-//              per 32 tokens it reads its accumulator columns with tcgen05.ld, applies
-//              SiLU(gate)*up (or the residual), and the warp transposes the 32 x 32
-//              block through shared memory so that each lane stores 16-byte vectors
-//              along output rows. The second TMEM accumulator lets the next tile's MMAs
-//              overlap this epilogue.
-//
+//              halves) and a kTok x 64 token tile through a ring of 48 KB (4 stages,
+//              128-token tiles) or 64 KB (3 stages, 256-token tiles) stages.
+//   warp 1     allocates 512 TMEM columns (accumulators of two chains of kTok columns)
+//              and issues tcgen05.mma (M=128, N=16..kTok, K=16) from one thread, two
+//              chains (one per weight half) sharing the token tile; commits free ring
+//              stages and publish finished accumulators.
+//   warps 2-9  epilogue: warps 2+q and 6+q read TMEM lanes [32q, 32q+32) (thread f of
+//              lane f owns output feature f of both chains) for alternate 32-token
+//              chunks. Per chunk: tcgen05.ld of both chains (the next chunk's loads are
+//              issued before this one's last rows are stored), SiLU(gate)*up (or the
+//              residual) in fp32,
+//              a 32 x 32 transpose through shared memory (bf16; fp32 in 16-token halves
+//              for the shared experts' fp32 sums) and 16-byte stores along output rows.
 // Every wait is bounded (wait_limit_ns); a role that gives up raises a CTA-wide abort
 // flag and a bit of the device status word, the CTA lets in-flight TMA loads and MMAs
 // finish (a wait bounded by at least one second, whatever the caller's limit), frees its
@@ -45,23 +52,21 @@ namespace {
 constexpr int kBK = 64;         // K per ring stage (one 128-byte swizzled row of bf16)
 constexpr int kFeat = 128;      // output features per MMA chain (the MMA's M, TMEM lanes)
 constexpr int kMmaK = 16;       // K of each bf16 tcgen05.mma
-constexpr int kThreads = 192;
-constexpr int kEpiThreads = 128;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kWBytes = 2 * kFeat * kBK * 2;  // 32 KB: two 128-row weight halves
-constexpr uint32_t kStageRow = 33;  // epilogue staging rows padded to 33 words
+constexpr uint32_t kStgRow = 40;                   // bf16 staging row: 32 values + 8 pad (80 B)
+constexpr uint32_t kStgRowF = 33;                  // fp32 staging row: 32 values + 1 pad
+constexpr uint32_t kStgBytes = 32 * kStgRow * 2;   // per epilogue warp: 32 bf16 rows or 16 fp32 rows
+static_assert(16 * kStgRowF * 4 <= kStgBytes, "fp32 half-chunk staging fits the bf16 chunk's");
 
-// Tile geometry of each projection: up to 128 tokens per tile, two accumulators (each two
-// 128-column chains) so the epilogue of one tile overlaps the MMAs of the next, and a
-// 4-stage ring of 48 KB. (256-token tiles with one accumulator stage fewer bytes per MAC
-// but measured slower at every shape tried: the epilogue no longer overlaps the MMAs.)
-template <bool kSwiGLU>
+template <int kTok>
 struct Geo {
-  static constexpr int kTok = kSwiGLU ? kGemmGateUpTokenTile : kGemmDownTokenTile;
   static constexpr uint32_t kChainCols = kTok;
   static constexpr uint32_t kAccCols = 2 * kChainCols;
   static constexpr int kBufs = static_cast<int>(kTmemCols / kAccCols);
-  static constexpr int kStages = 4;
+  static constexpr int kStages = kTok == 256 ? 3 : 4;
   static constexpr uint32_t kXBytes = kTok * kBK * 2;
   static constexpr uint32_t kStageBytes = kWBytes + kXBytes;
   static constexpr uint32_t kOffW = 0;
@@ -71,15 +76,15 @@ struct Geo {
   static constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
   static constexpr uint32_t kOffTiles = kOffMisc + 16;
   static constexpr uint32_t kOffEpi = (kOffTiles + (kGemmMaxGroups + 1) * 4 + 15) & ~15u;
-  static constexpr uint32_t kSmemUsed = kOffEpi + 4 * 32 * kStageRow * 4;
+  static constexpr uint32_t kSmemUsed = kOffEpi + kEpiWarps * kStgBytes;
   static constexpr size_t kSmemBytes = kSmemUsed + 1024;  // slack to align the ring to 1024 bytes
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert(kBufs >= 1 && kTok % 32 == 0 && kTok <= 256, "tile geometry");
+  static_assert(kBufs >= 1 && kBufs <= 2 && kTok % 32 == 0 && kTok <= 256, "tile geometry");
 };
 
-template <bool kSwiGLU>
+template <bool kSwiGLU, int kTok>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs a) {
-  using G_ = Geo<kSwiGLU>;
+  using G_ = Geo<kTok>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_addr(smem_raw) & 1023u)) & 1023u;
   uint8_t* base = smem_raw + pad;
@@ -99,7 +104,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = a.n_shared_groups + a.n_routed;
 
-  tile_counts<G_::kTok>(a, tile_start, G);
+  tile_counts<kTok>(a, tile_start, G);
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     *never_flag = 0;
@@ -109,7 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], kEpiThreads);
+      mbar_init(&acc_empty[i], kEpiWarps);  // one lane of each epilogue warp
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -138,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       uint32_t phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-        const Tile t = decode_tile<G_::kTok>(a, tile_start, G, tile);
+        const Tile t = decode_tile<kTok>(a, tile_start, G, tile);
         const CUtensorMap* tx = t.shared ? &a.a_shared : &a.a_routed;
         const CUtensorMap* tw0 = t.shared ? &a.b0_shared : &a.b0_routed;
         const CUtensorMap* tw1 = t.shared ? &a.b1_shared : &a.b1_routed;
@@ -180,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       bool ok = true;
       int it = 0;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++it) {
-        const Tile t = decode_tile<G_::kTok>(a, tile_start, G, tile);
+        const Tile t = decode_tile<kTok>(a, tile_start, G, tile);
         const int n_mma = (t.m_valid + 15) & ~15;  // tokens, rounded up to the MMA's N step
         const uint32_t idesc = idesc_bf16_f32(kFeat, n_mma);
         const int acc = it % G_::kBufs;
@@ -222,16 +227,19 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
     }
   } else {
     // -------------------------------------------------------------------- epilogue
-    // Thread f of TMEM lane f holds output feature f of both chains. Per 32 tokens, the
-    // warp transposes its 32 features x 32 tokens through a padded shared-memory tile,
-    // then lane L stores 8 consecutive features (16 B of bf16, 32 B of fp32) of token
-    // row L/4 + 8i: four lanes cover the warp's 32-feature segment of a row.
-    const int q = warp & 3;  // this warp may read TMEM lanes [32q, 32q+32)
-    float* stg = reinterpret_cast<float*>(base + G_::kOffEpi) + q * 32 * kStageRow;
+    // Warp w reads TMEM lanes [32q, 32q+32), q = w % 4: thread f of lane f holds output
+    // feature f of both chains. It takes the tile's 32-token chunks c with
+    // c % 2 == (w - 2) / 4, transposes each 32 features x 32 tokens block through its
+    // staging area, and lane L stores 8 consecutive features (16 B of bf16, 32 B of fp32)
+    // of token row L/4 + 8i: four lanes cover the warp's 32-feature segment of a row.
+    const int q = warp & 3, half = (warp - 2) >> 2;
+    uint8_t* stg_raw = base + G_::kOffEpi + (warp - 2) * kStgBytes;
+    uint16_t* stg = reinterpret_cast<uint16_t*>(stg_raw);  // [32 tokens][kStgRow] bf16
+    float* stgf = reinterpret_cast<float*>(stg_raw);       // [16 tokens][kStgRowF] fp32
     const int rr = lane >> 2, cc = (lane & 3) * 8;  // read-out: row (plus 8i), first feature
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
-      const Tile t = decode_tile<G_::kTok>(a, tile_start, G, tile);
+      const Tile t = decode_tile<kTok>(a, tile_start, G, tile);
       const int acc = it % G_::kBufs;
       if (!mbar_wait_warp_sleepy(&acc_full[acc], (it / G_::kBufs) & 1, a.wait_limit_ns, abort_flag)) {
         if (lane == 0) {
@@ -245,92 +253,124 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       const int n_valid = t.shared ? a.n_valid_shared : a.n_valid_routed;
       const int64_t ld = t.shared ? a.ld_shared : a.ld_routed;
       const bool f32_out = !kSwiGLU && t.shared && a.out_shared_f32 != nullptr;
+      // the backward pass's saved pre-activations: a (chain 0) and b (chain 1) as bf16
+      bf16* save = kSwiGLU ? (t.shared ? a.save_ab_shared : a.save_ab_routed) : nullptr;
       // chains whose values leave this tile: gate/up gives one output chain, down two
-      const int n_out = kSwiGLU ? 1 : 2;
+      constexpr int kOut = kSwiGLU ? 1 : 2;
+      const int n_chunks = (t.m_valid + 31) >> 5;
+      uint32_t v0[32], v1[32];  // this chunk's accumulator columns of the two chains
+      if (half < n_chunks) {
+        tmem_ld16(tb + 32 * half, *reinterpret_cast<uint32_t(*)[16]>(&v0[0]));
+        tmem_ld16(tb + 32 * half + 16, *reinterpret_cast<uint32_t(*)[16]>(&v0[16]));
+        tmem_ld16(tb + G_::kChainCols + 32 * half, *reinterpret_cast<uint32_t(*)[16]>(&v1[0]));
+        tmem_ld16(tb + G_::kChainCols + 32 * half + 16, *reinterpret_cast<uint32_t(*)[16]>(&v1[16]));
+      }
+      tmem_wait_ld();
 #pragma unroll 1
-      for (int c0 = 0; c0 < t.m_valid; c0 += 32) {
-        uint32_t v0[32], v1[32];
-        tmem_ld16(tb + c0, *reinterpret_cast<uint32_t(*)[16]>(&v0[0]));
-        tmem_ld16(tb + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v0[16]));
-        tmem_ld16(tb + G_::kChainCols + c0, *reinterpret_cast<uint32_t(*)[16]>(&v1[0]));
-        tmem_ld16(tb + G_::kChainCols + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v1[16]));
-        tmem_wait_ld();
-        // the backward pass's saved pre-activations: a (chain 0) and b (chain 1) as bf16
-        bf16* save = kSwiGLU ? (t.shared ? a.save_ab_shared : a.save_ab_routed) : nullptr;
+      for (int ch_i = half; ch_i < n_chunks; ch_i += 2) {
+        const int c0 = 32 * ch_i;
+        // Once the last staging write has read v0 / v1, the next chunk's columns are
+        // loaded into them while this chunk's rows are stored.
+        const bool more = ch_i + 2 < n_chunks;
+        auto load_next = [&]() {
+          if (more) {
+            const uint32_t cn = static_cast<uint32_t>(c0 + 64);
+            tmem_ld16(tb + cn, *reinterpret_cast<uint32_t(*)[16]>(&v0[0]));
+            tmem_ld16(tb + cn + 16, *reinterpret_cast<uint32_t(*)[16]>(&v0[16]));
+            tmem_ld16(tb + G_::kChainCols + cn, *reinterpret_cast<uint32_t(*)[16]>(&v1[0]));
+            tmem_ld16(tb + G_::kChainCols + cn + 16, *reinterpret_cast<uint32_t(*)[16]>(&v1[16]));
+          }
+        };
         if (kSwiGLU && save) {
           const int width = t.shared ? a.shared_col_stride : a.n_valid_routed;  // F_s or F
           const int64_t lds = 2 * (t.shared ? a.ld_shared : a.ld_routed);
           const int64_t col0 = t.shared ? static_cast<int64_t>(t.group) * 2 * width : 0;
           const int feat = t.n_blk * kFeat + q * 32 + cc;
-#pragma unroll 1
+#pragma unroll
           for (int ch = 0; ch < 2; ++ch) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) stg[j * kStageRow + lane] = __uint_as_float(ch == 0 ? v0[j] : v1[j]);
+            for (int j = 0; j < 32; ++j)
+              stg[j * kStgRow + lane] =
+                  __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(ch == 0 ? v0[j] : v1[j])));
             __syncwarp();
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int row = rr + 8 * i;
-              if (feat < width && c0 + row < t.m_valid) {
-                const float* src = stg + row * kStageRow + cc;
+              if (feat < width && c0 + row < t.m_valid)
                 *reinterpret_cast<uint4*>(save + static_cast<int64_t>(t.row0 + c0 + row) * lds + col0 +
                                           ch * width + feat) =
-                    make_uint4(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
-                               pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
-              }
+                    *reinterpret_cast<const uint4*>(stg + row * kStgRow + cc);
             }
             __syncwarp();
           }
         }
-#pragma unroll 1
-        for (int ch = 0; ch < n_out; ++ch) {
-          // stage: row = token (c0 + j), column = this lane's feature
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            float val;
-            if (kSwiGLU) {
-              const float g = __uint_as_float(v0[j]);
-              val = __fdividef(g, 1.0f + __expf(-g)) * __uint_as_float(v1[j]);  // SiLU(g) * u
-            } else {
-              val = __uint_as_float(ch == 0 ? v0[j] : v1[j]);
-            }
-            stg[j * kStageRow + lane] = val;
-          }
-          __syncwarp();
+        for (int ch = 0; ch < kOut; ++ch) {
           const int feat = (kSwiGLU ? t.n_blk * kFeat : t.n_blk * 2 * kFeat + ch * kFeat) + q * 32 + cc;
           const bool ok_f = feat < n_valid;  // n_valid is a multiple of 64, feat of 8
+          if (f32_out) {
+            // the shared experts' sum plus the residual x, in fp32: two 16-token halves
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int row = rr + 8 * i;
-            if (ok_f && c0 + row < t.m_valid) {
-              const float* src = stg + row * kStageRow + cc;
-              const int64_t o = static_cast<int64_t>(t.row0 + c0 + row) * ld + feat;
-              if (f32_out) {
-                const uint4 rv = *reinterpret_cast<const uint4*>(a.residual + o);
-                const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
-                float out8[8];
+            for (int hh = 0; hh < 2; ++hh) {
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                  const float2 xr = unpack_bf16x2(rw[k]);
-                  out8[2 * k] = src[2 * k] + xr.x;
-                  out8[2 * k + 1] = src[2 * k + 1] + xr.y;
+              for (int j = 0; j < 16; ++j)
+                stgf[j * kStgRowF + lane] = __uint_as_float(ch == 0 ? v0[16 * hh + j] : v1[16 * hh + j]);
+              __syncwarp();
+              if (ch == kOut - 1 && hh == 1) load_next();
+#pragma unroll
+              for (int i = 0; i < 2; ++i) {
+                const int row = rr + 8 * i, tok = c0 + 16 * hh + row;
+                if (ok_f && tok < t.m_valid) {
+                  const float* src = stgf + row * kStgRowF + cc;
+                  const int64_t o = static_cast<int64_t>(t.row0 + tok) * ld + feat;
+                  const uint4 rv = *reinterpret_cast<const uint4*>(a.residual + o);
+                  const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
+                  float out8[8];
+#pragma unroll
+                  for (int k = 0; k < 4; ++k) {
+                    const float2 xr = unpack_bf16x2(rw[k]);
+                    out8[2 * k] = src[2 * k] + xr.x;
+                    out8[2 * k + 1] = src[2 * k + 1] + xr.y;
+                  }
+                  float4* dst = reinterpret_cast<float4*>(a.out_shared_f32 + o);
+                  dst[0] = make_float4(out8[0], out8[1], out8[2], out8[3]);
+                  dst[1] = make_float4(out8[4], out8[5], out8[6], out8[7]);
                 }
-                float4* dst = reinterpret_cast<float4*>(a.out_shared_f32 + o);
-                dst[0] = make_float4(out8[0], out8[1], out8[2], out8[3]);
-                dst[1] = make_float4(out8[4], out8[5], out8[6], out8[7]);
-              } else {
-                bf16* obase = t.shared ? a.out_shared + static_cast<int64_t>(t.group) * a.shared_col_stride
-                                       : a.out_routed;
-                *reinterpret_cast<uint4*>(obase + o) =
-                    make_uint4(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
-                               pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
               }
+              __syncwarp();
             }
+          } else {
+            // stage: row = token (c0 + j), column = this lane's feature, rounded to bf16
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              float val;
+              if (kSwiGLU) {
+                const float g = __uint_as_float(v0[j]);
+                val = __fdividef(g, 1.0f + __expf(-g)) * __uint_as_float(v1[j]);  // SiLU(g) * u
+              } else {
+                val = __uint_as_float(ch == 0 ? v0[j] : v1[j]);
+              }
+              stg[j * kStgRow + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+            }
+            __syncwarp();
+            if (ch == kOut - 1) load_next();
+            bf16* obase = t.shared ? a.out_shared + static_cast<int64_t>(t.group) * a.shared_col_stride
+                                   : a.out_routed;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int row = rr + 8 * i;
+              if (ok_f && c0 + row < t.m_valid)
+                *reinterpret_cast<uint4*>(obase + static_cast<int64_t>(t.row0 + c0 + row) * ld + feat) =
+                    *reinterpret_cast<const uint4*>(stg + row * kStgRow + cc);
+            }
+            __syncwarp();
           }
-          __syncwarp();
         }
+        tmem_wait_ld();  // the next chunk's columns have landed in v0 / v1
       }
       tc_fence_before();
-      mbar_arrive(&acc_empty[acc]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
     }
   }
 
@@ -358,22 +398,23 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
 }
 }  // namespace
 
-cudaError_t launch_grouped_gemm(bool swiglu, const GemmArgs& a, int grid, cudaStream_t s) {
+namespace {
+template <bool kSwiGLU, int kTok>
+cudaError_t launch_one(const GemmArgs& a, int grid, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<kSwiGLU, kTok>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(Geo<kTok>::kSmemBytes));
+  if (e != cudaSuccess) return e;
+  grouped_gemm_kernel<kSwiGLU, kTok><<<grid, kThreads, Geo<kTok>::kSmemBytes, s>>>(a);
+  return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_grouped_gemm(bool swiglu, int tok, const GemmArgs& a, int grid, cudaStream_t s) {
   if (a.n_shared_groups + a.n_routed > kGemmMaxGroups) return cudaErrorInvalidValue;
   if (grid < 1) grid = 1;
-  cudaError_t e;
-  if (swiglu) {
-    e = cudaFuncSetAttribute(grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(Geo<true>::kSmemBytes));
-    if (e != cudaSuccess) return e;
-    grouped_gemm_kernel<true><<<grid, kThreads, Geo<true>::kSmemBytes, s>>>(a);
-  } else {
-    e = cudaFuncSetAttribute(grouped_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(Geo<false>::kSmemBytes));
-    if (e != cudaSuccess) return e;
-    grouped_gemm_kernel<false><<<grid, kThreads, Geo<false>::kSmemBytes, s>>>(a);
-  }
-  return cudaGetLastError();
+  if (tok == 256 && swiglu) return launch_one<true, 256>(a, grid, s);
+  if (tok != kGemmTokenTile) return cudaErrorInvalidValue;
+  return swiglu ? launch_one<true, kGemmTokenTile>(a, grid, s) : launch_one<false, kGemmTokenTile>(a, grid, s);
 }
 
 }  // namespace dsmoe

@@ -183,11 +183,18 @@ struct GemmF32Args {
 cudaError_t launch_gemm_f32_bf16(const GemmF32Args& a, cudaStream_t s);
 
 // ---------------------------------------------------------------- grouped GEMM (gemm_sm100.cu)
-// Tokens per grouped-GEMM tile of each projection (the row box of its token-side
-// tensor maps).
 constexpr int kGemmMaxGroups = 8 + 512;  // shared + routed groups of one grouped GEMM
-constexpr int kGemmGateUpTokenTile = 128;
-constexpr int kGemmDownTokenTile = 128;
+// Tokens per grouped-GEMM tile (the row box of the token-side tensor maps): 128, or 256
+// for the gate/up projection of layers with a long K loop and a few hundred rows per
+// expert, where the larger N moves fewer shared-memory bytes per MAC and the one
+// accumulator it leaves (the next tile waits for this tile's epilogue) costs less than
+// that saves (measured on the V3 shapes: d = 7168, about 256 rows per expert).
+constexpr int kGemmTokenTile = 128;
+constexpr int kGemmTokenTileLarge = 256;
+inline int gateup_token_tile(int d_model, int64_t routed_rows, int n_groups) {
+  return (d_model >= 4096 && n_groups > 0 && routed_rows >= 192LL * n_groups) ? kGemmTokenTileLarge
+                                                                              : kGemmTokenTile;
+}
 struct GemmArgs {
   CUtensorMap a_routed;   // 2D [rows, K] activations of routed slots, box (64, token tile)
   CUtensorMap a_shared;   // 2D [T, K_shared] activations of the shared groups, box (64, token tile)
@@ -219,7 +226,9 @@ struct GemmArgs {
   bf16* save_ab_routed;
   bf16* save_ab_shared;
 };
-cudaError_t launch_grouped_gemm(bool swiglu, const GemmArgs& a, int grid, cudaStream_t s);
+// tok: the token tile, kGemmTokenTile, or kGemmTokenTileLarge for the gate/up projection
+// (the token maps' row box must equal it)
+cudaError_t launch_grouped_gemm(bool swiglu, int tok, const GemmArgs& a, int grid, cudaStream_t s);
 
 // The experts' backward GEMMs (gemm_bwd_sm100.cu). kBwdDM: da | db from dy and W_down;
 // kBwdDX: dx rows from da | db and W_gate, W_up. The weight maps b0 / b1 of `g` are 4-D

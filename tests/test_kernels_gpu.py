@@ -24,8 +24,10 @@ if not torch.cuda.is_available():
 # the tensor-core router; both are checked through the scores they report.
 # The grouped GEMMs run on the default one-CTA kernel; the "-pair" cases run the CTA-pair
 # kernel.
+# v3_slice at T=800 (d = 7168, 200 rows per expert on average) takes the 256-token gate/up
+# tiles, with experts of one and of two (evenly split) token tiles.
 CASES = [("tiny", 300, 0), ("tiny", 200, 0), ("gshard_c", 700, 0), ("ds2b", 900, 0), ("v4_decode_t64", 64, 0),
-         ("tiny", 300, 1), ("ds2b", 900, 1)]
+         ("v3_slice", 800, 0), ("tiny", 300, 1), ("ds2b", 900, 1)]
 
 
 @pytest.mark.parametrize("name,T,pair", CASES,
