@@ -60,6 +60,10 @@ def parse_args():
     ap.add_argument("--decode", default="v4_decode_t256,v4_decode_t16",
                     help="decode workloads timed after the main one at N=1 (comma list; empty: none)")
     ap.add_argument("--decode-steps", type=int, default=20)
+    ap.add_argument("--role-cycles", action="store_true",
+                    help="profiling run: load the role-cycle build of the library (build.py --role-cycles) and "
+                         "print, per grouped-GEMM launch kind, the SM clock and the share of cycles each role "
+                         "waited, instead of the benchmark line")
     return ap.parse_args()
 
 
@@ -367,15 +371,16 @@ def run_native(args, cfg):
     # ---- roofline of the dominant kernel
     peaks, peak_src = load_peaks()
     S = cfg.T * cfg.top_k
+    # the routed experts' GEMMs (the shared experts' run as their own stage, beside routing)
     flops = {
-        "gemm_gate_up": 2.0 * 2 * cfg.d_model * (S * cfg.d_ff + cfg.T * cfg.n_shared * cfg.d_ff_shared),
-        "gemm_down": 2.0 * cfg.d_model * (S * cfg.d_ff + cfg.T * cfg.n_shared * cfg.d_ff_shared),
+        "gemm_gate_up": 2.0 * 2 * cfg.d_model * S * cfg.d_ff,
+        "gemm_down": 2.0 * cfg.d_model * S * cfg.d_ff,
     }
     dom = max(flops, key=lambda k: stage_ms.get(k, 0.0))
     counts = out["counts"].cpu().numpy()
     touched = int((counts > 0).sum())
-    weight_bytes = {"gemm_gate_up": 2 * cfg.d_model * (touched * 2 * cfg.d_ff + cfg.n_shared * 2 * cfg.d_ff_shared),
-                    "gemm_down": 2 * cfg.d_model * (touched * cfg.d_ff + cfg.n_shared * cfg.d_ff_shared)}
+    weight_bytes = {"gemm_gate_up": 2 * cfg.d_model * touched * 2 * cfg.d_ff,
+                    "gemm_down": 2 * cfg.d_model * touched * cfg.d_ff}
     dom_ms = stage_ms[dom]
     intensity = flops[dom] / max(weight_bytes[dom], 1)
     tensor_key = tensor_peak_key(clock_info)
@@ -522,10 +527,11 @@ def time_decode(M, W, name, dev, stream, steps, warmup, peaks, peak_src):
     touched = int((out["counts"] > 0).sum())
     layer.close()
     d, F, Fs, Ks = cfg.d_model, cfg.d_ff, cfg.d_ff_shared, cfg.n_shared
-    w_gate_up = 2 * d * 2 * (touched * F + Ks * Fs)
-    w_down = 2 * d * (touched * F + Ks * Fs)
+    w_gate_up = 2 * d * 2 * touched * F   # the routed gate/up stage (the shared experts run beside routing)
+    w_shared = 2 * d * 3 * Ks * Fs
+    w_down = 2 * d * touched * F
     router = 0 if cfg.score == W.ROUTE_HASH else cfg.n_routed * d * 2
-    step_bytes = w_gate_up + w_down + router + 2 * cfg.T * d * 2
+    step_bytes = w_gate_up + w_down + w_shared + router + 2 * cfg.T * d * 2
     gbs = step_bytes / (ms / 1e3) / 1e9
     gu_gbs = w_gate_up / (stage_ms["gemm_gate_up"] / 1e3) / 1e9
     del inp, out
@@ -538,12 +544,67 @@ def time_decode(M, W, name, dev, stream, steps, warmup, peaks, peak_src):
             "stage_ms": stage_ms, "clocks": clock_info, "steps": steps, "warmup": warmup}
 
 
+def run_role_cycles(args, cfg):
+    """One GPU: W warm-up forwards, then K forwards whose grouped-GEMM role counters
+    (role_clock.cuh) are read back; one JSON line per launch kind with the mean over CTAs
+    of each role's share of the CTA's cycles, the SM clock (cycles / ns), the launch time
+    and the tensor work per clock cycle against the tensor cores' 8192 bf16 FLOP per SM
+    per cycle (dense)."""
+    os.environ.setdefault("DSMOE_LIBRARY", os.path.join(ROOT, "mixture_experts_layer_score_b200",
+                                                        "libdsmoe_rolecycles.so"))
+    import numpy as np
+    import torch
+    import workloads as W
+    import mixture_experts_layer_score_b200 as M
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    inp = W.make_inputs(cfg, seed=0, device=dev, with_weights=True)
+    layer = M.DSMoE(M.cfg_from(cfg, cfg.T), inp, device=0)
+    out = layer.alloc_outputs(cfg.T)
+    for _ in range(args.warmup):
+        layer.forward(inp["x"], token_ids=inp["token_ids"], out=out)
+    torch.cuda.synchronize(dev)
+    M.dsmoe_gemm_role_cycles()  # clears the counters
+    for _ in range(args.steps):
+        layer.forward(inp["x"], token_ids=inp["token_ids"], out=out)
+    torch.cuda.synchronize(dev)
+    rc = M.dsmoe_gemm_role_cycles().astype(np.float64)
+    if M.dsmoe_get_status(layer.handle) != M.DSMOE_OK:
+        raise SystemExit(f"device status: {M.dsmoe_last_error()}")
+    slots = int(out["counts"].sum().item())
+    layer.close()
+    d, F, T = cfg.d_model, cfg.d_ff, cfg.T
+    KsFs = cfg.n_shared * cfg.d_ff_shared
+    flops = {"gemm_gate_up": 4.0 * d * F * slots, "gemm_down": 2.0 * d * F * slots,
+             "shared_gate_up": 4.0 * d * KsFs * T, "shared_down": 2.0 * d * KsFs * T}
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    names = M.ROLE_SLOT_NAMES
+    for k, kind in enumerate(M.ROLE_KINDS):
+        b = rc[k]
+        b = b[b[:, 0] > 0]
+        if b.shape[0] == 0:
+            continue
+        cyc, ns = b[:, 0], b[:, 1]
+        share = {n: float((b[:, i] / cyc).mean()) for i, n in enumerate(names) if i >= 2 and n != "tiles"}
+        mhz = float((cyc / ns).mean() * 1e3)
+        launch_s = float(ns.max()) / args.steps * 1e-9
+        rec = {"workload": cfg.name, "kind": kind, "ctas": int(b.shape[0]), "steps": args.steps,
+               "sm_mhz": mhz, "us_per_launch": launch_s * 1e6, "tiles_per_cta": float(b[:, 8].mean() / args.steps),
+               "tflops": flops[kind] / launch_s / 1e12,
+               "tensor_per_cycle": flops[kind] / launch_s / (mhz * 1e6 * sms * 8192),
+               "share_of_cycles": share}
+        print(json.dumps(rec), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     import workloads as W
     cfg = W.get_config(args.workload)
     if args.impl == "reference":
         return run_reference(args, cfg)
+    if args.role_cycles:
+        return run_role_cycles(args, cfg)
     return run_native(args, cfg)
 
 

@@ -441,19 +441,37 @@ dsmoe_status dsmoe_backward_router(dsmoe_handle* h, int32_t T, const void* x, co
                                    const float* dg, const float* f, float alpha, float* dlogits, float* dx,
                                    float* dW_router, void* stream);
 
-/* Per-stage timing: while enabled, each forward with T > 0 records CUDA events on its
- * stream at every stage boundary (no synchronisation). dsmoe_stage_times waits for
- * the recorded events and writes, per stage, the mean duration in ms over the last
- * min(64, forwards recorded since timing was enabled) forwards. Enabling (or
- * disabling) timing resets the record. */
+/* Per-stage timing: while enabled, each forward with T > 0 records CUDA events at every
+ * stage boundary (no synchronisation): on its stream for the chain router -> select ->
+ * scan -> permute -> routed gate/up GEMM -> routed down GEMM -> combine, and on the
+ * handle's side stream around the shared experts' two GEMMs, which run concurrently with
+ * the routing stages (an empty interval without shared experts). dsmoe_stage_times waits
+ * for the recorded events and writes, per stage, the mean duration in ms over the last
+ * min(64, forwards recorded since timing was enabled) forwards. Enabling (or disabling)
+ * timing resets the record. */
 dsmoe_status dsmoe_set_timing(dsmoe_handle* h, int32_t enable);
 dsmoe_status dsmoe_stage_times(dsmoe_handle* h, float* ms, int32_t max_n, int32_t* n);
 /* Name of stage i ("router", "select", "scan", "permute", "gemm_gate_up", "gemm_down",
- * "combine"), or NULL past the last. */
+ * "combine", "shared_experts"), or NULL past the last. */
 const char* dsmoe_stage_name(int32_t i);
 
 /* Number of kernels this handle has launched since creation. */
 dsmoe_status dsmoe_launch_count(dsmoe_handle* h, int64_t* n);
+
+/* Role cycle counters of the one-CTA grouped GEMM, for profiling (a library built with
+ * DSMOE_ROLE_CYCLES defined: `build.py --role-cycles`). Copies the counters of the current
+ * device, summed over every launch since the last call, to out[n], n >= 4 * 160 * 9 = 5760
+ * (uint64, layout [launch kind][CTA 0..159][slot]; kinds: 0 down and 1 gate/up launches
+ * with routed groups, 2 down and 3 gate/up launches of the shared experts alone), and
+ * clears them.
+ * Slots: 0 clock64 cycles from CTA start to exit, 1 globaltimer ns over the same interval,
+ * 2 producer cycles waiting for a free ring stage, 3 MMA-thread cycles waiting for a
+ * landed stage, 4 MMA-thread cycles waiting for a free accumulator, 5 MMA-thread cycles
+ * in its tile loop, 6 epilogue (first warp) cycles waiting for a finished accumulator,
+ * 7 epilogue cycles in its tile loop, 8 tiles. Synchronous. Returns
+ * DSMOE_ERR_UNSUPPORTED from a library built without the counters, DSMOE_ERR_INVALID_ARG
+ * for a NULL or short buffer. */
+dsmoe_status dsmoe_gemm_role_cycles(uint64_t* out, int32_t n);
 
 /*
  * Device address and shape of one intermediate buffer of the handle's workspace, for

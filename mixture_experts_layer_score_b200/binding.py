@@ -13,7 +13,9 @@ import os
 from typing import Dict, Optional, Sequence
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libdsmoe.so")
+# DSMOE_LIBRARY selects another build of the library, e.g. the profiling build with the
+# grouped GEMM's role cycle counters (build.py --role-cycles)
+LIB_PATH = os.environ.get("DSMOE_LIBRARY") or os.path.join(_HERE, "libdsmoe.so")
 
 DSMOE_OK, DSMOE_ERR_INVALID_ARG, DSMOE_ERR_UNSUPPORTED, DSMOE_ERR_WORKSPACE, DSMOE_ERR_CUDA, \
     DSMOE_ERR_DEVICE_TIMEOUT = range(6)
@@ -32,8 +34,12 @@ ABI_FUNCTIONS = (
     "dsmoe_set_selection", "dsmoe_get_selection", "dsmoe_set_expert_range", "dsmoe_get_expert_range",
     "dsmoe_round_bf16", "dsmoe_backward_gates", "dsmoe_backward_router", "dsmoe_ep_route", "dsmoe_ep_experts",
     "dsmoe_ep_combine", "dsmoe_forward_host_async", "dsmoe_host_join", "dsmoe_host_sync", "dsmoe_set_training",
-    "dsmoe_backward_experts", "dsmoe_backward_weights",
+    "dsmoe_backward_experts", "dsmoe_backward_weights", "dsmoe_gemm_role_cycles",
 )
+ROLE_CTAS, ROLE_SLOTS = 160, 9
+ROLE_KINDS = ("gemm_down", "gemm_gate_up", "shared_down", "shared_gate_up")
+ROLE_SLOT_NAMES = ("cycles", "nanoseconds", "producer_wait_stage", "mma_wait_stage", "mma_wait_acc", "mma_loop",
+                   "epi_wait_acc", "epi_loop", "tiles")
 
 
 class DsmoeCfg(ctypes.Structure):
@@ -84,6 +90,7 @@ def _load():
         "dsmoe_stage_times": (ctypes.c_int, [vp, ctypes.POINTER(ctypes.c_float), i32, ctypes.POINTER(i32)]),
         "dsmoe_stage_name": (ctypes.c_char_p, [i32]),
         "dsmoe_launch_count": (ctypes.c_int, [vp, ctypes.POINTER(i64)]),
+        "dsmoe_gemm_role_cycles": (ctypes.c_int, [vp, i32]),
         "dsmoe_balance_losses": (ctypes.c_int, [vp, vp, vp, i32, vp, ctypes.c_float, ctypes.c_float, vp, vp, vp,
                                                 vp]),
         "dsmoe_sequence_balance": (ctypes.c_int, [vp, i32, i32, vp, vp, ctypes.c_float, vp, vp, vp, vp]),
@@ -335,6 +342,16 @@ def dsmoe_stage_times(handle) -> Dict[str, float]:
     n = ctypes.c_int32(0)
     _check(_lib.dsmoe_stage_times(handle, buf, len(names), ctypes.byref(n)), "dsmoe_stage_times")
     return {names[i]: float(buf[i]) for i in range(n.value)}
+
+
+def dsmoe_gemm_role_cycles():
+    """The one-CTA grouped GEMM's role counters since the last call, as a uint64 array
+    [launch kind, CTA, slot] (kinds ROLE_KINDS, slots ROLE_SLOT_NAMES); a profiling build
+    of the library is required (DsmoeError with DSMOE_ERR_UNSUPPORTED otherwise)."""
+    import numpy as np
+    buf = np.zeros((len(ROLE_KINDS), ROLE_CTAS, ROLE_SLOTS), dtype=np.uint64)
+    _check(_lib.dsmoe_gemm_role_cycles(buf.ctypes.data, buf.size), "dsmoe_gemm_role_cycles")
+    return buf
 
 
 def dsmoe_launch_count(handle) -> int:

@@ -19,6 +19,7 @@
 
 #include "dsmoe.h"
 #include "kernels.h"
+#include "role_clock.cuh"
 
 #define DSMOE_EXPORT extern "C" __attribute__((visibility("default")))
 
@@ -26,9 +27,14 @@ using dsmoe::bf16;
 
 namespace {
 
-constexpr int kNumStages = 7;
+// Stages 0-6 run one after another on the caller's stream (marks 0..7 bracket them);
+// the shared experts' two GEMMs (stage 7) run on the handle's side stream, concurrently
+// with the routing stages, between marks 8 and 9.
+constexpr int kNumStages = 8;
+constexpr int kChainStages = 7;
+constexpr int kNumMarks = kChainStages + 3;
 const char* const kStageNames[kNumStages] = {"router", "select", "scan", "permute", "gemm_gate_up", "gemm_down",
-                                             "combine"};
+                                             "combine", "shared_experts"};
 constexpr int kSelectMaxBlocks = 1024;  // rows of the statistics partials
 constexpr int kTimingSlots = 64;        // forwards whose stage events are kept
 constexpr int kTcRouterMinTokens = 256; // below this the CUDA-core router spreads over more SMs
@@ -234,6 +240,10 @@ struct dsmoe_handle {
   cudaStream_t copy_stream_out = nullptr;  // output copies (both directions run at once)
   cudaEvent_t ev_in[2] = {}, ev_out[2] = {}, ev_d2h[2] = {};
   int64_t async_calls = 0;
+  // the shared experts' GEMMs depend on x alone: they run on this stream, forked from and
+  // joined back into the caller's stream, while the routing stages run
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   CUtensorMap tm_a1, tm_a1s;
   // weight maps, cached per pointer: W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, W_router
   // (the gate/up maps serve both GEMM kernels), then W_down and Ws_down for the pair down GEMM
@@ -245,7 +255,7 @@ struct dsmoe_handle {
   uint32_t rt_cols = 32;
   bool timing = false;
   int timed_forwards = 0;               // forwards recorded since timing was enabled
-  cudaEvent_t ev[kTimingSlots][kNumStages + 1] = {};
+  cudaEvent_t ev[kTimingSlots][kNumMarks] = {};
   int64_t launches = 0;
   int32_t ep_T = -1;  // tokens of the last dsmoe_ep_route (its slot table is in the workspace)
   // training buffers (dsmoe_set_training): the forward's saved pre-activations a | b, and
@@ -327,8 +337,11 @@ static void release(dsmoe_handle* h) {
   for (int i = 0; i < 2; ++i)
     for (cudaEvent_t e : {h->ev_in[i], h->ev_out[i], h->ev_d2h[i]})
       if (e) cudaEventDestroy(e);
+  if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+  if (h->ev_join) cudaEventDestroy(h->ev_join);
   if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
   if (h->copy_stream_out) cudaStreamDestroy(h->copy_stream_out);
+  if (h->side) cudaStreamDestroy(h->side);
   if (h->tr) cudaFree(h->tr);
   if (h->ws) cudaFree(h->ws);
   delete h;
@@ -423,6 +436,9 @@ DSMOE_EXPORT dsmoe_status dsmoe_create(const dsmoe_cfg* cfg, int32_t device, dsm
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->copy_stream_out, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming);
   if (e != cudaSuccess) {
     release(h);
     return fail(DSMOE_ERR_CUDA, "event or stream creation failed: %s", cudaGetErrorString(e));
@@ -658,7 +674,8 @@ dsmoe_status gemm_stage(dsmoe_handle* h, const GemmPlan& p, cudaStream_t s,
   // ---- gate/up GEMM with SiLU(gate) * up
   {
     // token tile of this launch (the pair kernel stages 128 of its 256 token rows per CTA)
-    const int tok = pair ? dsmoe::kGemmTokenTile : dsmoe::gateup_token_tile(d, p.routed_rows, p.n_groups);
+    const int tok = pair ? dsmoe::kGemmTokenTile
+                         : dsmoe::gateup_token_tile(d, p.routed_rows + static_cast<int64_t>(T) * Ks, p.n_groups + Ks);
     CUtensorMap m_rows, m_x;
     bool ok = true;
     if (p.n_groups > 0) ok = map_2d(&m_rows, p.rows, d, p.rows_extent, tok);
@@ -819,30 +836,55 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
   if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map of this call");
 
   CUDA_TRY(mark(0));
+  if (Ks > 0) {  // the side stream starts after everything the caller queued before this call
+    CUDA_TRY(cudaEventRecord(h->ev_fork, s));
+    CUDA_TRY(cudaStreamWaitEvent(h->side, h->ev_fork, 0));
+  }
   int sel_grid = 0;
   STAGE_TRY(route_stage(h, a, s, &sel_grid, mark));
+  p.x = a.x;
+  p.T = T;
+  p.residual = static_cast<const bf16*>(a.x);
+  p.save_ab = h->tr != nullptr;
+  p.offsets = h->offsets + e0;
+  p.expert_mod = 0;
+  const std::function<cudaError_t(int)> no_mark = [](int) { return cudaSuccess; };
+  if (Ks > 0) {
+    // shared experts (gate/up into A1s, down into Hs with the residual), queued after the
+    // router so that its CTAs are placed first; the permute's CTAs fit beside these GEMMs'
+    if (timing) CUDA_TRY(cudaEventRecord(evs[kChainStages + 1], h->side));
+    GemmPlan sp = p;
+    sp.rows = a.x;
+    sp.rows_extent = static_cast<uint64_t>(T);
+    sp.n_groups = 0;
+    sp.routed_rows = 0;
+    sp.Ks = Ks;
+    sp.Y_out = nullptr;
+    STAGE_TRY(gemm_stage(h, sp, h->side, no_mark));
+    if (timing) CUDA_TRY(cudaEventRecord(evs[kChainStages + 2], h->side));
+    CUDA_TRY(cudaEventRecord(h->ev_join, h->side));
+  }
   CUDA_TRY(mark(2));
   STAGE_TRY(scan_permute_stage(h, a, s, sel_grid, e0, e0 + NL, mark));
   CUDA_TRY(mark(4));
   p.rows = h->Xp;
   p.rows_extent = static_cast<uint64_t>(c.max_tokens) * c.top_k;
-  p.x = a.x;
-  p.offsets = h->offsets + e0;
   p.n_groups = NL;
-  p.expert_mod = 0;
   p.routed_rows = static_cast<int64_t>(T) * K;
-  p.T = T;
-  p.Ks = Ks;
-  p.residual = static_cast<const bf16*>(a.x);
+  p.Ks = 0;
   p.Y_out = h->Y;
-  p.save_ab = h->tr != nullptr;
   STAGE_TRY(gemm_stage(h, p, s, mark));
+  if (Ks > 0) CUDA_TRY(cudaStreamWaitEvent(s, h->ev_join, 0));
   if (h->tr) {
     h->saved_T = T;
     h->dab_ready = false;
   }
   STAGE_TRY(combine_stage(h, a, h->Y, Ks, h->add_shared, h->partial, s));
   CUDA_TRY(mark(7));
+  if (timing && Ks == 0) {  // no shared-expert stage: an empty interval
+    CUDA_TRY(cudaEventRecord(evs[kChainStages + 1], s));
+    CUDA_TRY(cudaEventRecord(evs[kChainStages + 2], s));
+  }
   if (timing) h->timed_forwards += 1;
   return DSMOE_OK;
 }
@@ -1564,10 +1606,13 @@ DSMOE_EXPORT dsmoe_status dsmoe_stage_times(dsmoe_handle* h, float* ms, int32_t 
   for (int i = 0; i < cnt; ++i) ms[i] = 0.f;
   for (int f = 0; f < kept; ++f) {
     cudaEvent_t* evs = h->ev[(h->timed_forwards - 1 - f) % kTimingSlots];
-    CUDA_TRY(cudaEventSynchronize(evs[kNumStages]));
+    CUDA_TRY(cudaEventSynchronize(evs[kChainStages]));
+    CUDA_TRY(cudaEventSynchronize(evs[kChainStages + 2]));
     for (int i = 0; i < cnt; ++i) {
+      // chain stages: consecutive marks; the shared experts: their own pair of marks
+      const int m0 = i < kChainStages ? i : kChainStages + 1;
       float v = 0.f;
-      CUDA_TRY(cudaEventElapsedTime(&v, evs[i], evs[i + 1]));
+      CUDA_TRY(cudaEventElapsedTime(&v, evs[m0], evs[m0 + 1]));
       ms[i] += v / kept;
     }
   }
@@ -1577,6 +1622,16 @@ DSMOE_EXPORT dsmoe_status dsmoe_stage_times(dsmoe_handle* h, float* ms, int32_t 
 
 DSMOE_EXPORT const char* dsmoe_stage_name(int32_t i) {
   return (i >= 0 && i < kNumStages) ? kStageNames[i] : nullptr;
+}
+
+DSMOE_EXPORT dsmoe_status dsmoe_gemm_role_cycles(uint64_t* out, int32_t n) {
+  if (!out || n < dsmoe::kRoleCounters)
+    return fail(DSMOE_ERR_INVALID_ARG, "a buffer of %d counters is required", dsmoe::kRoleCounters);
+  cudaError_t e = cudaSuccess;
+  if (!dsmoe::read_role_cycles(reinterpret_cast<unsigned long long*>(out), &e))
+    return fail(DSMOE_ERR_UNSUPPORTED, "this library was built without the role cycle counters");
+  if (e != cudaSuccess) return fail(DSMOE_ERR_CUDA, "reading the role counters failed: %s", cudaGetErrorString(e));
+  return DSMOE_OK;
 }
 
 DSMOE_EXPORT dsmoe_status dsmoe_launch_count(dsmoe_handle* h, int64_t* n) {

@@ -44,11 +44,27 @@
 // finish (a wait bounded by at least one second, whatever the caller's limit), frees its
 // TMEM and returns.
 #include "grouped_tiles.cuh"
+#include "role_clock.cuh"
 #include "sm100_ptx.cuh"
 
 namespace dsmoe {
 
+#ifdef DSMOE_ROLE_CYCLES
+__device__ unsigned long long g_role_cycles[kRoleKernels][kRoleCtas][kRsSlots];
+#endif
+
 namespace {
+// Adds v to this CTA's counter `slot` of kernel `k` (profiling builds only).
+__device__ __forceinline__ void role_add(int k, int slot, long long v) {
+#ifdef DSMOE_ROLE_CYCLES
+  if (blockIdx.x < kRoleCtas) atomicAdd(&g_role_cycles[k][blockIdx.x][slot], static_cast<unsigned long long>(v));
+#else
+  (void)k;
+  (void)slot;
+  (void)v;
+#endif
+}
+
 constexpr int kBK = 64;         // K per ring stage (one 128-byte swizzled row of bf16)
 constexpr int kFeat = 128;      // output features per MMA chain (the MMA's M, TMEM lanes)
 constexpr int kMmaK = 16;       // K of each bf16 tcgen05.mma
@@ -85,6 +101,10 @@ struct Geo {
 template <bool kSwiGLU, int kTok>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs a) {
   using G_ = Geo<kTok>;
+  RoleClock rc_kernel;
+  rc_kernel.start();
+  const unsigned long long rc_ns0 = role_ns();
+  const int rk = (kSwiGLU ? 1 : 0) + (a.n_routed == 0 ? 2 : 0);  // role counter set
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_addr(smem_raw) & 1023u)) & 1023u;
   uint8_t* base = smem_raw + pad;
@@ -142,6 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      RoleClock rc_wait;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
         const Tile t = decode_tile<kTok>(a, tile_start, G, tile);
         const CUtensorMap* tx = t.shared ? &a.a_shared : &a.a_routed;
@@ -149,10 +170,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         const CUtensorMap* tw1 = t.shared ? &a.b1_shared : &a.b1_routed;
         const int kb_per = t.shared ? a.kb_per_b_expert_shared : t.kb_n;
         for (int kb = 0; kb < t.kb_n; ++kb) {
+          rc_wait.start();
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, a.wait_limit_ns, abort_flag)) {
             ok = false;
             break;
           }
+          rc_wait.stop();
           mbar_arrive_expect_tx(&full[stage], G_::kStageBytes);
           const int be = t.expert + kb / kb_per;
           const int bk = (kb % kb_per) * kBK;
@@ -176,6 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         *abort_flag = 1;
         atomicOr(a.status, kStatusTimeoutProducer);
       }
+      role_add(rk, kRsProducerWaitStage, rc_wait.total);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -184,22 +208,28 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       uint32_t phase = 0;
       bool ok = true;
       int it = 0;
+      RoleClock rc_loop, rc_stage, rc_acc;
+      rc_loop.start();
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++it) {
         const Tile t = decode_tile<kTok>(a, tile_start, G, tile);
         const int n_mma = (t.m_valid + 15) & ~15;  // tokens, rounded up to the MMA's N step
         const uint32_t idesc = idesc_bf16_f32(kFeat, n_mma);
         const int acc = it % G_::kBufs;
+        rc_acc.start();
         if (!mbar_wait_bounded(&acc_empty[acc], ((it / G_::kBufs) & 1) ^ 1u, a.wait_limit_ns, abort_flag)) {
           ok = false;
           break;
         }
+        rc_acc.stop();
         tc_fence_after();
         const uint32_t d0 = tmem_base + acc * G_::kAccCols;
         for (int kb = 0; kb < t.kb_n; ++kb) {
+          rc_stage.start();
           if (!mbar_wait_bounded(&full[stage], phase, a.wait_limit_ns, abort_flag)) {
             ok = false;
             break;
           }
+          rc_stage.stop();
           tc_fence_after();
           const uint64_t w0 = smem_desc_kmajor_sw128(smem_addr(sW + stage * kWBytes));
           const uint64_t w1 = smem_desc_kmajor_sw128(smem_addr(sW + stage * kWBytes + kWBytes / 2));
@@ -224,6 +254,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         *abort_flag = 1;
         atomicOr(a.status, kStatusTimeoutMma);
       }
+      rc_loop.stop();
+      role_add(rk, kRsMmaWaitStage, rc_stage.total);
+      role_add(rk, kRsMmaWaitAcc, rc_acc.total);
+      role_add(rk, kRsMmaLoop, rc_loop.total);
+      role_add(rk, kRsTiles, it);
     }
   } else {
     // -------------------------------------------------------------------- epilogue
@@ -238,9 +273,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
     float* stgf = reinterpret_cast<float*>(stg_raw);       // [16 tokens][kStgRowF] fp32
     const int rr = lane >> 2, cc = (lane & 3) * 8;  // read-out: row (plus 8i), first feature
     int it = 0;
+    RoleClock rc_loop, rc_acc;
+    rc_loop.start();
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
       const Tile t = decode_tile<kTok>(a, tile_start, G, tile);
       const int acc = it % G_::kBufs;
+      rc_acc.start();
       if (!mbar_wait_warp_sleepy(&acc_full[acc], (it / G_::kBufs) & 1, a.wait_limit_ns, abort_flag)) {
         if (lane == 0) {
           *abort_flag = 1;
@@ -248,6 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         }
         break;
       }
+      rc_acc.stop();
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * G_::kAccCols;
       const int n_valid = t.shared ? a.n_valid_shared : a.n_valid_routed;
@@ -372,6 +411,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
     }
+    rc_loop.stop();
+    if (warp == 2 && lane == 0) {
+      role_add(rk, kRsEpiWaitAcc, rc_acc.total);
+      role_add(rk, kRsEpiLoop, rc_loop.total);
+    }
   }
 
   __syncthreads();
@@ -395,6 +439,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
+  if (threadIdx.x == 0) {
+    rc_kernel.stop();
+    role_add(rk, kRsCycles, rc_kernel.total);
+    role_add(rk, kRsNanoseconds, static_cast<long long>(role_ns() - rc_ns0));
+  }
 }
 }  // namespace
 
@@ -408,6 +457,19 @@ cudaError_t launch_one(const GemmArgs& a, int grid, cudaStream_t s) {
   return cudaGetLastError();
 }
 }  // namespace
+
+bool read_role_cycles(unsigned long long* host, cudaError_t* err) {
+#ifdef DSMOE_ROLE_CYCLES
+  static unsigned long long zeros[kRoleCounters];
+  *err = cudaMemcpyFromSymbol(host, g_role_cycles, sizeof(zeros));
+  if (*err == cudaSuccess) *err = cudaMemcpyToSymbol(g_role_cycles, zeros, sizeof(zeros));
+  return true;
+#else
+  (void)host;
+  *err = cudaSuccess;
+  return false;
+#endif
+}
 
 cudaError_t launch_grouped_gemm(bool swiglu, int tok, const GemmArgs& a, int grid, cudaStream_t s) {
   if (a.n_shared_groups + a.n_routed > kGemmMaxGroups) return cudaErrorInvalidValue;

@@ -191,9 +191,9 @@ constexpr int kGemmMaxGroups = 8 + 512;  // shared + routed groups of one groupe
 // that saves (measured on the V3 shapes: d = 7168, about 256 rows per expert).
 constexpr int kGemmTokenTile = 128;
 constexpr int kGemmTokenTileLarge = 256;
-inline int gateup_token_tile(int d_model, int64_t routed_rows, int n_groups) {
-  return (d_model >= 4096 && n_groups > 0 && routed_rows >= 192LL * n_groups) ? kGemmTokenTileLarge
-                                                                              : kGemmTokenTile;
+// rows, groups: the token rows and the groups (routed and shared) of the launch
+inline int gateup_token_tile(int d_model, int64_t rows, int groups) {
+  return (d_model >= 4096 && groups > 0 && rows >= 192LL * groups) ? kGemmTokenTileLarge : kGemmTokenTile;
 }
 struct GemmArgs {
   CUtensorMap a_routed;   // 2D [rows, K] activations of routed slots, box (64, token tile)
@@ -229,6 +229,9 @@ struct GemmArgs {
 // tok: the token tile, kGemmTokenTile, or kGemmTokenTileLarge for the gate/up projection
 // (the token maps' row box must equal it)
 cudaError_t launch_grouped_gemm(bool swiglu, int tok, const GemmArgs& a, int grid, cudaStream_t s);
+// Profiling builds (DSMOE_ROLE_CYCLES, role_clock.cuh): copy the one-CTA grouped GEMM's role
+// counters to host[kRoleCounters] and clear them; false in any other build.
+bool read_role_cycles(unsigned long long* host, cudaError_t* err);
 
 // The experts' backward GEMMs (gemm_bwd_sm100.cu). kBwdDM: da | db from dy and W_down;
 // kBwdDX: dx rows from da | db and W_gate, W_up. The weight maps b0 / b1 of `g` are 4-D

@@ -130,7 +130,9 @@ __device__ __forceinline__ float score_sqrt_softplus(float l) {
 
 template <int kNPL>
 __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(const SelectArgs a) {
-  __shared__ float red[kSelWarps][kNPL * 32];
+  // 4 KB at kNPL = 8, so that a block fits on an SM beside a grouped-GEMM CTA (the shared
+  // experts' GEMMs run concurrently with this kernel)
+  __shared__ float red[kSelWarps / 2][kNPL * 32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = a.N, K = a.K;
   float pacc[kNPL];
@@ -244,14 +246,23 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(const SelectArgs
         if (lane + 32 * j < N) srow[lane + 32 * j] = s[j];
     }
   }
-  // per-block partial sums of the scores, reduced over warps in a fixed order
+  // per-block partial sums of the scores, reduced over warps in a fixed order: warp w + 4
+  // into row w, warp w adds its own, then the 4 rows in order
+  constexpr int kHalf = kSelWarps / 2;
+  if (warp >= kHalf) {
 #pragma unroll
-  for (int j = 0; j < kNPL; ++j) red[warp][lane + 32 * j] = pacc[j];
+    for (int j = 0; j < kNPL; ++j) red[warp - kHalf][lane + 32 * j] = pacc[j];
+  }
+  __syncthreads();
+  if (warp < kHalf) {
+#pragma unroll
+    for (int j = 0; j < kNPL; ++j) red[warp][lane + 32 * j] += pacc[j];
+  }
   __syncthreads();
   for (int i = threadIdx.x; i < N; i += blockDim.x) {
     float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < kSelWarps; ++w) v += red[w][i];
+    for (int w = 0; w < kHalf; ++w) v += red[w][i];
     a.P_part[static_cast<int64_t>(blockIdx.x) * N + i] = v;
   }
 }

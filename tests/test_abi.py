@@ -33,7 +33,8 @@ def test_abi_version_and_status_strings():
     names = [M.dsmoe_status_string(i) for i in range(6)]
     assert names[0] == "ok" and len(set(names)) == 6
     assert M.dsmoe_status_string(99) == "unknown status"
-    assert M.stage_names() == ["router", "select", "scan", "permute", "gemm_gate_up", "gemm_down", "combine"]
+    assert M.stage_names() == ["router", "select", "scan", "permute", "gemm_gate_up", "gemm_down", "combine",
+                              "shared_experts"]
 
 
 @pytest.mark.parametrize("name", sorted(W.CONFIGS))
@@ -97,3 +98,17 @@ def test_null_handle_is_rejected_without_a_gpu():
     with pytest.raises(M.DsmoeError):
         M.dsmoe_set_gemm_kernel(None, M.DSMOE_GEMM_SINGLE)
     assert M.dsmoe_get_gemm_kernel(None) == -1
+
+
+def test_role_cycle_counters_need_the_profiling_build():
+    """The default library carries no role counters: the call says so before touching a GPU;
+    a short buffer is rejected first."""
+    if os.environ.get("DSMOE_LIBRARY"):
+        pytest.skip("a non-default library build is loaded")
+    lib = ctypes.CDLL(M.LIB_PATH)
+    lib.dsmoe_gemm_role_cycles.argtypes = [ctypes.c_void_p, ctypes.c_int32]
+    buf = (ctypes.c_uint64 * 8)()
+    assert lib.dsmoe_gemm_role_cycles(buf, 8) == M.DSMOE_ERR_INVALID_ARG
+    with pytest.raises(M.DsmoeError) as ei:
+        M.dsmoe_gemm_role_cycles()
+    assert ei.value.status == M.DSMOE_ERR_UNSUPPORTED

@@ -238,12 +238,14 @@ def test_stage_timing_and_launch_count():
     layer.forward(gpu["x"])
     t = M.dsmoe_stage_times(layer.handle)
     assert list(t) == M.stage_names() and all(v >= 0 for v in t.values())
-    # router logits (tensor cores for T >= 256), select, scan, permute, two GEMMs, combine
-    assert M.dsmoe_launch_count(layer.handle) - n0 == 7
+    # router logits (tensor cores for T >= 256), select, scan, permute, the routed experts'
+    # two GEMMs, combine; and the shared experts' two GEMMs on the side stream
+    n_launch = 7 + (2 if cfg.n_shared else 0)
+    assert M.dsmoe_launch_count(layer.handle) - n0 == n_launch
     M.dsmoe_set_timing(layer.handle, False)
     n1 = M.dsmoe_launch_count(layer.handle)
     layer.forward(gpu["x"][:100].contiguous())  # CUDA-core router logits below 256 tokens
-    assert M.dsmoe_launch_count(layer.handle) - n1 == 7
+    assert M.dsmoe_launch_count(layer.handle) - n1 == n_launch
     layer.close()
 
 
