@@ -60,6 +60,9 @@ def parse_args():
     ap.add_argument("--decode", default="v4_decode_t256,v4_decode_t16",
                     help="decode workloads timed after the main one at N=1 (comma list; empty: none)")
     ap.add_argument("--decode-steps", type=int, default=20)
+    ap.add_argument("--backward", action="store_true",
+                    help="time a training step instead (forward saving the pre-activations, gate, router, "
+                         "expert input and weight gradients) and print one JSON line of stage times and rates")
     ap.add_argument("--role-cycles", action="store_true",
                     help="profiling run: load the role-cycle build of the library (build.py --role-cycles) and "
                          "print, per grouped-GEMM launch kind, the SM clock and the share of cycles each role "
@@ -544,6 +547,96 @@ def time_decode(M, W, name, dev, stream, steps, warmup, peaks, peak_src):
             "stage_ms": stage_ms, "clocks": clock_info, "steps": steps, "warmup": warmup}
 
 
+def run_backward(args, cfg):
+    """One GPU: W warm-up and K timed training steps of the layer (an upstream gradient dh
+    drawn once): the forward with the pre-activations saved, then dsmoe_backward_gates,
+    dsmoe_backward_router (expert-level balance term, alpha 0.01), dsmoe_backward_experts
+    and dsmoe_backward_weights, each bracketed by CUDA events on the launching stream.
+    Prints one JSON line: per stage ms and its MMA work's TFLOP/s (the GEMM stages), the
+    step's time and tokens/s; weight gradients are fp32, summed over the step's tokens."""
+    import numpy as np
+    import torch
+    import workloads as W
+    import mixture_experts_layer_score_b200 as M
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    inp = W.make_inputs(cfg, seed=0, device=dev, with_weights=True)
+    T, d, N, K, F = cfg.T, cfg.d_model, cfg.n_routed, cfg.top_k, cfg.d_ff
+    Ks, Fs = cfg.n_shared, cfg.d_ff_shared
+    layer = M.DSMoE(M.cfg_from(cfg, T), inp, device=0)
+    M.dsmoe_set_training(layer.handle, True)
+    out = layer.alloc_outputs(T, with_scores=True)
+    dh = W.normal_bf16((T, d), 1.0, 0, "dh", 0, dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    dg = torch.empty((T, K), **f32)
+    dY = torch.empty((T * K, d), dtype=torch.bfloat16, device=dev)
+    hash_route = cfg.score == W.ROUTE_HASH
+    dl = torch.empty((T, N), **f32)
+    dx_r = torch.zeros((T, d), **f32)
+    dWr = torch.empty((N, d), **f32)
+    dx = torch.empty((T, d), **f32)
+    dW = [torch.empty(shp, **f32) for shp in ((N, F, d), (N, F, d), (N, d, F))]
+    dWs = [torch.empty(shp, **f32) if Ks else None for shp in ((Ks, Fs, d), (Ks, Fs, d), (Ks, d, Fs))]
+    stream = torch.cuda.current_stream(dev)
+    names = ["forward", "gates", "router", "experts_input", "experts_weights"]
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+    acc = {n: 0.0 for n in names}
+
+    def step(timed):
+        if timed:
+            ev[0].record(stream)
+        layer.forward(inp["x"], token_ids=inp["token_ids"], out=out, stream=stream)
+        if timed:
+            ev[1].record(stream)
+        M.dsmoe_backward_gates(layer.handle, T, dh, out["gates"], dg, dY, stream=stream)
+        if timed:
+            ev[2].record(stream)
+        if not hash_route:
+            M.dsmoe_backward_router(layer.handle, T, inp["x"], inp["W_router"], out["topk_idx"], out["gates"],
+                                    out["scores"], dg, out["f"], 0.01, dl, dx_r, dWr, stream=stream)
+        if timed:
+            ev[3].record(stream)
+        M.dsmoe_backward_experts(layer.handle, T, dh, dY, inp["W_gate"], inp["W_up"], inp["W_down"],
+                                 inp.get("Ws_gate"), inp.get("Ws_up"), inp.get("Ws_down"), dx_r, dx, stream=stream)
+        if timed:
+            ev[4].record(stream)
+        M.dsmoe_backward_weights(layer.handle, T, dh, dY, inp["x"], dW[0], dW[1], dW[2], dWs[0], dWs[1], dWs[2],
+                                 stream=stream)
+        if timed:
+            ev[5].record(stream)
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(True)
+        torch.cuda.synchronize(dev)  # read this step's stage events
+        for i, n in enumerate(names):
+            acc[n] += ev[i].elapsed_time(ev[i + 1]) / args.steps
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if M.dsmoe_get_status(layer.handle) != M.DSMOE_OK:
+        raise SystemExit(f"device status: {M.dsmoe_last_error()}")
+    layer.close()
+    S = T * K
+    flops = {"forward": cfg.flops_per_token() * T,
+             # dm = W_down^T dy (+ SiLU backward), then du = W_gate^T da + W_up^T db
+             "experts_input": 2.0 * d * F * S * 3 + 2.0 * d * Ks * Fs * T * 3,
+             # dW_down, dW_gate, dW_up
+             "experts_weights": 2.0 * d * F * S * 3 + 2.0 * d * Ks * Fs * T * 3}
+    step_ms = sum(acc.values())
+    rec = {"metric": "DeepSeekMoE layer training step (forward + backward) tokens/s on 1 B200",
+           "workload": cfg.name, "steps": args.steps, "warmup": args.warmup, "dtype": "bf16 (fp32 accumulation, "
+           "fp32 weight gradients)", "step_ms": step_ms, "tokens_per_s": T / (step_ms / 1e3),
+           "stage_ms": acc, "stage_tflops": {k: flops[k] / (acc[k] / 1e3) / 1e12 for k in flops},
+           "step_tflops": sum(flops.values()) / (step_ms / 1e3) / 1e12,
+           "note": "stage events on the launching stream, the host synchronising after each step"}
+    print(json.dumps(rec), flush=True)
+    return 0
+
+
 def run_role_cycles(args, cfg):
     """One GPU: W warm-up forwards, then K forwards whose grouped-GEMM role counters
     (role_clock.cuh) are read back; one JSON line per launch kind with the mean over CTAs
@@ -605,6 +698,8 @@ def main():
         return run_reference(args, cfg)
     if args.role_cycles:
         return run_role_cycles(args, cfg)
+    if args.backward:
+        return run_backward(args, cfg)
     return run_native(args, cfg)
 
 
