@@ -553,7 +553,12 @@ def run_backward(args, cfg):
     dsmoe_backward_router (expert-level balance term, alpha 0.01), dsmoe_backward_experts
     and dsmoe_backward_weights, each bracketed by CUDA events on the launching stream.
     Prints one JSON line: per stage ms and its MMA work's TFLOP/s (the GEMM stages), the
-    step's time and tokens/s; weight gradients are fp32, summed over the step's tokens."""
+    step's time and tokens/s; weight gradients are fp32, summed over the step's tokens.
+    With --role-cycles (the profiling build) it also prints the weight-gradient GEMM's role
+    counters over the timed steps."""
+    if args.role_cycles:
+        os.environ.setdefault("DSMOE_LIBRARY", os.path.join(ROOT, "mixture_experts_layer_score_b200",
+                                                            "libdsmoe_rolecycles.so"))
     import numpy as np
     import torch
     import workloads as W
@@ -608,6 +613,8 @@ def run_backward(args, cfg):
     for _ in range(args.warmup):
         step(False)
     torch.cuda.synchronize(dev)
+    if args.role_cycles:
+        M.dsmoe_gemm_role_cycles()  # clears the counters
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
@@ -619,6 +626,7 @@ def run_backward(args, cfg):
     torch.cuda.synchronize(dev)
     if M.dsmoe_get_status(layer.handle) != M.DSMOE_OK:
         raise SystemExit(f"device status: {M.dsmoe_last_error()}")
+    roles = M.dsmoe_gemm_role_cycles().astype(np.float64) if args.role_cycles else None
     layer.close()
     S = T * K
     flops = {"forward": cfg.flops_per_token() * T,
@@ -634,6 +642,14 @@ def run_backward(args, cfg):
            "step_tflops": sum(flops.values()) / (step_ms / 1e3) / 1e12,
            "note": "stage events on the launching stream, the host synchronising after each step"}
     print(json.dumps(rec), flush=True)
+    if roles is not None:
+        b = roles[M.ROLE_KINDS.index("weight_grad")]
+        b = b[b[:, 0] > 0]
+        cyc, ns = b[:, 0], b[:, 1]
+        share = {n: float((b[:, i] / cyc).mean()) for i, n in enumerate(M.ROLE_SLOT_NAMES) if i >= 2 and n != "tiles"}
+        print(json.dumps({"workload": cfg.name, "kind": "weight_grad", "ctas": int(b.shape[0]), "steps": args.steps,
+                          "sm_mhz": float((cyc / ns).mean() * 1e3), "us_per_step": float(ns.max()) / args.steps / 1e3,
+                          "tiles_per_cta": float(b[:, 8].mean() / args.steps), "share_of_cycles": share}), flush=True)
     return 0
 
 
@@ -696,10 +712,10 @@ def main():
     cfg = W.get_config(args.workload)
     if args.impl == "reference":
         return run_reference(args, cfg)
-    if args.role_cycles:
-        return run_role_cycles(args, cfg)
     if args.backward:
         return run_backward(args, cfg)
+    if args.role_cycles:
+        return run_role_cycles(args, cfg)
     return run_native(args, cfg)
 
 

@@ -427,7 +427,9 @@ dsmoe_status dsmoe_backward_gates(dsmoe_handle* h, int32_t T, const void* dh, co
  *                        (all three NULL iff the handle adds no shared experts)
  *   Grouped GEMMs on the tensor cores reducing over token rows (both operands MN-major,
  *   each routed expert's rows a ragged K range), fp32 accumulation of bf16 products.
- *   An expert no token picked gets a zero gradient.
+ *   An expert no token picked gets a zero gradient. The six gradient buffers must be
+ *   32-byte aligned (rows are stored as 32-byte vectors), dh, dY and x 16-byte aligned;
+ *   else DSMOE_ERR_INVALID_ARG.
  */
 dsmoe_status dsmoe_backward_weights(dsmoe_handle* h, int32_t T, const void* dh, const void* dY, const void* x,
                                     float* dW_gate, float* dW_up, float* dW_down, float* dWs_gate, float* dWs_up,
@@ -458,12 +460,12 @@ const char* dsmoe_stage_name(int32_t i);
 /* Number of kernels this handle has launched since creation. */
 dsmoe_status dsmoe_launch_count(dsmoe_handle* h, int64_t* n);
 
-/* Role cycle counters of the one-CTA grouped GEMM, for profiling (a library built with
+/* Role cycle counters of the grouped GEMMs, for profiling (a library built with
  * DSMOE_ROLE_CYCLES defined: `build.py --role-cycles`). Copies the counters of the current
- * device, summed over every launch since the last call, to out[n], n >= 4 * 160 * 9 = 5760
+ * device, summed over every launch since the last call, to out[n], n >= 5 * 160 * 9 = 7200
  * (uint64, layout [launch kind][CTA 0..159][slot]; kinds: 0 down and 1 gate/up launches
- * with routed groups, 2 down and 3 gate/up launches of the shared experts alone), and
- * clears them.
+ * with routed groups, 2 down and 3 gate/up launches of the shared experts alone, 4 the
+ * weight-gradient GEMM of dsmoe_backward_weights), and clears them.
  * Slots: 0 clock64 cycles from CTA start to exit, 1 globaltimer ns over the same interval,
  * 2 producer cycles waiting for a free ring stage, 3 MMA-thread cycles waiting for a
  * landed stage, 4 MMA-thread cycles waiting for a free accumulator, 5 MMA-thread cycles

@@ -37,7 +37,7 @@ ABI_FUNCTIONS = (
     "dsmoe_backward_experts", "dsmoe_backward_weights", "dsmoe_gemm_role_cycles",
 )
 ROLE_CTAS, ROLE_SLOTS = 160, 9
-ROLE_KINDS = ("gemm_down", "gemm_gate_up", "shared_down", "shared_gate_up")
+ROLE_KINDS = ("gemm_down", "gemm_gate_up", "shared_down", "shared_gate_up", "weight_grad")
 ROLE_SLOT_NAMES = ("cycles", "nanoseconds", "producer_wait_stage", "mma_wait_stage", "mma_wait_acc", "mma_loop",
                    "epi_wait_acc", "epi_loop", "tiles")
 

@@ -244,56 +244,81 @@ __global__ void __launch_bounds__(128) dx_combine_kernel(const bf16* __restrict_
 
 // C[m, n] = sum_k A(m, k) B[k, n] on the CUDA cores: A fp32 with element (m, k) at
 // A[m * a_sm + k * a_sk], B bf16 row-major [K, ldb], C fp32 [M, ldc]. A block computes a
-// 64 x 128 tile from 32-deep slices staged in shared memory; each thread owns 4 x 8
-// outputs (fixed summation order: k ascending).
-constexpr int kGm = 64, kGn = 128, kGk = 32, kGThreads = 256;
+// 128 x 128 tile from 16-deep slices staged in shared memory (B converted to fp32 there);
+// each thread owns 8 x 8 outputs, rows 4ty.. and 64 + 4ty.., columns 4tx.. and 64 + 4tx..,
+// read as float4 from shared memory (fixed summation order: k ascending).
+constexpr int kGm = 128, kGn = 128, kGk = 16, kGThreads = 256;
 
-__global__ void __launch_bounds__(kGThreads) gemm_f32_bf16_kernel(const GemmF32Args a) {
-  __shared__ float sA[kGk][kGm + 1];
-  __shared__ float sB[kGk][kGn + 4];
+__global__ void __launch_bounds__(kGThreads, 2) gemm_f32_bf16_kernel(const GemmF32Args a) {
+  __shared__ __align__(16) float sA[kGk][kGm];
+  __shared__ __align__(16) float sB[kGk][kGn];
   const int m0 = blockIdx.y * kGm, n0 = blockIdx.x * kGn;
-  const int tm = threadIdx.x >> 4, tn = threadIdx.x & 15;  // 16 x 16 threads
-  float acc[4][8];
+  // split z of the K range (split-K: each split writes its own partial C, summed later)
+  const int kc = a.splits > 1 ? ((a.K + a.splits - 1) / a.splits + kGk - 1) / kGk * kGk : a.K;
+  const int kz0 = blockIdx.z * kc, kz1 = min(a.K, kz0 + kc);
+  float* C = a.splits > 1 ? a.partial + static_cast<int64_t>(blockIdx.z) * a.M * a.ldc : a.C;
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;  // 16 x 16 threads
+  const bool m_fast = a.a_sm == 1;  // A's contiguous dimension
+  float acc[8][8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-  for (int k0 = 0; k0 < a.K; k0 += kGk) {
-    for (int idx = threadIdx.x; idx < kGm * kGk; idx += kGThreads) {
-      const int mm = idx / kGk, kk = idx % kGk;  // consecutive threads walk k (a_sk == 1 case)
+  for (int k0 = kz0; k0 < kz1; k0 += kGk) {
+    // consecutive threads walk A's contiguous dimension: m when a_sm == 1, else k
+#pragma unroll
+    for (int u = 0; u < kGm * kGk / kGThreads; ++u) {
+      const int idx = threadIdx.x + u * kGThreads;
+      const int mm = m_fast ? idx % kGm : idx / kGk, kk = m_fast ? idx / kGm : idx % kGk;
       const int m = m0 + mm, k = k0 + kk;
-      sA[kk][mm] = (m < a.M && k < a.K) ? a.A[static_cast<int64_t>(m) * a.a_sm + static_cast<int64_t>(k) * a.a_sk]
-                                        : 0.f;
+      sA[kk][mm] = (m < a.M && k < kz1) ? a.A[static_cast<int64_t>(m) * a.a_sm + static_cast<int64_t>(k) * a.a_sk]
+                                         : 0.f;
     }
-    for (int idx = threadIdx.x; idx < kGk * kGn; idx += kGThreads) {
+#pragma unroll
+    for (int u = 0; u < kGk * kGn / kGThreads; ++u) {
+      const int idx = threadIdx.x + u * kGThreads;
       const int kk = idx / kGn, nn = idx % kGn;
       const int k = k0 + kk, n = n0 + nn;
-      sB[kk][nn] = (k < a.K && n < a.N) ? __bfloat162float(a.B[static_cast<int64_t>(k) * a.ldb + n]) : 0.f;
+      sB[kk][nn] = (k < kz1 && n < a.N) ? __bfloat162float(a.B[static_cast<int64_t>(k) * a.ldb + n]) : 0.f;
     }
     __syncthreads();
-#pragma unroll 4
+#pragma unroll
     for (int kk = 0; kk < kGk; ++kk) {
-      float av[4], bv[8];
+      const float4 a0 = *reinterpret_cast<const float4*>(&sA[kk][4 * ty]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&sA[kk][64 + 4 * ty]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&sB[kk][4 * tx]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&sB[kk][64 + 4 * tx]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) av[i] = sA[kk][tm + 16 * i];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) bv[j] = sB[kk][tn + 16 * j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
     __syncthreads();
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int m = m0 + tm + 16 * i;
+  for (int i = 0; i < 8; ++i) {
+    const int m = m0 + (i < 4 ? 4 * ty + i : 64 + 4 * ty + i - 4);
     if (m >= a.M) continue;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const int n = n0 + tn + 16 * j;
-      if (n < a.N) a.C[static_cast<int64_t>(m) * a.ldc + n] = acc[i][j];
+      const int n = n0 + (j < 4 ? 4 * tx + j : 64 + 4 * tx + j - 4);
+      if (n < a.N) C[static_cast<int64_t>(m) * a.ldc + n] = acc[i][j];
     }
+  }
+}
+
+// C[m, n] = sum over z = 0.. in order of partial[z][m, n] (the split-K partial sums).
+__global__ void split_sum_kernel(const float* __restrict__ partial, int splits, int M, int N, int64_t ldc,
+                                 float* __restrict__ C) {
+  const int64_t total = static_cast<int64_t>(M) * N;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t m = i / N, n = i % N, o = m * ldc + n;
+    float v = 0.f;
+    for (int z = 0; z < splits; ++z) v += partial[z * static_cast<int64_t>(M) * ldc + o];
+    C[o] = v;
   }
 }
 }  // namespace
@@ -340,9 +365,16 @@ cudaError_t launch_dx_combine(const bf16* dh, const float* dXs, const float* dx_
 
 cudaError_t launch_gemm_f32_bf16(const GemmF32Args& a, cudaStream_t s) {
   if (a.M <= 0 || a.N <= 0) return cudaSuccess;
-  const dim3 grid((a.N + kGn - 1) / kGn, (a.M + kGm - 1) / kGm);
-  if (grid.y > 65535) return cudaErrorInvalidValue;
+  const int splits = a.splits > 1 ? a.splits : 1;
+  if (splits > 1 && !a.partial) return cudaErrorInvalidValue;
+  const dim3 grid((a.N + kGn - 1) / kGn, (a.M + kGm - 1) / kGm, splits);
+  if (grid.y > 65535 || splits > 64) return cudaErrorInvalidValue;
   gemm_f32_bf16_kernel<<<grid, kGThreads, 0, s>>>(a);
+  if (splits > 1) {
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    split_sum_kernel<<<1024, 256, 0, s>>>(a.partial, splits, a.M, a.N, a.ldc, a.C);
+  }
   return cudaGetLastError();
 }
 

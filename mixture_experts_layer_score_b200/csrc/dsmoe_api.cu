@@ -1335,20 +1335,11 @@ DSMOE_EXPORT dsmoe_status dsmoe_backward_router(dsmoe_handle* h, int32_t T, cons
   r.dlogits = dlogits;
   r.status = h->status;
   CUDA_TRY(dsmoe::launch_router_backward(r, h->num_sms, st));
-  // dx = dlogits W_router  (M = T, K = N', N = d)
   dsmoe::GemmF32Args a;
-  a.A = dlogits;
-  a.a_sm = N;
-  a.a_sk = 1;
-  a.B = static_cast<const bf16*>(W_router);
-  a.ldb = d;
-  a.C = dx;
-  a.ldc = d;
-  a.M = T;
-  a.N = d;
-  a.K = N;
-  CUDA_TRY(dsmoe::launch_gemm_f32_bf16(a, st));
-  // dW_router = dlogits^T x  (M = N', K = T, N = d)
+  memset(&a, 0, sizeof(a));
+  // dW_router = dlogits^T x  (M = N', K = T, N = d). Few output tiles and a long K: the K
+  // range is split so that about two blocks per SM work; the partial sums go to dx's
+  // memory (T x d >= splits x N' x d floats), which the next GEMM then overwrites.
   a.A = dlogits;
   a.a_sm = 1;
   a.a_sk = N;
@@ -1359,6 +1350,28 @@ DSMOE_EXPORT dsmoe_status dsmoe_backward_router(dsmoe_handle* h, int32_t T, cons
   a.M = N;
   a.N = d;
   a.K = T;
+  {
+    const int64_t tiles = static_cast<int64_t>(cdiv(N, 128)) * cdiv(d, 128);  // 128 x 128 output tiles
+    int64_t splits = (2 * h->num_sms + tiles - 1) / tiles;
+    splits = std::min<int64_t>(splits, std::min<int64_t>(32, T / 256));  // slices of >= 256 tokens
+    splits = std::min<int64_t>(splits, T / N);                           // partials fit in dx
+    a.splits = static_cast<int>(std::max<int64_t>(splits, 1));
+    a.partial = a.splits > 1 ? dx : nullptr;
+  }
+  CUDA_TRY(dsmoe::launch_gemm_f32_bf16(a, st));
+  // dx = dlogits W_router  (M = T, K = N', N = d)
+  memset(&a, 0, sizeof(a));
+  a.A = dlogits;
+  a.a_sm = N;
+  a.a_sk = 1;
+  a.B = static_cast<const bf16*>(W_router);
+  a.ldb = d;
+  a.C = dx;
+  a.ldc = d;
+  a.M = T;
+  a.N = d;
+  a.K = N;
+  a.splits = 1;
   CUDA_TRY(dsmoe::launch_gemm_f32_bf16(a, st));
   h->launches += 3;
   return DSMOE_OK;
@@ -1525,9 +1538,13 @@ DSMOE_EXPORT dsmoe_status dsmoe_backward_weights(dsmoe_handle* h, int32_t T, con
   const int Ks = h->add_shared ? c.n_shared : 0;
   if (!dh || !dY || !x || !dW_gate || !dW_up || !dW_down || (Ks && (!dWs_gate || !dWs_up || !dWs_down)))
     return fail(DSMOE_ERR_INVALID_ARG, "NULL argument");
-  const void* must_align[] = {dh, dY, x, dW_gate, dW_up, dW_down, dWs_gate, dWs_up, dWs_down};
+  const void* must_align[] = {dh, dY, x};
   for (const void* q : must_align)
     if (q && !aligned16(q)) return fail(DSMOE_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", q);
+  const void* must_align32[] = {dW_gate, dW_up, dW_down, dWs_gate, dWs_up, dWs_down};  // 32-byte row stores
+  for (const void* q : must_align32)
+    if (q && (reinterpret_cast<uintptr_t>(q) & 31u))
+      return fail(DSMOE_ERR_INVALID_ARG, "weight-gradient pointer %p is not 32-byte aligned", q);
   DeviceGuard gd(h->device);
   if (!gd.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -9,27 +9,42 @@
 // each routed expert's K range is its segment of the slot order (ragged), each shared
 // expert's all T tokens.
 //
-// One CTA per SM, 192 threads: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
-// warps 2-5 epilogue. A tile is 256 output rows (two M=128 chains) by 128 output columns;
+// One CTA per SM, 320 threads: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
+// warps 2-9 epilogue (each thread stores its own output row in 32-byte vectors). A tile is 256 output rows (two M=128 chains) by 128 output columns;
 // per 64-row K block the producer stages A (256 columns of the A buffer) and B (128
 // columns of the B buffer) through 3-D views (64, rows, cols / 64) that land as 64-element
 // MN-major swizzle-128B atoms 8 KB apart. A K block that runs past the group's last row
-// holds rows of the next group (or the buffer's zero fill): the MMA warp zeroes those rows
-// in shared memory (and makes the stores visible to the tensor core) before the MMAs. A
-// group with no rows gets a zero tile. Output fp32, D row-major per group.
+// holds rows of the next group (or the buffer's zero fill): only its 16-row MMA steps that
+// hold valid rows are issued, and the MMA warp zeroes the invalid rows of the last of them
+// in shared memory (making the stores visible to the tensor core) first. A group with no
+// rows gets a zero tile. Output fp32, D row-major per group.
 // Every wait is bounded; a role that gives up raises the abort flag and a status bit, the
 // CTA waits (at least one second) for its copies and MMAs in flight, frees TMEM, returns.
 #include "kernels.h"
+#include "role_clock.cuh"
 #include "sm100_ptx.cuh"
 
 namespace dsmoe {
 
+#ifdef DSMOE_ROLE_CYCLES
+__device__ unsigned long long g_role_cycles_dw[kRoleCtas][kRsSlots];
+#endif
+
 namespace {
+__device__ __forceinline__ void role_add_dw(int slot, long long v) {
+#ifdef DSMOE_ROLE_CYCLES
+  if (blockIdx.x < kRoleCtas) atomicAdd(&g_role_cycles_dw[blockIdx.x][slot], static_cast<unsigned long long>(v));
+#else
+  (void)slot;
+  (void)v;
+#endif
+}
+
 constexpr int kBK = 64;
 constexpr int kFeat = 128;
 constexpr int kMmaK = 16;
-constexpr int kThreads = 192;
-constexpr int kEpiThreads = 128;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kN = 128;                             // output columns per tile (the MMA's N)
 constexpr int kStages = 4;
@@ -38,15 +53,14 @@ constexpr uint32_t kBBytes = kN * kBK * 2;         // 16 KB: 128 output columns 
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kAccCols = 2 * kN;
 constexpr int kBufs = 2;
-constexpr uint32_t kStageRow = 33;
 constexpr uint32_t kAtom = kBK * 128;              // one 64-element atom column of a stage: 8 KB
 constexpr uint32_t kOffA = 0;
 constexpr uint32_t kOffB = kOffA + kStages * kABytes;
 constexpr uint32_t kOffBars = kOffB + kStages * kBBytes;
 constexpr uint32_t kNumBars = 2 * kStages + 2 * kBufs + 1;
 constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
-constexpr uint32_t kOffEpi = (kOffMisc + 16 + 15) & ~15u;
-constexpr uint32_t kSmemUsed = kOffEpi + 4 * 32 * kStageRow * 4;
+constexpr uint32_t kOffOffs = (kOffMisc + 16 + 15) & ~15u;  // the groups' row offsets
+constexpr uint32_t kSmemUsed = kOffOffs + (kGemmMaxGroups + 1) * 4;
 constexpr size_t kSmemBytes = kSmemUsed + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
@@ -73,7 +87,7 @@ struct DwTile {
   int group, shared, row0, rows, m_blk, n_blk;
 };
 
-__device__ __forceinline__ DwTile dw_decode(const GemmDwArgs& a, int tile) {
+__device__ __forceinline__ DwTile dw_decode(const GemmDwArgs& a, const int32_t* offs, int tile) {
   DwTile t;
   const int tiles_s = a.m_tiles_shared * a.n_tiles_shared, tiles_r = a.m_tiles_routed * a.n_tiles_routed;
   int local, n_tiles;
@@ -90,8 +104,8 @@ __device__ __forceinline__ DwTile dw_decode(const GemmDwArgs& a, int tile) {
     t.group = r / tiles_r;
     local = r - t.group * tiles_r;
     n_tiles = a.n_tiles_routed;
-    t.row0 = a.offsets[t.group];
-    t.rows = max(a.offsets[t.group + 1] - t.row0, 0);
+    t.row0 = offs[t.group];
+    t.rows = max(offs[t.group + 1] - t.row0, 0);
   }
   t.m_blk = local / n_tiles;
   t.n_blk = local % n_tiles;
@@ -99,6 +113,9 @@ __device__ __forceinline__ DwTile dw_decode(const GemmDwArgs& a, int tile) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_constant__ GemmDwArgs a) {
+  RoleClock rc_kernel;
+  rc_kernel.start();
+  const unsigned long long rc_ns0 = role_ns();
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_addr(smem_raw) & 1023u)) & 1023u;
   uint8_t* base = smem_raw + pad;
@@ -113,6 +130,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + kOffMisc + 4);
   volatile int* never_flag = reinterpret_cast<volatile int*>(base + kOffMisc + 8);
+  int32_t* offs = reinterpret_cast<int32_t*>(base + kOffOffs);
+  for (int i = threadIdx.x; i <= a.n_routed; i += blockDim.x) offs[i] = a.offsets[i];  // (barrier below)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total = a.n_shared * a.m_tiles_shared * a.n_tiles_shared +
@@ -126,7 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
     }
     for (int i = 0; i < kBufs; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], kEpiThreads);
+      mbar_init(&acc_empty[i], kEpiWarps);  // one lane of each epilogue warp
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -147,8 +166,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      RoleClock rc_wait;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-        const DwTile t = dw_decode(a, tile);
+        const DwTile t = dw_decode(a, offs, tile);
         const CUtensorMap* ta = t.shared ? &a.a_shared : &a.a_routed;
         const CUtensorMap* tb = t.shared ? &a.b_shared : &a.b_routed;
         const int a_atom = (t.shared ? a.a_atom0_shared + t.group * a.a_atom_step_shared : a.a_atom0_routed) +
@@ -157,10 +177,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
                            t.n_blk * (kN / 64);
         const int kb_n = (t.rows + kBK - 1) / kBK;
         for (int kb = 0; kb < kb_n; ++kb) {
+          rc_wait.start();
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, a.wait_limit_ns, abort_flag)) {
             ok = false;
             break;
           }
+          rc_wait.stop();
           mbar_arrive_expect_tx(&full[stage], kStageBytes);
           tma_load_3d_view(sA + stage * kABytes, ta, &full[stage], t.row0 + kb * kBK, a_atom);
           tma_load_3d_view(sB + stage * kBBytes, tb, &full[stage], t.row0 + kb * kBK, b_atom);
@@ -176,6 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
         *abort_flag = 1;
         atomicOr(a.status, kStatusTimeoutProducer);
       }
+      role_add_dw(kRsProducerWaitStage, rc_wait.total);
     }
   } else if (warp == 1) {
     // -------------------------------------------------------------------- MMA issuer
@@ -186,31 +209,40 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
     bool ok = true;
     int it = 0;
     const uint32_t idesc = idesc_bf16_f32(kFeat, kN) | (1u << 15) | (1u << 16);  // A and B MN-major
+    RoleClock rc_loop, rc_stage, rc_acc;
+    rc_loop.start();
     for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++it) {
-      const DwTile t = dw_decode(a, tile);
+      const DwTile t = dw_decode(a, offs, tile);
       const int kb_n = (t.rows + kBK - 1) / kBK;
       const int acc = it % kBufs;
+      rc_acc.start();
       if (!mbar_wait_warp(&acc_empty[acc], ((it / kBufs) & 1) ^ 1u, a.wait_limit_ns, abort_flag)) {
         ok = false;
         break;
       }
+      rc_acc.stop();
       tc_fence_after();
       const uint32_t d0 = tmem_base + acc * kAccCols;
       for (int kb = 0; kb < kb_n; ++kb) {
+        rc_stage.start();
         if (!mbar_wait_warp(&full[stage], phase, a.wait_limit_ns, abort_flag)) {
           ok = false;
           break;
         }
+        rc_stage.stop();
         tc_fence_after();
-        const int valid = t.rows - kb * kBK;  // rows of this K block inside the group
-        if (valid < kBK) {
-          // 6 atom columns (4 of A, 2 of B) x (64 - valid) rows of 128 B, 16 B per lane
-          const int bad = kBK - valid;
-          for (int i = lane; i < 6 * bad * 8; i += 32) {
-            const int col = i / (bad * 8), rem = i - col * bad * 8;
-            const int r = valid + rem / 8, q = rem % 8;
+        const int valid = t.rows - kb * kBK;  // rows of this K block inside the group (> 0)
+        // K steps of 16 rows that hold any of them; the rows of the last such step past the
+        // group's end (fewer than 16) are zeroed in both operands, 6 atom columns of 128 B
+        // rows (4 of A, 2 of B): lane l clears the 16-byte chunk l % 8 of rows r + l / 8
+        const int ksteps = valid >= kBK ? kBK / kMmaK : (valid + kMmaK - 1) / kMmaK;
+        const int z1 = ksteps * kMmaK;
+        if (valid < z1) {
+          const int q = lane & 7;
+          for (int col = 0; col < 6; ++col) {
             uint8_t* atom = col < 4 ? sA + stage * kABytes + col * kAtom : sB + stage * kBBytes + (col - 4) * kAtom;
-            *reinterpret_cast<uint4*>(atom + r * 128 + q * 16) = make_uint4(0u, 0u, 0u, 0u);  // row r: 128 B
+            for (int r = valid + (lane >> 3); r < z1; r += 4)
+              *reinterpret_cast<uint4*>(atom + r * 128 + q * 16) = make_uint4(0u, 0u, 0u, 0u);
           }
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           __syncwarp();
@@ -219,6 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
           const uint32_t abase = smem_addr(sA + stage * kABytes), bbase = smem_addr(sB + stage * kBBytes);
 #pragma unroll
           for (int k = 0; k < kBK / kMmaK; ++k) {
+            if (k >= ksteps) break;
             const uint32_t accum = (kb | k) ? 1u : 0u;
             const uint32_t koff = static_cast<uint32_t>(k) * kMmaK * 128;
             const uint64_t bd = desc_mn_sw128(bbase + koff);
@@ -241,15 +274,29 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
       *abort_flag = 1;
       atomicOr(a.status, kStatusTimeoutMma);
     }
+    rc_loop.stop();
+    if (lane == 0) {
+      role_add_dw(kRsMmaWaitStage, rc_stage.total);
+      role_add_dw(kRsMmaWaitAcc, rc_acc.total);
+      role_add_dw(kRsMmaLoop, rc_loop.total);
+      role_add_dw(kRsTiles, it);
+    }
   } else {
     // -------------------------------------------------------------------- epilogue
-    const int q = warp & 3;
-    float* stg = reinterpret_cast<float*>(base + kOffEpi) + q * 32 * kStageRow;
-    const int rr = lane >> 2, cc = (lane & 3) * 8;
+    // Warp w reads TMEM lanes [32q, 32q+32), q = w % 4: thread l of lane l holds output row
+    // 32q + l of each chain, 32 consecutive fp32 columns per chunk, and stores them as four
+    // 32-byte vectors along its own row (no transpose: the row is the output's contiguous
+    // dimension). Warps 2+q and 6+q take alternate chunks of the tile's 2 x kN/32; the next
+    // chunk's TMEM reads are issued before this chunk's stores.
+    const int q = warp & 3, half = (warp - 2) >> 2;
+    constexpr int kChunks = 2 * (kN / 32);
     int it = 0;
+    RoleClock rc_loop, rc_acc;
+    rc_loop.start();
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
-      const DwTile t = dw_decode(a, tile);
+      const DwTile t = dw_decode(a, offs, tile);
       const int acc = it % kBufs;
+      rc_acc.start();
       if (!mbar_wait_warp_sleepy(&acc_full[acc], (it / kBufs) & 1, a.wait_limit_ns, abort_flag)) {
         if (lane == 0) {
           *abort_flag = 1;
@@ -257,42 +304,48 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
         }
         break;
       }
+      rc_acc.stop();
       tc_fence_after();
       const bool empty_group = t.rows == 0;
       const int M = t.shared ? a.m_shared : a.m_routed, N = t.shared ? a.n_shared_cols : a.n_routed_cols;
       float* out = (t.shared ? a.out_shared : a.out_routed) + static_cast<int64_t>(t.group) * M * N;
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
+      uint32_t v[32];
+      auto load = [&](int idx) {
+        const uint32_t col = static_cast<uint32_t>((idx / (kN / 32)) * kN + (idx % (kN / 32)) * 32);
+        tmem_ld16(tb + col, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+        tmem_ld16(tb + col + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
+      };
+      load(half);
+      tmem_wait_ld();
 #pragma unroll 1
-      for (int ch = 0; ch < 2; ++ch) {
-#pragma unroll 1
-        for (int c0 = 0; c0 < kN; c0 += 32) {
-          uint32_t v[32];
-          tmem_ld16(tb + ch * kN + c0, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
-          tmem_ld16(tb + ch * kN + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
-          tmem_wait_ld();
+      for (int idx = half; idx < kChunks; idx += 2) {
+        float r[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) stg[j * kStageRow + lane] = empty_group ? 0.f : __uint_as_float(v[j]);
-          __syncwarp();
-          // lane L writes 8 consecutive columns c0 + cc.. of output row m_base + L/4 + 8i
-          const int m_base = t.m_blk * 2 * kFeat + ch * kFeat + q * 32;
-          const int n = t.n_blk * kN + c0 + cc;
+        for (int j = 0; j < 32; ++j) r[j] = empty_group ? 0.f : __uint_as_float(v[j]);
+        if (idx + 2 < kChunks) load(idx + 2);  // lands while this chunk is stored
+        const int ch = idx / (kN / 32);
+        const int row = t.m_blk * 2 * kFeat + ch * kFeat + q * 32 + lane;
+        const int n = t.n_blk * kN + (idx % (kN / 32)) * 32;  // N is a multiple of 64: all or none
+        if (row < M && n < N) {
+          float* dst = out + static_cast<int64_t>(row) * N + n;  // 32-byte aligned (host-checked base)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int row = rr + 8 * i;
-            if (m_base + row < M && n < N) {
-              float vals[8];
-#pragma unroll
-              for (int k = 0; k < 8; ++k) vals[k] = stg[(cc + k) * kStageRow + row];
-              float4* dst = reinterpret_cast<float4*>(out + static_cast<int64_t>(m_base + row) * N + n);
-              dst[0] = make_float4(vals[0], vals[1], vals[2], vals[3]);
-              dst[1] = make_float4(vals[4], vals[5], vals[6], vals[7]);
-            }
-          }
-          __syncwarp();
+          for (int s8 = 0; s8 < 4; ++s8)
+            asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + 8 * s8),
+                         "f"(r[8 * s8]), "f"(r[8 * s8 + 1]), "f"(r[8 * s8 + 2]), "f"(r[8 * s8 + 3]),
+                         "f"(r[8 * s8 + 4]), "f"(r[8 * s8 + 5]), "f"(r[8 * s8 + 6]), "f"(r[8 * s8 + 7])
+                         : "memory");
         }
+        tmem_wait_ld();
       }
       tc_fence_before();
-      mbar_arrive(&acc_empty[acc]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+    }
+    rc_loop.stop();
+    if (warp == 2 && lane == 0) {
+      role_add_dw(kRsEpiWaitAcc, rc_acc.total);
+      role_add_dw(kRsEpiLoop, rc_loop.total);
     }
   }
 
@@ -316,10 +369,29 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
+  if (threadIdx.x == 0) {
+    rc_kernel.stop();
+    role_add_dw(kRsCycles, rc_kernel.total);
+    role_add_dw(kRsNanoseconds, static_cast<long long>(role_ns() - rc_ns0));
+  }
 }
 }  // namespace
 
+bool read_role_cycles_dw(unsigned long long* host, cudaError_t* err) {
+#ifdef DSMOE_ROLE_CYCLES
+  static unsigned long long zeros[kRoleCtas * kRsSlots];
+  *err = cudaMemcpyFromSymbol(host, g_role_cycles_dw, sizeof(zeros));
+  if (*err == cudaSuccess) *err = cudaMemcpyToSymbol(g_role_cycles_dw, zeros, sizeof(zeros));
+  return true;
+#else
+  (void)host;
+  *err = cudaSuccess;
+  return false;
+#endif
+}
+
 cudaError_t launch_grouped_dw(const GemmDwArgs& a, int num_sms, cudaStream_t s) {
+  if (a.n_routed > kGemmMaxGroups) return cudaErrorInvalidValue;
   const int64_t total = static_cast<int64_t>(a.n_shared) * a.m_tiles_shared * a.n_tiles_shared +
                         static_cast<int64_t>(a.n_routed) * a.m_tiles_routed * a.n_tiles_routed;
   if (total <= 0) return cudaSuccess;

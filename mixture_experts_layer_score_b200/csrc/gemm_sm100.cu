@@ -50,7 +50,7 @@
 namespace dsmoe {
 
 #ifdef DSMOE_ROLE_CYCLES
-__device__ unsigned long long g_role_cycles[kRoleKernels][kRoleCtas][kRsSlots];
+__device__ unsigned long long g_role_cycles[kRoleKindDw][kRoleCtas][kRsSlots];
 #endif
 
 namespace {
@@ -461,8 +461,9 @@ cudaError_t launch_one(const GemmArgs& a, int grid, cudaStream_t s) {
 bool read_role_cycles(unsigned long long* host, cudaError_t* err) {
 #ifdef DSMOE_ROLE_CYCLES
   static unsigned long long zeros[kRoleCounters];
-  *err = cudaMemcpyFromSymbol(host, g_role_cycles, sizeof(zeros));
-  if (*err == cudaSuccess) *err = cudaMemcpyToSymbol(g_role_cycles, zeros, sizeof(zeros));
+  *err = cudaMemcpyFromSymbol(host, g_role_cycles, sizeof(g_role_cycles));
+  if (*err == cudaSuccess) *err = cudaMemcpyToSymbol(g_role_cycles, zeros, sizeof(g_role_cycles));
+  if (*err == cudaSuccess) read_role_cycles_dw(host + kRoleKindDw * kRoleCtas * kRsSlots, err);
   return true;
 #else
   (void)host;

@@ -179,6 +179,10 @@ struct GemmF32Args {
   float* C;
   int64_t ldc;
   int M, N, K;
+  // split-K (splits > 1): the K range is cut into `splits` slices whose partial products go
+  // to partial[splits][M][ldc] and are then summed in slice order into C (deterministic)
+  int splits;
+  float* partial;
 };
 cudaError_t launch_gemm_f32_bf16(const GemmF32Args& a, cudaStream_t s);
 
@@ -232,6 +236,8 @@ cudaError_t launch_grouped_gemm(bool swiglu, int tok, const GemmArgs& a, int gri
 // Profiling builds (DSMOE_ROLE_CYCLES, role_clock.cuh): copy the one-CTA grouped GEMM's role
 // counters to host[kRoleCounters] and clear them; false in any other build.
 bool read_role_cycles(unsigned long long* host, cudaError_t* err);
+// The weight-gradient GEMM's counters (one row set, kRoleCtas x kRsSlots), cleared likewise.
+bool read_role_cycles_dw(unsigned long long* host, cudaError_t* err);
 
 // The experts' backward GEMMs (gemm_bwd_sm100.cu). kBwdDM: da | db from dy and W_down;
 // kBwdDX: dx rows from da | db and W_gate, W_up. The weight maps b0 / b1 of `g` are 4-D

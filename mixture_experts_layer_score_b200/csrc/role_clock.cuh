@@ -1,4 +1,4 @@
-// role_clock.cuh -- per-CTA cycle counters of the one-CTA grouped GEMM's roles (profiling).
+// role_clock.cuh -- per-CTA cycle counters of the grouped GEMMs' roles (profiling).
 //
 // In a build with DSMOE_ROLE_CYCLES defined (build.py --role-cycles writes it to its own
 // library file), every CTA of the one-CTA grouped GEMM adds to its row of counters, per
@@ -28,8 +28,10 @@ enum RoleSlot : int {
   kRsSlots
 };
 constexpr int kRoleCtas = 160;   // counter rows: CTAs with blockIdx.x < kRoleCtas
-// launches: 0 down, 1 gate/up (with routed groups); 2 down, 3 gate/up (shared experts only)
-constexpr int kRoleKernels = 4;
+// launches: 0 down, 1 gate/up (with routed groups); 2 down, 3 gate/up (shared experts
+// only) of the one-CTA grouped GEMM; 4 the weight-gradient GEMM (gemm_dw_sm100.cu)
+constexpr int kRoleKernels = 5;
+constexpr int kRoleKindDw = 4;
 constexpr int kRoleCounters = kRoleKernels * kRoleCtas * kRsSlots;
 
 #ifdef DSMOE_ROLE_CYCLES
