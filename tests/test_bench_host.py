@@ -36,7 +36,7 @@ def test_captured_traffic_prefers_the_benchmarked_workload(tmp_path, monkeypatch
         "gemm_gate_up 0000000000000000 999 1 big_case stale\n")
     csrc = tmp_path / "mixture_experts_layer_score_b200" / "csrc"
     csrc.mkdir(parents=True)
-    for name in ("gemm_sm100.cu", "grouped_tiles.cuh"):
+    for name in ("gemm_sm100.cu", "grouped_tiles.cuh", "gemm_gateup_pair_sm100.cu"):
         (csrc / name).write_bytes(open(os.path.join(ROOT, bench.CSRC, name), "rb").read())
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert abs(bench.captured_traffic("gemm_gate_up", 400.0, "single", "big_case") - 440.0) < 1e-9  # 220/200
