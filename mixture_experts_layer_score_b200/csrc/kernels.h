@@ -189,15 +189,16 @@ cudaError_t launch_gemm_f32_bf16(const GemmF32Args& a, cudaStream_t s);
 // ---------------------------------------------------------------- grouped GEMM (gemm_sm100.cu)
 constexpr int kGemmMaxGroups = 8 + 512;  // shared + routed groups of one grouped GEMM
 // Tokens per grouped-GEMM tile (the row box of the token-side tensor maps): 128, or 256
-// for the gate/up projection of layers with a long K loop and a few hundred rows per
-// expert, where the larger N moves fewer shared-memory bytes per MAC and the one
-// accumulator it leaves (the next tile waits for this tile's epilogue) costs less than
-// that saves (measured on the V3 shapes: d = 7168, about 256 rows per expert).
+// for the gate/up projection of layers with a K loop of at least 20 blocks of 64 and a
+// few hundred rows per expert, where the larger N moves fewer shared-memory bytes per MAC
+// and the one accumulator it leaves (the next tile waits for this tile's epilogue) costs
+// less than that saves (measured: V3, d = 7168, gate/up -5%; the 2B-shaped layer,
+// d = 1280, -3.5%; the GShard shapes, d = 1024, +2-5%, so they keep 128).
 constexpr int kGemmTokenTile = 128;
 constexpr int kGemmTokenTileLarge = 256;
 // rows, groups: the token rows and the groups (routed and shared) of the launch
 inline int gateup_token_tile(int d_model, int64_t rows, int groups) {
-  return (d_model >= 4096 && groups > 0 && rows >= 192LL * groups) ? kGemmTokenTileLarge : kGemmTokenTile;
+  return (d_model >= 1280 && groups > 0 && rows >= 192LL * groups) ? kGemmTokenTileLarge : kGemmTokenTile;
 }
 struct GemmArgs {
   CUtensorMap a_routed;   // 2D [rows, K] activations of routed slots, box (64, token tile)
