@@ -60,6 +60,9 @@ def parse_args():
     ap.add_argument("--decode", default="v4_decode_t256,v4_decode_t16",
                     help="decode workloads timed after the main one at N=1 (comma list; empty: none)")
     ap.add_argument("--decode-steps", type=int, default=20)
+    ap.add_argument("--graph", action="store_true",
+                    help="N=1: capture one forward in a CUDA graph after the warm-up and time its replays "
+                         "(the device work is the same; host launch overhead leaves the timed region)")
     ap.add_argument("--backward", action="store_true",
                     help="time a training step instead (forward saving the pre-activations, gate, router, "
                          "expert input and weight gradients) and print one JSON line of stage times and rates")
@@ -342,6 +345,24 @@ def run_native(args, cfg):
     # ---- timed region (device)
     M.dsmoe_set_timing(layer.handle, True)
     launches0 = M.dsmoe_launch_count(layer.handle)
+    graph = None
+    if args.graph and world == 1:
+        # one untimed forward on the capture stream, then the capture with the stage events
+        # (timing on): every replay records them again, into the one recorded slot
+        M.dsmoe_set_timing(layer.handle, False)
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            layer.forward(inp["x"], token_ids=inp["token_ids"], out=out, stream=cap)
+        stream.wait_stream(cap)
+        M.dsmoe_set_timing(layer.handle, True)
+        l0 = M.dsmoe_launch_count(layer.handle)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            layer.forward(inp["x"], token_ids=inp["token_ids"], out=out)
+        per_forward = M.dsmoe_launch_count(layer.handle) - l0
+        launches0 = M.dsmoe_launch_count(layer.handle)
+        step = graph.replay  # noqa: F811
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
@@ -359,6 +380,8 @@ def run_native(args, cfg):
     ms = e0.elapsed_time(e1)
     clock_info = clocks.stop()
     launches = M.dsmoe_launch_count(layer.handle) - launches0
+    if graph is not None:
+        launches = per_forward * args.steps  # replays launch the captured kernels
     stage_ms = M.dsmoe_stage_times(layer.handle)
     M.dsmoe_set_timing(layer.handle, False)
     if world > 1:
@@ -485,7 +508,9 @@ def run_native(args, cfg):
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; random weights of the layer's shape)",
-                "config": dict(config_block(cfg, world), gemm_kernel=args.gemm), "roofline": roof,
+                "config": dict(config_block(cfg, world), gemm_kernel=args.gemm,
+                               launch="cuda graph replay" if graph is not None else "stream launches"),
+                "roofline": roof,
                 "cpu_baseline": cpu_base, "e2e": e2e, "gpu_launches": int(launches), "clocks": clock_info,
                 "layer_tflops": layer_tflops, "stage_ms": stage_ms, "experts_touched": touched, "decode": decode}
         print(json.dumps(line), flush=True)

@@ -817,8 +817,12 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
   const int e0 = h->e_begin, NL = h->e_end - h->e_begin;  // routed experts applied here
   const bool timing = h->timing && T > 0;
   cudaEvent_t* evs = h->ev[h->timed_forwards % kTimingSlots];
+  // under stream capture the stage events become graph nodes that record on every replay
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (timing) CUDA_TRY(cudaStreamIsCapturing(s, &cap));
+  const unsigned rec_flags = cap == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
   const std::function<cudaError_t(int)> mark = [&](int i) -> cudaError_t {
-    return timing ? cudaEventRecord(evs[i], s) : cudaSuccess;
+    return timing ? cudaEventRecordWithFlags(evs[i], s, rec_flags) : cudaSuccess;
   };
 
   if (T == 0) return zero_stats(a, N, s);
@@ -852,7 +856,7 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
   if (Ks > 0) {
     // shared experts (gate/up into A1s, down into Hs with the residual), queued after the
     // router so that its CTAs are placed first; the permute's CTAs fit beside these GEMMs'
-    if (timing) CUDA_TRY(cudaEventRecord(evs[kChainStages + 1], h->side));
+    if (timing) CUDA_TRY(cudaEventRecordWithFlags(evs[kChainStages + 1], h->side, rec_flags));
     GemmPlan sp = p;
     sp.rows = a.x;
     sp.rows_extent = static_cast<uint64_t>(T);
@@ -861,7 +865,7 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
     sp.Ks = Ks;
     sp.Y_out = nullptr;
     STAGE_TRY(gemm_stage(h, sp, h->side, no_mark));
-    if (timing) CUDA_TRY(cudaEventRecord(evs[kChainStages + 2], h->side));
+    if (timing) CUDA_TRY(cudaEventRecordWithFlags(evs[kChainStages + 2], h->side, rec_flags));
     CUDA_TRY(cudaEventRecord(h->ev_join, h->side));
   }
   CUDA_TRY(mark(2));
@@ -882,8 +886,8 @@ dsmoe_status run_forward(dsmoe_handle* h, const FwdArgs& a, cudaStream_t s) {
   STAGE_TRY(combine_stage(h, a, h->Y, Ks, h->add_shared, h->partial, s));
   CUDA_TRY(mark(7));
   if (timing && Ks == 0) {  // no shared-expert stage: an empty interval
-    CUDA_TRY(cudaEventRecord(evs[kChainStages + 1], s));
-    CUDA_TRY(cudaEventRecord(evs[kChainStages + 2], s));
+    CUDA_TRY(cudaEventRecordWithFlags(evs[kChainStages + 1], s, rec_flags));
+    CUDA_TRY(cudaEventRecordWithFlags(evs[kChainStages + 2], s, rec_flags));
   }
   if (timing) h->timed_forwards += 1;
   return DSMOE_OK;

@@ -158,6 +158,43 @@ def test_repeatable_bitwise():
     layer.close()
 
 
+@pytest.mark.parametrize("name,T", [("ds2b", 700), ("gshard_b", 512)])
+def test_forward_captured_in_a_cuda_graph(name, T):
+    """The forward has no host synchronisation and no allocation, so it can be captured
+    into a CUDA graph, side stream included (the shared experts' GEMMs fork from and join
+    the capturing stream through events). A replay gives the eager forward's outputs bit
+    for bit, and after new values are copied into the captured input buffer, a replay gives
+    the eager forward of those values."""
+    cfg = W.get_config(name).replace(T=T)
+    gpu, _ = make_case(cfg, T)
+    layer = M.DSMoE(M.cfg_from(cfg, T), gpu)
+    x = gpu["x"].clone()
+    x2 = W.normal_bf16((T, cfg.d_model), 1.0, 0, "x_graph", 1, "cuda")
+    ref = {k: v.clone() for k, v in layer.forward(x).items() if v is not None}
+    ref2 = {k: v.clone() for k, v in layer.forward(x2).items() if v is not None}
+    out = layer.alloc_outputs(T)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # warm the capture stream
+        layer.forward(x, out=out)
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer.forward(x, out=out)
+    g.replay()
+    torch.cuda.synchronize()
+    assert M.dsmoe_get_status(layer.handle) == M.DSMOE_OK
+    for k in ("h", "topk_idx", "gates", "counts", "f", "P"):
+        assert torch.equal(out[k], ref[k]), k
+    x.copy_(x2)
+    g.replay()
+    torch.cuda.synchronize()
+    for k in ("h", "topk_idx", "gates", "counts", "f", "P"):
+        assert torch.equal(out[k], ref2[k]), k
+    del g
+    layer.close()
+
+
 def test_host_entry_point_matches_device_entry_point():
     cfg = W.get_config("tiny")
     gpu, _ = make_case(cfg, cfg.T)
