@@ -382,7 +382,10 @@ dsmoe_status dsmoe_ep_combine(dsmoe_handle* h, int32_t T, const void* x, const v
  *                               sigma(l) / (2 s) uses sigma(l) = 1 - exp(-s^2))
  *     dx      fp32 [T, d] out   dlogits W_router (the router's part of dL/du)
  *     dW_router fp32 [N', d] out dlogits^T x
- *   All sums run in a fixed order (deterministic).
+ *   Both products run on the CUDA cores in fp32. dW_router (few outputs, K = T) is split
+ *   over T into slices whose partial sums are held in dx's memory until they are added,
+ *   before dx itself is computed; dx must not alias another argument. All sums run in a
+ *   fixed order (deterministic).
  */
 dsmoe_status dsmoe_backward_gates(dsmoe_handle* h, int32_t T, const void* dh, const float* gates, float* dg,
                                   void* dY, void* stream);
