@@ -17,8 +17,9 @@
 //        (K = 2F, K-major). Routed rows are written as bf16 per slot; the shared experts
 //        form one group whose K loop runs over every shared expert's da | db and whose
 //        fp32 rows sum all of them.
-// Both: one CTA per SM, 192 threads (warp 0 TMA producer, warp 1 TMEM owner and MMA
-// issuer, warps 2-5 epilogue), tiles of 256 M rows (two M=128 chains) by at most 128
+// Both: one CTA per SM, 320 threads (warp 0 TMA producer, warp 1 TMEM owner and MMA
+// issuer, warps 2-9 epilogue: warps 2+q and 6+q read TMEM lanes [32q, 32q+32) for
+// alternate 32-token chunks), tiles of 256 M rows (two M=128 chains) by at most 128
 // tokens, a 4-stage ring of 48 KB, two TMEM accumulators of 2 x 128 columns. The A
 // operand of a stage (256 M rows x 64 K rows) arrives in one TMA copy through a 4-D view
 // (64 M, K, M / 64, experts) of the weights, which lands as four 64-row MN-major
@@ -34,8 +35,8 @@ namespace {
 constexpr int kBK = 64;
 constexpr int kFeat = 128;
 constexpr int kMmaK = 16;
-constexpr int kThreads = 192;
-constexpr int kEpiThreads = 128;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kTok = 128;
 constexpr int kStages = 4;
@@ -53,7 +54,8 @@ constexpr uint32_t kNumBars = 2 * kStages + 2 * kBufs + 1;
 constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
 constexpr uint32_t kOffTiles = kOffMisc + 16;
 constexpr uint32_t kOffEpi = (kOffTiles + (kGemmMaxGroups + 1) * 4 + 15) & ~15u;
-constexpr uint32_t kSmemUsed = kOffEpi + 4 * 32 * kStageRow * 4;
+constexpr uint32_t kStgFloats = 16 * kStageRow;  // per epilogue warp: 16 token rows of 32 (+1) floats
+constexpr uint32_t kSmemUsed = kOffEpi + kEpiWarps * kStgFloats * 4;
 constexpr size_t kSmemBytes = kSmemUsed + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
@@ -110,7 +112,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bwd_kernel(const __g
     }
     for (int i = 0; i < kBufs; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], kEpiThreads);
+      mbar_init(&acc_empty[i], kEpiWarps);  // one lane of each epilogue warp
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -227,10 +229,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bwd_kernel(const __g
   } else {
     // -------------------------------------------------------------------- epilogue
     // Thread f of TMEM lane f holds M row f of both chains. Per 32 tokens the warp
-    // transposes its 32 rows x 32 tokens through shared memory, then lane L handles 8
-    // consecutive M rows of token row L/4 + 8i (16-byte vectors).
-    const int q = warp & 3;
-    float* stg = reinterpret_cast<float*>(base + kOffEpi) + q * 32 * kStageRow;
+    // transposes its 32 rows x 32 tokens through shared memory in two 16-token halves,
+    // then lane L handles 8 consecutive M rows of token row L/4 + 8i (16-byte vectors).
+    const int q = warp & 3, half = (warp - 2) >> 2;
+    float* stg = reinterpret_cast<float*>(base + kOffEpi) + (warp - 2) * kStgFloats;
     const int rr = lane >> 2, cc = (lane & 3) * 8;
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
@@ -247,63 +249,68 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bwd_kernel(const __g
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
       const int n_valid = t.shared ? g.n_valid_shared : g.n_valid_routed;
 #pragma unroll 1
-      for (int c0 = 0; c0 < t.m_valid; c0 += 32) {
+      for (int c0 = 32 * half; c0 < t.m_valid; c0 += 64) {
         uint32_t v0[32], v1[32];
         tmem_ld16(tb + c0, *reinterpret_cast<uint32_t(*)[16]>(&v0[0]));
         tmem_ld16(tb + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v0[16]));
         tmem_ld16(tb + kChainCols + c0, *reinterpret_cast<uint32_t(*)[16]>(&v1[0]));
         tmem_ld16(tb + kChainCols + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v1[16]));
         tmem_wait_ld();
-#pragma unroll 1
-        for (int ch = 0; ch < 2; ++ch) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) stg[j * kStageRow + lane] = __uint_as_float(ch == 0 ? v0[j] : v1[j]);
-          __syncwarp();
+        for (int ch = 0; ch < 2; ++ch) {
           const int f = t.n_blk * 2 * kFeat + ch * kFeat + q * 32 + cc;  // first of this lane's 8 M rows
           const bool ok_f = f < n_valid;  // n_valid is a multiple of 64, f of 8
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int row = rr + 8 * i;
-            if (!ok_f || c0 + row >= t.m_valid) continue;
-            const float* src = stg + row * kStageRow + cc;
-            const int64_t r = t.row0 + c0 + row;
-            if (kMode == kBwdDM) {
-              // saved pre-activations a | b of this row, and the da | db outputs, side by side
-              const int64_t ld = t.shared ? a.ld_ab_shared : a.ld_ab_routed;
-              const int64_t col = t.shared ? static_cast<int64_t>(t.group) * 2 * a.width_shared + f : f;
-              const int64_t half = t.shared ? a.width_shared : a.width_routed;
-              const bf16* ab = t.shared ? a.ab_shared : a.ab_routed;
-              bf16* dab = t.shared ? a.dab_shared : a.dab_routed;
-              const uint4 av = *reinterpret_cast<const uint4*>(ab + r * ld + col);
-              const uint4 bv = *reinterpret_cast<const uint4*>(ab + r * ld + col + half);
-              const uint32_t aw[4] = {av.x, av.y, av.z, av.w}, bw[4] = {bv.x, bv.y, bv.z, bv.w};
-              uint32_t da[4], db[4];
+          for (int hh = 0; hh < 2; ++hh) {
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const float2 x = unpack_bf16x2(aw[k]), y = unpack_bf16x2(bw[k]);
-                const float s0 = __fdividef(1.0f, 1.0f + __expf(-x.x)), s1 = __fdividef(1.0f, 1.0f + __expf(-x.y));
-                const float dm0 = src[2 * k], dm1 = src[2 * k + 1];
-                da[k] = pack_bf16x2(dm0 * y.x * s0 * (1.0f + x.x * (1.0f - s0)),
-                                    dm1 * y.y * s1 * (1.0f + x.y * (1.0f - s1)));
-                db[k] = pack_bf16x2(dm0 * x.x * s0, dm1 * x.y * s1);
+            for (int j = 0; j < 16; ++j)
+              stg[j * kStageRow + lane] = __uint_as_float(ch == 0 ? v0[16 * hh + j] : v1[16 * hh + j]);
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int row = rr + 8 * i, tok = c0 + 16 * hh + row;
+              if (!ok_f || tok >= t.m_valid) continue;
+              const float* src = stg + row * kStageRow + cc;
+              const int64_t r = t.row0 + tok;
+              if (kMode == kBwdDM) {
+                // saved pre-activations a | b of this row, and the da | db outputs, side by side
+                const int64_t ld = t.shared ? a.ld_ab_shared : a.ld_ab_routed;
+                const int64_t col = t.shared ? static_cast<int64_t>(t.group) * 2 * a.width_shared + f : f;
+                const int64_t wh = t.shared ? a.width_shared : a.width_routed;
+                const bf16* ab = t.shared ? a.ab_shared : a.ab_routed;
+                bf16* dab = t.shared ? a.dab_shared : a.dab_routed;
+                const uint4 av = *reinterpret_cast<const uint4*>(ab + r * ld + col);
+                const uint4 bv = *reinterpret_cast<const uint4*>(ab + r * ld + col + wh);
+                const uint32_t aw[4] = {av.x, av.y, av.z, av.w}, bw[4] = {bv.x, bv.y, bv.z, bv.w};
+                uint32_t da[4], db[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const float2 x = unpack_bf16x2(aw[k]), y = unpack_bf16x2(bw[k]);
+                  const float s0 = __fdividef(1.0f, 1.0f + __expf(-x.x)), s1 = __fdividef(1.0f, 1.0f + __expf(-x.y));
+                  const float dm0 = src[2 * k], dm1 = src[2 * k + 1];
+                  da[k] = pack_bf16x2(dm0 * y.x * s0 * (1.0f + x.x * (1.0f - s0)),
+                                      dm1 * y.y * s1 * (1.0f + x.y * (1.0f - s1)));
+                  db[k] = pack_bf16x2(dm0 * x.x * s0, dm1 * x.y * s1);
+                }
+                *reinterpret_cast<uint4*>(dab + r * ld + col) = make_uint4(da[0], da[1], da[2], da[3]);
+                *reinterpret_cast<uint4*>(dab + r * ld + col + wh) = make_uint4(db[0], db[1], db[2], db[3]);
+              } else if (t.shared) {  // fp32 sum over the shared experts, one row per token
+                float4* dst = reinterpret_cast<float4*>(a.dx_shared + r * a.ld_dx + f);
+                dst[0] = make_float4(src[0], src[1], src[2], src[3]);
+                dst[1] = make_float4(src[4], src[5], src[6], src[7]);
+              } else {
+                *reinterpret_cast<uint4*>(a.dx_routed + r * a.ld_dx + f) =
+                    make_uint4(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
+                               pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
               }
-              *reinterpret_cast<uint4*>(dab + r * ld + col) = make_uint4(da[0], da[1], da[2], da[3]);
-              *reinterpret_cast<uint4*>(dab + r * ld + col + half) = make_uint4(db[0], db[1], db[2], db[3]);
-            } else if (t.shared) {  // fp32 sum over the shared experts, one row per token
-              float4* dst = reinterpret_cast<float4*>(a.dx_shared + r * a.ld_dx + f);
-              dst[0] = make_float4(src[0], src[1], src[2], src[3]);
-              dst[1] = make_float4(src[4], src[5], src[6], src[7]);
-            } else {
-              *reinterpret_cast<uint4*>(a.dx_routed + r * a.ld_dx + f) =
-                  make_uint4(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
-                             pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
             }
+            __syncwarp();
           }
-          __syncwarp();
         }
       }
       tc_fence_before();
-      mbar_arrive(&acc_empty[acc]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
     }
   }
 
