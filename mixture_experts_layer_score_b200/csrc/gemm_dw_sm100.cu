@@ -16,8 +16,8 @@
 // MN-major swizzle-128B atoms 8 KB apart. A K block that runs past the group's last row
 // holds rows of the next group (or the buffer's zero fill): only its 16-row MMA steps that
 // hold valid rows are issued, and the MMA warp zeroes the invalid rows of the last of them
-// in shared memory (making the stores visible to the tensor core) first. A group with no
-// rows gets a zero tile. Output fp32, D row-major per group.
+// in the B operand's shared memory (making the stores visible to the tensor core) first.
+// A group with no rows gets a zero tile. Output fp32, D row-major per group.
 // Every wait is bounded; a role that gives up raises the abort flag and a status bit, the
 // CTA waits (at least one second) for its copies and MMAs in flight, frees TMEM, returns.
 #include "kernels.h"
@@ -233,14 +233,16 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
         tc_fence_after();
         const int valid = t.rows - kb * kBK;  // rows of this K block inside the group (> 0)
         // K steps of 16 rows that hold any of them; the rows of the last such step past the
-        // group's end (fewer than 16) are zeroed in both operands, 6 atom columns of 128 B
-        // rows (4 of A, 2 of B): lane l clears the 16-byte chunk l % 8 of rows r + l / 8
+        // group's end (fewer than 16) are zeroed in the B operand, whose 2 atom columns of
+        // 128-byte rows cancel those rows' products (A's rows there are finite: the next
+        // group's data or the copy's zero fill): lane l clears the 16-byte chunk l % 8 of
+        // rows r + l / 8
         const int ksteps = valid >= kBK ? kBK / kMmaK : (valid + kMmaK - 1) / kMmaK;
         const int z1 = ksteps * kMmaK;
         if (valid < z1) {
           const int q = lane & 7;
-          for (int col = 0; col < 6; ++col) {
-            uint8_t* atom = col < 4 ? sA + stage * kABytes + col * kAtom : sB + stage * kBBytes + (col - 4) * kAtom;
+          for (int col = 0; col < 2; ++col) {
+            uint8_t* atom = sB + stage * kBBytes + col * kAtom;
             for (int r = valid + (lane >> 3); r < z1; r += 4)
               *reinterpret_cast<uint4*>(atom + r * 128 + q * 16) = make_uint4(0u, 0u, 0u, 0u);
           }
