@@ -23,7 +23,11 @@
  *   - No entry point allocates device memory except dsmoe_create, and no
  *     entry point synchronises the device except where it says so. Work is
  *     enqueued on the caller's stream (a cudaStream_t passed as void*; NULL is
- *     the legacy default stream).
+ *     the legacy default stream); a forward with shared experts also runs their
+ *     GEMMs on the handle's own side stream, forked from the caller's stream at the
+ *     start of the call and joined back into it before the call's last kernel, so
+ *     the caller's stream still orders everything (a CUDA graph capture of the call
+ *     captures both).
  *   - Errors are returned, never raised: no exit, abort or trap. A kernel that
  *     gives up a bounded wait records DSMOE_ERR_DEVICE_TIMEOUT in a device
  *     status word that dsmoe_get_status() reports.
