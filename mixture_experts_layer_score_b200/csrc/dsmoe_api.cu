@@ -128,6 +128,20 @@ bool map_view_mn(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3D fp32 map (cols, rows, groups) of a [groups, rows, cols] tensor, 128-byte swizzle,
+// box (32, 32, 1): the weight-gradient GEMM's bulk stores of 32 x 32 chunks.
+bool map_out_f32(CUtensorMap* m, float* ptr, uint64_t rows, uint64_t cols, uint64_t groups) {
+  auto enc = tensor_map_encoder();
+  if (!enc || cols % 32 || rows % 32 || groups == 0) return false;
+  cuuint64_t dims[3] = {cols, rows, groups};
+  cuuint64_t strides[2] = {cols * 4, rows * cols * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct DeviceGuard {
   int prev = -1, want;
   bool ok = false;
@@ -1542,13 +1556,9 @@ DSMOE_EXPORT dsmoe_status dsmoe_backward_weights(dsmoe_handle* h, int32_t T, con
   const int Ks = h->add_shared ? c.n_shared : 0;
   if (!dh || !dY || !x || !dW_gate || !dW_up || !dW_down || (Ks && (!dWs_gate || !dWs_up || !dWs_down)))
     return fail(DSMOE_ERR_INVALID_ARG, "NULL argument");
-  const void* must_align[] = {dh, dY, x};
+  const void* must_align[] = {dh, dY, x, dW_gate, dW_up, dW_down, dWs_gate, dWs_up, dWs_down};
   for (const void* q : must_align)
     if (q && !aligned16(q)) return fail(DSMOE_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", q);
-  const void* must_align32[] = {dW_gate, dW_up, dW_down, dWs_gate, dWs_up, dWs_down};  // 32-byte row stores
-  for (const void* q : must_align32)
-    if (q && (reinterpret_cast<uintptr_t>(q) & 31u))
-      return fail(DSMOE_ERR_INVALID_ARG, "weight-gradient pointer %p is not 32-byte aligned", q);
   DeviceGuard gd(h->device);
   if (!gd.ok) return fail(DSMOE_ERR_CUDA, "cannot select device %d", h->device);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -1581,6 +1591,12 @@ DSMOE_EXPORT dsmoe_status dsmoe_backward_weights(dsmoe_handle* h, int32_t T, con
     g.status = h->status;
     g.wait_limit_ns = h->wait_ns;
   };
+  // outputs: routed [NL, M, N], shared [Ks, Ms, Ns]
+  auto outputs = [&](dsmoe::GemmDwArgs& g, float* routed, float* shared) {
+    bool m_ok = NL == 0 || map_out_f32(&g.out_map_routed, routed, g.m_routed, g.n_routed_cols, NL);
+    if (Ks) m_ok = m_ok && map_out_f32(&g.out_map_shared, shared, g.m_shared, g.n_shared_cols, Ks);
+    return m_ok;
+  };
   // dW_down[e] = sum_r dy_r m_r^T: A = dY (d columns), B = A1 (F columns)
   dsmoe::GemmDwArgs g;
   plan(g, d, F, d, Fs);
@@ -1589,8 +1605,8 @@ DSMOE_EXPORT dsmoe_status dsmoe_backward_weights(dsmoe_handle* h, int32_t T, con
   g.a_shared = Ks ? v_dh : v_dY;
   g.b_shared = Ks ? v_A1s : v_A1;
   g.b_atom_step_shared = Fs / 64;
-  g.out_routed = dW_down;
-  g.out_shared = dWs_down;
+  if (!outputs(g, dW_down, dWs_down))
+    return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a weight-gradient output map");
   CUDA_TRY(dsmoe::launch_grouped_dw(g, h->num_sms, s));
   // dW_gate[e] = sum_r da_r u_r^T and dW_up[e] = sum_r db_r u_r^T: A = da | db, B = Xp (x)
   for (int up = 0; up < 2; ++up) {
@@ -1602,8 +1618,8 @@ DSMOE_EXPORT dsmoe_status dsmoe_backward_weights(dsmoe_handle* h, int32_t T, con
     g.a_atom0_routed = up ? F / 64 : 0;
     g.a_atom0_shared = up ? Fs / 64 : 0;
     g.a_atom_step_shared = 2 * Fs / 64;
-    g.out_routed = up ? dW_up : dW_gate;
-    g.out_shared = up ? dWs_up : dWs_gate;
+    if (!outputs(g, up ? dW_up : dW_gate, up ? dWs_up : dWs_gate))
+      return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a weight-gradient output map");
     CUDA_TRY(dsmoe::launch_grouped_dw(g, h->num_sms, s));
   }
   h->launches += 3;

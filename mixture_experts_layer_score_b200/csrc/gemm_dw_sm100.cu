@@ -10,7 +10,9 @@
 // expert's all T tokens.
 //
 // One CTA per SM, 320 threads: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
-// warps 2-9 epilogue (each thread stores its own output row in 32-byte vectors). A tile is 256 output rows (two M=128 chains) by 128 output columns;
+// warps 2-9 epilogue (each stages 32 x 32 fp32 chunks of the accumulator in its own 4 KB of
+// shared memory and writes them to the output with bulk tensor stores, whole 128-byte
+// lines). A tile is 256 output rows (two M=128 chains) by 128 output columns;
 // per 64-row K block the producer stages A (256 columns of the A buffer) and B (128
 // columns of the B buffer) through 3-D views (64, rows, cols / 64) that land as 64-element
 // MN-major swizzle-128B atoms 8 KB apart. A K block that runs past the group's last row
@@ -56,11 +58,12 @@ constexpr int kBufs = 2;
 constexpr uint32_t kAtom = kBK * 128;              // one 64-element atom column of a stage: 8 KB
 constexpr uint32_t kOffA = 0;
 constexpr uint32_t kOffB = kOffA + kStages * kABytes;
-constexpr uint32_t kOffBars = kOffB + kStages * kBBytes;
+constexpr uint32_t kStgBytes = 32 * 32 * 4;        // one warp's staged 32 x 32 fp32 chunk
+constexpr uint32_t kOffStg = kOffB + kStages * kBBytes;
+constexpr uint32_t kOffBars = kOffStg + kEpiWarps * kStgBytes;
 constexpr uint32_t kNumBars = 2 * kStages + 2 * kBufs + 1;
 constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
-constexpr uint32_t kOffOffs = (kOffMisc + 16 + 15) & ~15u;  // the groups' row offsets
-constexpr uint32_t kSmemUsed = kOffOffs + (kGemmMaxGroups + 1) * 4;
+constexpr uint32_t kSmemUsed = kOffMisc + 16;
 constexpr size_t kSmemBytes = kSmemUsed + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
@@ -83,11 +86,25 @@ __device__ __forceinline__ void tma_load_3d_view(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// Bulk tensor store of one staged chunk: box (32 fp32 columns, 32 rows, 1 group) of a 3-D
+// map (columns, rows, groups) with the 128-byte swizzle; rows past a group's end are not
+// written (the map's row extent is the group's).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int32_t col, int32_t row,
+                                             int32_t group) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(col), "r"(row), "r"(group)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 struct DwTile {
   int group, shared, row0, rows, m_blk, n_blk;
 };
 
-__device__ __forceinline__ DwTile dw_decode(const GemmDwArgs& a, const int32_t* offs, int tile) {
+__device__ __forceinline__ DwTile dw_decode(const GemmDwArgs& a, int tile) {
   DwTile t;
   const int tiles_s = a.m_tiles_shared * a.n_tiles_shared, tiles_r = a.m_tiles_routed * a.n_tiles_routed;
   int local, n_tiles;
@@ -104,8 +121,8 @@ __device__ __forceinline__ DwTile dw_decode(const GemmDwArgs& a, const int32_t* 
     t.group = r / tiles_r;
     local = r - t.group * tiles_r;
     n_tiles = a.n_tiles_routed;
-    t.row0 = offs[t.group];
-    t.rows = max(offs[t.group + 1] - t.row0, 0);
+    t.row0 = __ldg(a.offsets + t.group);
+    t.rows = max(__ldg(a.offsets + t.group + 1) - t.row0, 0);
   }
   t.m_blk = local / n_tiles;
   t.n_blk = local % n_tiles;
@@ -130,8 +147,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + kOffMisc + 4);
   volatile int* never_flag = reinterpret_cast<volatile int*>(base + kOffMisc + 8);
-  int32_t* offs = reinterpret_cast<int32_t*>(base + kOffOffs);
-  for (int i = threadIdx.x; i <= a.n_routed; i += blockDim.x) offs[i] = a.offsets[i];  // (barrier below)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total = a.n_shared * a.m_tiles_shared * a.n_tiles_shared +
@@ -168,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
       bool ok = true;
       RoleClock rc_wait;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-        const DwTile t = dw_decode(a, offs, tile);
+        const DwTile t = dw_decode(a, tile);
         const CUtensorMap* ta = t.shared ? &a.a_shared : &a.a_routed;
         const CUtensorMap* tb = t.shared ? &a.b_shared : &a.b_routed;
         const int a_atom = (t.shared ? a.a_atom0_shared + t.group * a.a_atom_step_shared : a.a_atom0_routed) +
@@ -212,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
     RoleClock rc_loop, rc_stage, rc_acc;
     rc_loop.start();
     for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++it) {
-      const DwTile t = dw_decode(a, offs, tile);
+      const DwTile t = dw_decode(a, tile);
       const int kb_n = (t.rows + kBK - 1) / kBK;
       const int acc = it % kBufs;
       rc_acc.start();
@@ -286,17 +301,20 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
   } else {
     // -------------------------------------------------------------------- epilogue
     // Warp w reads TMEM lanes [32q, 32q+32), q = w % 4: thread l of lane l holds output row
-    // 32q + l of each chain, 32 consecutive fp32 columns per chunk, and stores them as four
-    // 32-byte vectors along its own row (no transpose: the row is the output's contiguous
-    // dimension). Warps 2+q and 6+q take alternate chunks of the tile's 2 x kN/32; the next
-    // chunk's TMEM reads are issued before this chunk's stores.
+    // 32q + l of each chain, 32 consecutive fp32 columns per chunk. It writes that 128-byte
+    // row into the warp's staging buffer with the 128-byte swizzle (16-byte unit c of row r
+    // at unit c ^ (r % 8): a quarter-warp's stores hit all 32 banks once) and lane 0 stores
+    // the 32 x 32 chunk with one bulk tensor copy. Warps 2+q and 6+q take alternate chunks of
+    // the tile's 2 x kN/32; the next chunk's TMEM reads are issued before this chunk is
+    // staged, and the buffer is rewritten only after the previous copy has read it.
     const int q = warp & 3, half = (warp - 2) >> 2;
     constexpr int kChunks = 2 * (kN / 32);
+    const uint32_t stg = smem_addr(base + kOffStg + (warp - 2) * kStgBytes);
     int it = 0;
     RoleClock rc_loop, rc_acc;
     rc_loop.start();
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
-      const DwTile t = dw_decode(a, offs, tile);
+      const DwTile t = dw_decode(a, tile);
       const int acc = it % kBufs;
       rc_acc.start();
       if (!mbar_wait_warp_sleepy(&acc_full[acc], (it / kBufs) & 1, a.wait_limit_ns, abort_flag)) {
@@ -310,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
       tc_fence_after();
       const bool empty_group = t.rows == 0;
       const int M = t.shared ? a.m_shared : a.m_routed, N = t.shared ? a.n_shared_cols : a.n_routed_cols;
-      float* out = (t.shared ? a.out_shared : a.out_routed) + static_cast<int64_t>(t.group) * M * N;
+      const CUtensorMap* omap = t.shared ? &a.out_map_shared : &a.out_map_routed;
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
       uint32_t v[32];
       auto load = [&](int idx) {
@@ -322,21 +340,27 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
       tmem_wait_ld();
 #pragma unroll 1
       for (int idx = half; idx < kChunks; idx += 2) {
-        float r[32];
+        uint32_t r[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) r[j] = empty_group ? 0.f : __uint_as_float(v[j]);
+        for (int j = 0; j < 32; ++j) r[j] = empty_group ? 0u : v[j];
         if (idx + 2 < kChunks) load(idx + 2);  // lands while this chunk is stored
         const int ch = idx / (kN / 32);
-        const int row = t.m_blk * 2 * kFeat + ch * kFeat + q * 32 + lane;
-        const int n = t.n_blk * kN + (idx % (kN / 32)) * 32;  // N is a multiple of 64: all or none
-        if (row < M && n < N) {
-          float* dst = out + static_cast<int64_t>(row) * N + n;  // 32-byte aligned (host-checked base)
+        const int row0 = t.m_blk * 2 * kFeat + ch * kFeat + q * 32;  // M and N are multiples of 64:
+        const int n = t.n_blk * kN + (idx % (kN / 32)) * 32;         // a chunk is all inside or all out
+        if (row0 < M && n < N) {
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
 #pragma unroll
-          for (int s8 = 0; s8 < 4; ++s8)
-            asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + 8 * s8),
-                         "f"(r[8 * s8]), "f"(r[8 * s8 + 1]), "f"(r[8 * s8 + 2]), "f"(r[8 * s8 + 3]),
-                         "f"(r[8 * s8 + 4]), "f"(r[8 * s8 + 5]), "f"(r[8 * s8 + 6]), "f"(r[8 * s8 + 7])
+          for (int c = 0; c < 8; ++c)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg + lane * 128 + ((c ^ (lane & 7)) << 4)),
+                         "r"(r[4 * c]), "r"(r[4 * c + 1]), "r"(r[4 * c + 2]), "r"(r[4 * c + 3])
                          : "memory");
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(omap, stg, n, row0, t.group);
+            bulk_commit();
+          }
         }
         tmem_wait_ld();
       }
@@ -344,6 +368,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
     }
+    if (lane == 0) bulk_wait_all();  // the CTA's shared memory outlives every copy from it
+    __syncwarp();
     rc_loop.stop();
     if (warp == 2 && lane == 0) {
       role_add_dw(kRsEpiWaitAcc, rc_acc.total);

@@ -272,8 +272,9 @@ struct GemmDwArgs {
   int32_t n_routed, n_shared, T;
   int32_t m_tiles_routed, n_tiles_routed, m_tiles_shared, n_tiles_shared;  // 256-row x 128-col tiles
   int32_t m_routed, n_routed_cols, m_shared, n_shared_cols;                // output [M, N] per group
-  float* out_routed;       // [n_routed, m_routed, n_routed_cols] fp32
-  float* out_shared;       // [n_shared, m_shared, n_shared_cols] fp32
+  // fp32 outputs [groups, M, N] as 3-D maps (N, M, groups), box (32, 32, 1), 128-byte
+  // swizzle: routed [n_routed, m_routed, n_routed_cols], shared [n_shared, m_shared, n_shared_cols]
+  CUtensorMap out_map_routed, out_map_shared;
   uint32_t* status;
   uint64_t wait_limit_ns;
 };
