@@ -386,10 +386,16 @@ dsmoe_status dsmoe_ep_combine(dsmoe_handle* h, int32_t T, const void* x, const v
  *                               sigma(l) / (2 s) uses sigma(l) = 1 - exp(-s^2))
  *     dx      fp32 [T, d] out   dlogits W_router (the router's part of dL/du)
  *     dW_router fp32 [N', d] out dlogits^T x
- *   Both products run on the CUDA cores in fp32. dW_router (few outputs, K = T) is split
- *   over T into slices whose partial sums are held in dx's memory until they are added,
- *   before dx itself is computed; dx must not alias another argument. All sums run in a
- *   fixed order (deterministic).
+ *   With N' a multiple of 64, d a multiple of 64, T >= 256, T >= 2 N' and all pointers
+ *   16-byte aligned, both products run on the tensor cores: dlogits is split into bf16
+ *   parts hi + lo (what remains is below 2^-16 of each value; the [hi | lo] rows overwrite
+ *   the handle's "logits" workspace, which only the forward reads), dW_router = hi^T x +
+ *   lo^T x on the weight-gradient GEMM (the two fp32 results held in dx's memory until
+ *   they are added, hi first) and dx = [hi | lo] [W_router; W_router] on the input-
+ *   gradient GEMM. Otherwise both run on the CUDA cores in fp32, dW_router (few outputs,
+ *   K = T) split over T into slices whose partial sums are held in dx's memory until
+ *   they are added, before dx itself is computed. dx must not alias another argument.
+ *   All sums run in a fixed order (deterministic).
  */
 dsmoe_status dsmoe_backward_gates(dsmoe_handle* h, int32_t T, const void* dh, const float* gates, float* dg,
                                   void* dY, void* stream);

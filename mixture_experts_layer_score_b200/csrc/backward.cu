@@ -321,7 +321,45 @@ __global__ void split_sum_kernel(const float* __restrict__ partial, int splits, 
     C[o] = v;
   }
 }
+// dl = hi + lo with hi = bf16(dl) and lo = bf16(dl - hi) (what remains is below 2^-16 of
+// |dl|), written as rows [hi | lo] of 2N bf16: the router's backward contractions then run
+// on the tensor cores as bf16 products summed in fp32. Four consecutive values per thread.
+__global__ void hilo_split_kernel(const float* __restrict__ src, bf16* __restrict__ dst, int T, int N) {
+  const int64_t quads = static_cast<int64_t>(T) * N / 4;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < quads;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t e = 4 * i, t = e / N;
+    const int j = static_cast<int>(e - t * N);
+    const float4 v = *reinterpret_cast<const float4*>(src + e);
+    const float x[4] = {v.x, v.y, v.z, v.w};
+    __align__(8) bf16 hi[4], lo[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      hi[k] = __float2bfloat16_rn(x[k]);
+      lo[k] = __float2bfloat16_rn(x[k] - __bfloat162float(hi[k]));
+    }
+    bf16* row = dst + t * 2 * N;
+    *reinterpret_cast<uint2*>(row + j) = *reinterpret_cast<const uint2*>(hi);
+    *reinterpret_cast<uint2*>(row + N + j) = *reinterpret_cast<const uint2*>(lo);
+  }
+}
 }  // namespace
+
+cudaError_t launch_hilo_split(const float* src, bf16* dst, int T, int N, int num_sms, cudaStream_t s) {
+  if (N % 4) return cudaErrorInvalidValue;
+  const int64_t quads = static_cast<int64_t>(T) * N / 4;
+  if (quads <= 0) return cudaSuccess;
+  int64_t grid = (quads + 255) / 256;
+  if (grid > 8 * num_sms) grid = 8 * num_sms;
+  hilo_split_kernel<<<static_cast<int>(grid), 256, 0, s>>>(src, dst, T, N);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_split_sum(const float* partial, int splits, int M, int N, int64_t ldc, float* C, cudaStream_t s) {
+  if (M <= 0 || N <= 0) return cudaSuccess;
+  split_sum_kernel<<<1024, 256, 0, s>>>(partial, splits, M, N, ldc, C);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_gate_grad(const GateGradArgs& a, int num_sms, cudaStream_t s) {
   int grid = a.T;

@@ -1353,6 +1353,68 @@ DSMOE_EXPORT dsmoe_status dsmoe_backward_router(dsmoe_handle* h, int32_t T, cons
   r.dlogits = dlogits;
   r.status = h->status;
   CUDA_TRY(dsmoe::launch_router_backward(r, h->num_sms, st));
+  // The two contractions on the tensor cores where the shapes allow: dlogits split into
+  // bf16 parts hi + lo (what remains is below 2^-16 of each value), every product exact in
+  // the fp32 accumulation. [hi | lo] goes to the router-logits workspace, which the
+  // forward alone uses.
+  const size_t hilo_bytes = static_cast<size_t>(T) * N * 4;
+  const bool on_tensor_cores = N % 64 == 0 && d % 64 == 0 && T >= kTcRouterMinTokens && T >= 2 * N &&
+                               hilo_bytes <= h->L.counts_ws - h->L.logits && aligned16(dlogits) && aligned16(x) &&
+                               aligned16(W_router) && aligned16(dx) && aligned16(dW_router);
+  if (on_tensor_cores) {
+    bf16* hilo = reinterpret_cast<bf16*>(h->logits);
+    CUDA_TRY(dsmoe::launch_hilo_split(dlogits, hilo, T, N, h->num_sms, st));
+    // dW_router = hi^T x + lo^T x: the weight-gradient GEMM over all T rows with the two
+    // parts as two groups; their fp32 results go to dx's memory (T x d >= 2 x N' x d
+    // floats), which the dx GEMM overwrites afterwards, and are added in that order
+    dsmoe::GemmDwArgs w;
+    memset(&w, 0, sizeof(w));
+    CUtensorMap m_hilo, m_w;
+    bool ok = map_view_mn(&w.a_shared, hilo, T, 2 * static_cast<uint64_t>(N), 4) &&
+              map_view_mn(&w.b_shared, x, T, d, 2) && map_out_f32(&w.out_map_shared, dx, N, d, 2) &&
+              map_2d(&m_hilo, hilo, 2 * static_cast<uint64_t>(N), T, 128) && map_4d_mn(&m_w, W_router, N, d, 1);
+    if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map of the router backward");
+    w.a_routed = w.a_shared;
+    w.b_routed = w.b_shared;
+    w.a_atom_step_shared = N / 64;
+    w.offsets = h->offsets;
+    w.n_routed = 0;
+    w.n_shared = 2;
+    w.T = T;
+    w.m_tiles_shared = cdiv(N, 256);
+    w.n_tiles_shared = cdiv(d, 128);
+    w.m_shared = N;
+    w.n_shared_cols = d;
+    w.status = h->status;
+    w.wait_limit_ns = h->wait_ns;
+    CUDA_TRY(dsmoe::launch_grouped_dw(w, h->num_sms, st));
+    CUDA_TRY(dsmoe::launch_split_sum(dx, 2, N, d, d, dW_router, st));
+    // dx = dl W_router: the input-gradient GEMM (weights read MN-major) with W_router as
+    // both halves of one dense group's K loop over [hi | lo], fp32 rows
+    dsmoe::GemmBwdArgs b;
+    memset(&b, 0, sizeof(b));
+    dsmoe::GemmArgs& g = b.g;
+    g.a_routed = g.a_shared = m_hilo;
+    g.b0_routed = g.b1_routed = g.b0_shared = g.b1_shared = m_w;
+    g.offsets = h->offsets;
+    g.n_routed = 0;
+    g.n_shared_groups = 1;
+    g.m_shared = T;
+    g.n_tiles_routed = cdiv(d, 256);
+    g.n_tiles_shared = cdiv(d, 256);
+    g.kb_routed = g.kb_shared = 2 * N / 64;
+    g.n_valid_routed = g.n_valid_shared = d;
+    g.status = h->status;
+    g.wait_limit_ns = h->wait_ns;
+    b.kb_half_routed = b.kb_half_shared = N / 64;
+    b.dx_shared = dx;
+    b.ld_dx = d;
+    const int64_t tiles = cdiv(T, 128) * static_cast<int64_t>(g.n_tiles_shared);
+    CUDA_TRY(dsmoe::launch_grouped_gemm_bwd(dsmoe::kBwdDX, b, static_cast<int>(std::min<int64_t>(tiles, h->num_sms)),
+                                            st));
+    h->launches += 5;
+    return DSMOE_OK;
+  }
   dsmoe::GemmF32Args a;
   memset(&a, 0, sizeof(a));
   // dW_router = dlogits^T x  (M = N', K = T, N = d). Few output tiles and a long K: the K

@@ -185,6 +185,11 @@ struct GemmF32Args {
   float* partial;
 };
 cudaError_t launch_gemm_f32_bf16(const GemmF32Args& a, cudaStream_t s);
+// dst [T, 2N] bf16 = rows [hi | lo] of src [T, N] fp32 (hi = bf16(v), lo = bf16(v - hi));
+// N a multiple of 4, src 16-byte and dst 8-byte aligned.
+cudaError_t launch_hilo_split(const float* src, bf16* dst, int T, int N, int num_sms, cudaStream_t s);
+// C[m, n] = sum over z = 0 .. splits-1, in order, of partial[z][m, n] ([splits, M, ldc] floats).
+cudaError_t launch_split_sum(const float* partial, int splits, int M, int N, int64_t ldc, float* C, cudaStream_t s);
 
 // ---------------------------------------------------------------- grouped GEMM (gemm_sm100.cu)
 constexpr int kGemmMaxGroups = 8 + 512;  // shared + routed groups of one grouped GEMM
