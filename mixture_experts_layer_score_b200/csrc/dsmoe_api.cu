@@ -1370,8 +1370,8 @@ DSMOE_EXPORT dsmoe_status dsmoe_backward_router(dsmoe_handle* h, int32_t T, cons
     dsmoe::GemmDwArgs w;
     memset(&w, 0, sizeof(w));
     CUtensorMap m_hilo, m_w;
-    bool ok = map_view_mn(&w.a_shared, hilo, T, 2 * static_cast<uint64_t>(N), 4) &&
-              map_view_mn(&w.b_shared, x, T, d, 2) && map_out_f32(&w.out_map_shared, dx, N, d, 2) &&
+    bool ok = map_view_mn(&w.a_shared, hilo, T, 2 * static_cast<uint64_t>(N), 2) &&
+              map_view_mn(&w.b_shared, x, T, d, 4) && map_out_f32(&w.out_map_shared, dx, N, d, 2) &&
               map_2d(&m_hilo, hilo, 2 * static_cast<uint64_t>(N), T, 128) && map_4d_mn(&m_w, W_router, N, d, 1);
     if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map of the router backward");
     w.a_routed = w.a_shared;
@@ -1381,8 +1381,8 @@ DSMOE_EXPORT dsmoe_status dsmoe_backward_router(dsmoe_handle* h, int32_t T, cons
     w.n_routed = 0;
     w.n_shared = 2;
     w.T = T;
-    w.m_tiles_shared = cdiv(N, 256);
-    w.n_tiles_shared = cdiv(d, 128);
+    w.m_tiles_shared = cdiv(N, 128);
+    w.n_tiles_shared = cdiv(d, 256);
     w.m_shared = N;
     w.n_shared_cols = d;
     w.status = h->status;
@@ -1630,11 +1630,11 @@ DSMOE_EXPORT dsmoe_status dsmoe_backward_weights(dsmoe_handle* h, int32_t T, con
   // copies read zeros past them), shared rows = the T tokens
   const uint64_t S = static_cast<uint64_t>(T) * h->k_active, KsFs = static_cast<uint64_t>(Ks) * Fs;
   CUtensorMap v_dY, v_A1, v_dAB, v_Xp, v_dh, v_A1s, v_dABs, v_x;
-  bool ok = map_view_mn(&v_dY, dY, S, d, 4) && map_view_mn(&v_A1, h->A1, S, F, 2) &&
-            map_view_mn(&v_dAB, h->dAB, S, 2 * static_cast<uint64_t>(F), 4) && map_view_mn(&v_Xp, h->Xp, S, d, 2);
+  bool ok = map_view_mn(&v_dY, dY, S, d, 2) && map_view_mn(&v_A1, h->A1, S, F, 4) &&
+            map_view_mn(&v_dAB, h->dAB, S, 2 * static_cast<uint64_t>(F), 2) && map_view_mn(&v_Xp, h->Xp, S, d, 4);
   if (Ks)
-    ok = ok && map_view_mn(&v_dh, dh, T, d, 4) && map_view_mn(&v_A1s, h->A1s, T, KsFs, 2) &&
-         map_view_mn(&v_dABs, h->dABs, T, 2 * KsFs, 4) && map_view_mn(&v_x, x, T, d, 2);
+    ok = ok && map_view_mn(&v_dh, dh, T, d, 2) && map_view_mn(&v_A1s, h->A1s, T, KsFs, 4) &&
+         map_view_mn(&v_dABs, h->dABs, T, 2 * KsFs, 2) && map_view_mn(&v_x, x, T, d, 4);
   if (!ok) return fail(DSMOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map of the weight gradients");
   auto plan = [&](dsmoe::GemmDwArgs& g, int M, int N, int Ms, int Ns) {
     memset(&g, 0, sizeof(g));
@@ -1646,10 +1646,10 @@ DSMOE_EXPORT dsmoe_status dsmoe_backward_weights(dsmoe_handle* h, int32_t T, con
     g.n_routed_cols = N;
     g.m_shared = Ms;
     g.n_shared_cols = Ns;
-    g.m_tiles_routed = cdiv(M, 256);
-    g.n_tiles_routed = cdiv(N, 128);
-    g.m_tiles_shared = Ks ? cdiv(Ms, 256) : 0;
-    g.n_tiles_shared = Ks ? cdiv(Ns, 128) : 0;
+    g.m_tiles_routed = cdiv(M, 128);
+    g.n_tiles_routed = cdiv(N, 256);
+    g.m_tiles_shared = Ks ? cdiv(Ms, 128) : 0;
+    g.n_tiles_shared = Ks ? cdiv(Ns, 256) : 0;
     g.status = h->status;
     g.wait_limit_ns = h->wait_ns;
   };

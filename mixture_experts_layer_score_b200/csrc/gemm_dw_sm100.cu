@@ -12,13 +12,15 @@
 // One CTA per SM, 320 threads: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
 // warps 2-9 epilogue (each stages 32 x 32 fp32 chunks of the accumulator in its own 4 KB of
 // shared memory and writes them to the output with bulk tensor stores, whole 128-byte
-// lines). A tile is 256 output rows (two M=128 chains) by 128 output columns;
-// per 64-row K block the producer stages A (256 columns of the A buffer) and B (128
-// columns of the B buffer) through 3-D views (64, rows, cols / 64) that land as 64-element
-// MN-major swizzle-128B atoms 8 KB apart. A K block that runs past the group's last row
-// holds rows of the next group (or the buffer's zero fill): only its 16-row MMA steps that
-// hold valid rows are issued, and the MMA warp zeroes the invalid rows of the last of them
-// in the B operand's shared memory (making the stores visible to the tensor core) first.
+// lines). A tile is 128 output rows by 256 output columns, one M=128, N=256 chain (per
+// MAC it reads a quarter fewer shared-memory bytes than two M=128, N=128 chains, whose
+// operand reads alone fill the shared memory's bandwidth); per 64-row K block the
+// producer stages A (128 columns of the A buffer) and B (256 columns of the B buffer)
+// through 3-D views (64, rows, cols / 64) that land as 64-element MN-major swizzle-128B
+// atoms 8 KB apart. A K block that runs past the group's last row holds rows of the next
+// group (or the buffer's zero fill): only its 16-row MMA steps that hold valid rows are
+// issued, and the MMA warp zeroes the invalid rows of the last of them in the A
+// operand's shared memory (making the stores visible to the tensor core) first.
 // A group with no rows gets a zero tile. Output fp32, D row-major per group.
 // Every wait is bounded; a role that gives up raises the abort flag and a status bit, the
 // CTA waits (at least one second) for its copies and MMAs in flight, frees TMEM, returns.
@@ -43,17 +45,17 @@ __device__ __forceinline__ void role_add_dw(int slot, long long v) {
 }
 
 constexpr int kBK = 64;
-constexpr int kFeat = 128;
+constexpr int kFeat = 128;                          // output rows per tile (the MMA's M)
 constexpr int kMmaK = 16;
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kN = 128;                             // output columns per tile (the MMA's N)
+constexpr int kN = 256;                             // output columns per tile (the MMA's N)
 constexpr int kStages = 4;
-constexpr uint32_t kABytes = 2 * kFeat * kBK * 2;  // 32 KB: 256 output rows x 64 K rows
-constexpr uint32_t kBBytes = kN * kBK * 2;         // 16 KB: 128 output columns x 64 K rows
+constexpr uint32_t kABytes = kFeat * kBK * 2;      // 16 KB: 128 output rows x 64 K rows
+constexpr uint32_t kBBytes = kN * kBK * 2;         // 32 KB: 256 output columns x 64 K rows
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
-constexpr uint32_t kAccCols = 2 * kN;
+constexpr uint32_t kAccCols = kN;
 constexpr int kBufs = 2;
 constexpr uint32_t kAtom = kBK * 128;              // one 64-element atom column of a stage: 8 KB
 constexpr uint32_t kOffA = 0;
@@ -187,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
         const CUtensorMap* ta = t.shared ? &a.a_shared : &a.a_routed;
         const CUtensorMap* tb = t.shared ? &a.b_shared : &a.b_routed;
         const int a_atom = (t.shared ? a.a_atom0_shared + t.group * a.a_atom_step_shared : a.a_atom0_routed) +
-                           t.m_blk * (2 * kFeat / 64);
+                           t.m_blk * (kFeat / 64);
         const int b_atom = (t.shared ? a.b_atom0_shared + t.group * a.b_atom_step_shared : a.b_atom0_routed) +
                            t.n_blk * (kN / 64);
         const int kb_n = (t.rows + kBK - 1) / kBK;
@@ -218,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
   } else if (warp == 1) {
     // -------------------------------------------------------------------- MMA issuer
     // The whole warp follows the loop: on a K block that runs past the group's rows it
-    // zeroes those rows of both operands first; lane 0 issues the MMAs.
+    // zeroes those rows of the A operand first; lane 0 issues the MMAs.
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
@@ -248,8 +250,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
         tc_fence_after();
         const int valid = t.rows - kb * kBK;  // rows of this K block inside the group (> 0)
         // K steps of 16 rows that hold any of them; the rows of the last such step past the
-        // group's end (fewer than 16) are zeroed in the B operand, whose 2 atom columns of
-        // 128-byte rows cancel those rows' products (A's rows there are finite: the next
+        // group's end (fewer than 16) are zeroed in the A operand, whose 2 atom columns of
+        // 128-byte rows cancel those rows' products (B's rows there are finite: the next
         // group's data or the copy's zero fill): lane l clears the 16-byte chunk l % 8 of
         // rows r + l / 8
         const int ksteps = valid >= kBK ? kBK / kMmaK : (valid + kMmaK - 1) / kMmaK;
@@ -257,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
         if (valid < z1) {
           const int q = lane & 7;
           for (int col = 0; col < 2; ++col) {
-            uint8_t* atom = sB + stage * kBBytes + col * kAtom;
+            uint8_t* atom = sA + stage * kABytes + col * kAtom;
             for (int r = valid + (lane >> 3); r < z1; r += 4)
               *reinterpret_cast<uint4*>(atom + r * 128 + q * 16) = make_uint4(0u, 0u, 0u, 0u);
           }
@@ -271,9 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
             if (k >= ksteps) break;
             const uint32_t accum = (kb | k) ? 1u : 0u;
             const uint32_t koff = static_cast<uint32_t>(k) * kMmaK * 128;
-            const uint64_t bd = desc_mn_sw128(bbase + koff);
-            mma_bf16_ss(d0, desc_mn_sw128(abase + koff), bd, idesc, accum);
-            mma_bf16_ss(d0 + kN, desc_mn_sw128(abase + 2 * kAtom + koff), bd, idesc, accum);
+            mma_bf16_ss(d0, desc_mn_sw128(abase + koff), desc_mn_sw128(bbase + koff), idesc, accum);
           }
           mma_commit(&empty[stage]);
         }
@@ -301,14 +301,14 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
   } else {
     // -------------------------------------------------------------------- epilogue
     // Warp w reads TMEM lanes [32q, 32q+32), q = w % 4: thread l of lane l holds output row
-    // 32q + l of each chain, 32 consecutive fp32 columns per chunk. It writes that 128-byte
+    // 32q + l, 32 consecutive fp32 columns per chunk. It writes that 128-byte
     // row into the warp's staging buffer with the 128-byte swizzle (16-byte unit c of row r
     // at unit c ^ (r % 8): a quarter-warp's stores hit all 32 banks once) and lane 0 stores
     // the 32 x 32 chunk with one bulk tensor copy. Warps 2+q and 6+q take alternate chunks of
-    // the tile's 2 x kN/32; the next chunk's TMEM reads are issued before this chunk is
+    // the tile's kN/32; the next chunk's TMEM reads are issued before this chunk is
     // staged, and the buffer is rewritten only after the previous copy has read it.
     const int q = warp & 3, half = (warp - 2) >> 2;
-    constexpr int kChunks = 2 * (kN / 32);
+    constexpr int kChunks = kN / 32;
     const uint32_t stg = smem_addr(base + kOffStg + (warp - 2) * kStgBytes);
     int it = 0;
     RoleClock rc_loop, rc_acc;
@@ -332,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
       uint32_t v[32];
       auto load = [&](int idx) {
-        const uint32_t col = static_cast<uint32_t>((idx / (kN / 32)) * kN + (idx % (kN / 32)) * 32);
+        const uint32_t col = static_cast<uint32_t>(idx * 32);
         tmem_ld16(tb + col, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
         tmem_ld16(tb + col + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
       };
@@ -344,9 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
 #pragma unroll
         for (int j = 0; j < 32; ++j) r[j] = empty_group ? 0u : v[j];
         if (idx + 2 < kChunks) load(idx + 2);  // lands while this chunk is stored
-        const int ch = idx / (kN / 32);
-        const int row0 = t.m_blk * 2 * kFeat + ch * kFeat + q * 32;  // M and N are multiples of 64:
-        const int n = t.n_blk * kN + (idx % (kN / 32)) * 32;         // a chunk is all inside or all out
+        const int row0 = t.m_blk * kFeat + q * 32;  // M and N are multiples of 64:
+        const int n = t.n_blk * kN + idx * 32;      // a chunk is all inside or all out
         if (row0 < M && n < N) {
           if (lane == 0) bulk_wait_read_all();
           __syncwarp();

@@ -267,15 +267,15 @@ cudaError_t launch_grouped_gemm_bwd(int mode, const GemmBwdArgs& a, int grid, cu
 // The experts' weight gradients (gemm_dw_sm100.cu): per group g, out[g][i][j] =
 // sum_r A[r, i] B[r, j] over the group's rows r (routed group g: rows offsets[g] ..
 // offsets[g+1] of the slot order; shared group: rows 0 .. T). A and B are 3-D views
-// (64, rows, cols / 64) of [rows, cols] bf16 buffers, A with box (64, 64, 4), B with box
-// (64, 64, 2); an operand starts at atom column atom0 (+ g * step for shared group g).
+// (64, rows, cols / 64) of [rows, cols] bf16 buffers, A with box (64, 64, 2), B with box
+// (64, 64, 4); an operand starts at atom column atom0 (+ g * step for shared group g).
 struct GemmDwArgs {
   CUtensorMap a_routed, b_routed, a_shared, b_shared;
   int32_t a_atom0_routed, b_atom0_routed;
   int32_t a_atom0_shared, b_atom0_shared, a_atom_step_shared, b_atom_step_shared;
   const int32_t* offsets;  // [n_routed + 1]
   int32_t n_routed, n_shared, T;
-  int32_t m_tiles_routed, n_tiles_routed, m_tiles_shared, n_tiles_shared;  // 256-row x 128-col tiles
+  int32_t m_tiles_routed, n_tiles_routed, m_tiles_shared, n_tiles_shared;  // 128-row x 256-col tiles
   int32_t m_routed, n_routed_cols, m_shared, n_shared_cols;                // output [M, N] per group
   // fp32 outputs [groups, M, N] as 3-D maps (N, M, groups), box (32, 32, 1), 128-byte
   // swizzle: routed [n_routed, m_routed, n_routed_cols], shared [n_shared, m_shared, n_shared_cols]
