@@ -388,7 +388,8 @@ dsmoe_status dsmoe_ep_combine(dsmoe_handle* h, int32_t T, const void* x, const v
  *     dW_router fp32 [N', d] out dlogits^T x
  *   With N' a multiple of 64, d a multiple of 64, T >= 256, T >= 2 N' and all pointers
  *   16-byte aligned, both products run on the tensor cores: dlogits is split into bf16
- *   parts hi + lo (what remains is below 2^-16 of each value; the [hi | lo] rows overwrite
+ *   parts hi + lo (what remains is below 2^-16 of each value of magnitude below 3.39e38,
+ *   the largest finite bf16; the [hi | lo] rows overwrite
  *   the handle's "logits" workspace, which only the forward reads), dW_router = hi^T x +
  *   lo^T x on the weight-gradient GEMM (the two fp32 results held in dx's memory until
  *   they are added, hi first) and dx = [hi | lo] [W_router; W_router] on the input-
