@@ -442,7 +442,7 @@ dsmoe_status dsmoe_backward_gates(dsmoe_handle* h, int32_t T, const void* dh, co
  *   Grouped GEMMs on the tensor cores reducing over token rows (both operands MN-major,
  *   each routed expert's rows a ragged K range), fp32 accumulation of bf16 products.
  *   An expert no token picked gets a zero gradient. All nine pointers must be 16-byte
- *   aligned (the gradients are written by bulk tensor copies of 32 x 32 fp32 chunks);
+ *   aligned (the gradients are written by bulk tensor copies of 32 x 16 fp32 blocks);
  *   else DSMOE_ERR_INVALID_ARG.
  */
 dsmoe_status dsmoe_backward_weights(dsmoe_handle* h, int32_t T, const void* dh, const void* dY, const void* x,

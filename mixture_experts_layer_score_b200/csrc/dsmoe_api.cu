@@ -128,17 +128,17 @@ bool map_view_mn(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3D fp32 map (cols, rows, groups) of a [groups, rows, cols] tensor, 128-byte swizzle,
-// box (32, 32, 1): the weight-gradient GEMM's bulk stores of 32 x 32 chunks.
+// 3D fp32 map (cols, rows, groups) of a [groups, rows, cols] tensor, 64-byte swizzle,
+// box (16, 32, 1): the weight-gradient GEMM's bulk stores of 32-row x 16-column halves.
 bool map_out_f32(CUtensorMap* m, float* ptr, uint64_t rows, uint64_t cols, uint64_t groups) {
   auto enc = tensor_map_encoder();
   if (!enc || cols % 32 || rows % 32 || groups == 0) return false;
   cuuint64_t dims[3] = {cols, rows, groups};
   cuuint64_t strides[2] = {cols * 4, rows * cols * 4};
-  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t box[3] = {16, 32, 1};
   cuuint32_t es[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

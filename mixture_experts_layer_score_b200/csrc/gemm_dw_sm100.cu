@@ -10,9 +10,9 @@
 // expert's all T tokens.
 //
 // One CTA per SM, 320 threads: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
-// warps 2-9 epilogue (each stages 32 x 32 fp32 chunks of the accumulator in its own 4 KB of
-// shared memory and writes them to the output with bulk tensor stores, whole 128-byte
-// lines). A tile is 128 output rows by 256 output columns, one M=128, N=256 chain (per
+// warps 2-9 epilogue (each stages 32-row x 16-column fp32 halves of the accumulator in two
+// 2 KB buffers of its own shared memory and writes them to the output with bulk tensor
+// stores of whole 64-byte row segments). A tile is 128 output rows by 256 output columns, one M=128, N=256 chain (per
 // MAC it reads a quarter fewer shared-memory bytes than two M=128, N=128 chains, whose
 // operand reads alone fill the shared memory's bandwidth); per 64-row K block the
 // producer stages A (128 columns of the A buffer) and B (256 columns of the B buffer)
@@ -60,7 +60,7 @@ constexpr int kBufs = 2;
 constexpr uint32_t kAtom = kBK * 128;              // one 64-element atom column of a stage: 8 KB
 constexpr uint32_t kOffA = 0;
 constexpr uint32_t kOffB = kOffA + kStages * kABytes;
-constexpr uint32_t kStgBytes = 32 * 32 * 4;        // one warp's staged 32 x 32 fp32 chunk
+constexpr uint32_t kStgBytes = 32 * 32 * 4;        // one warp's two 32 x 16 fp32 staging buffers
 constexpr uint32_t kOffStg = kOffB + kStages * kBBytes;
 constexpr uint32_t kOffBars = kOffStg + kEpiWarps * kStgBytes;
 constexpr uint32_t kNumBars = 2 * kStages + 2 * kBufs + 1;
@@ -88,8 +88,8 @@ __device__ __forceinline__ void tma_load_3d_view(void* dst, const CUtensorMap* m
       : "memory");
 }
 
-// Bulk tensor store of one staged chunk: box (32 fp32 columns, 32 rows, 1 group) of a 3-D
-// map (columns, rows, groups) with the 128-byte swizzle; rows past a group's end are not
+// Bulk tensor store of one staged half: box (16 fp32 columns, 32 rows, 1 group) of a 3-D
+// map (columns, rows, groups) with the 64-byte swizzle; rows past a group's end are not
 // written (the map's row extent is the group's).
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int32_t col, int32_t row,
                                              int32_t group) {
@@ -99,7 +99,10 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t sr
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// every committed copy but the most recent one has finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_but_last() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 struct DwTile {
@@ -301,15 +304,17 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
   } else {
     // -------------------------------------------------------------------- epilogue
     // Warp w reads TMEM lanes [32q, 32q+32), q = w % 4: thread l of lane l holds output row
-    // 32q + l, 32 consecutive fp32 columns per chunk. It writes that 128-byte
-    // row into the warp's staging buffer with the 128-byte swizzle (16-byte unit c of row r
-    // at unit c ^ (r % 8): a quarter-warp's stores hit all 32 banks once) and lane 0 stores
-    // the 32 x 32 chunk with one bulk tensor copy. Warps 2+q and 6+q take alternate chunks of
-    // the tile's kN/32; the next chunk's TMEM reads are issued before this chunk is
-    // staged, and the buffer is rewritten only after the previous copy has read it.
+    // 32q + l, 32 consecutive fp32 columns per chunk. Each 16-column half of the chunk goes
+    // into one of the warp's two staging buffers (a quarter-warp's stores hit all 32 banks
+    // once) and lane 0 stores it with one bulk tensor copy, alternating buffers, so a
+    // buffer waits only for the copy before the last. Warps 2+q and 6+q take alternate
+    // chunks of the tile's kN/32; the next chunk's TMEM reads are issued before this chunk
+    // is staged. (One 4 KB buffer of whole 32-column chunks, each waiting for the previous
+    // copy, ran the V3 weight gradients 1.5% slower.)
     const int q = warp & 3, half = (warp - 2) >> 2;
     constexpr int kChunks = kN / 32;
     const uint32_t stg = smem_addr(base + kOffStg + (warp - 2) * kStgBytes);
+    uint32_t sc = 0;  // staged halves so far: the buffer of the next one is sc % 2
     int it = 0;
     RoleClock rc_loop, rc_acc;
     rc_loop.start();
@@ -347,18 +352,28 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_dw_kernel(const __grid_co
         const int row0 = t.m_blk * kFeat + q * 32;  // M and N are multiples of 64:
         const int n = t.n_blk * kN + idx * 32;      // a chunk is all inside or all out
         if (row0 < M && n < N) {
-          if (lane == 0) bulk_wait_read_all();
-          __syncwarp();
+          // two 16-column halves, each staged in one of the warp's two 2 KB buffers (64-byte
+          // rows, 64-byte swizzle: 16-byte unit c of row r at unit c ^ ((r / 2) % 4)) and
+          // stored by its own copy; a buffer is rewritten once the copy before the last has
+          // read it
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg + lane * 128 + ((c ^ (lane & 7)) << 4)),
-                         "r"(r[4 * c]), "r"(r[4 * c + 1]), "r"(r[4 * c + 2]), "r"(r[4 * c + 3])
-                         : "memory");
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_3d(omap, stg, n, row0, t.group);
-            bulk_commit();
+          for (int hf = 0; hf < 2; ++hf) {
+            const uint32_t buf = stg + (sc & 1u) * (kStgBytes / 2);
+            ++sc;
+            if (lane == 0) bulk_wait_read_but_last();
+            __syncwarp();
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(buf + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)),
+                           "r"(r[16 * hf + 4 * c]), "r"(r[16 * hf + 4 * c + 1]), "r"(r[16 * hf + 4 * c + 2]),
+                           "r"(r[16 * hf + 4 * c + 3])
+                           : "memory");
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(omap, buf, n + 16 * hf, row0, t.group);
+              bulk_commit();
+            }
           }
         }
         tmem_wait_ld();

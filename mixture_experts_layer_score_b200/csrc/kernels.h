@@ -277,7 +277,7 @@ struct GemmDwArgs {
   int32_t n_routed, n_shared, T;
   int32_t m_tiles_routed, n_tiles_routed, m_tiles_shared, n_tiles_shared;  // 128-row x 256-col tiles
   int32_t m_routed, n_routed_cols, m_shared, n_shared_cols;                // output [M, N] per group
-  // fp32 outputs [groups, M, N] as 3-D maps (N, M, groups), box (32, 32, 1), 128-byte
+  // fp32 outputs [groups, M, N] as 3-D maps (N, M, groups), box (16, 32, 1), 64-byte
   // swizzle: routed [n_routed, m_routed, n_routed_cols], shared [n_shared, m_shared, n_shared_cols]
   CUtensorMap out_map_routed, out_map_shared;
   uint32_t* status;
